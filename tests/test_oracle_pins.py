@@ -1,0 +1,297 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+closed forms, invariants, library routines, brute force on tiny inputs and an
+independent NumPy writing of the method.  CPU only."""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_30_b200 import synth
+from oracle import numpy_twin as twin
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# (T, H, W, tile, heads, d, topk) -- tiny grids, incl. ragged ones
+TINY = [
+    (2, 4, 4, (2, 2, 2), 2, 8, 2),
+    (4, 8, 8, (4, 4, 4), 2, 16, 2),
+    (5, 6, 7, (4, 4, 4), 2, 16, 3),
+    (4, 8, 8, (2, 2, 2), 1, 8, 5),
+    (3, 5, 9, (2, 2, 2), 2, 8, 7),
+]
+
+
+def _inputs(T, H, W, tile, heads, d, seed=0, B=1, amplitude=1.0):
+    return synth.make_qkv(B, heads, d, T, H, W, tile, amplitude, seed)
+
+
+def _f64(x):
+    return x.to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------------ tiling map
+
+def test_tile_map_matches_coordinate_formula(oracle_mod):
+    for T, H, W, tile, *_ in TINY:
+        slots = oracle_mod.tile_slots(T, H, W, tile)
+        cube, nt = twin.cube_of_token(T, H, W, tile)
+        assert slots.shape[0] == nt
+        valid = slots[slots >= 0]
+        # bijection onto the grid's tokens
+        assert np.array_equal(np.sort(valid), np.arange(T * H * W))
+        # every token sits in the cube the coordinate formula names
+        for j in range(nt):
+            toks = slots[j][slots[j] >= 0]
+            assert np.all(cube[toks] == j)
+
+
+def test_ragged_720p_tile_classes_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "ragged_720p_tile_classes.json")))
+    slots = oracle_mod.tile_slots(*g["grid"], tuple(g["tile"]))
+    assert slots.shape[0] == g["num_tiles"]
+    counts = (slots >= 0).sum(1)
+    hist = {str(c): int((counts == c).sum()) for c in np.unique(counts)}
+    assert hist == g["valid_count_histogram"]
+    assert counts.sum() == g["total_valid_tokens"]
+
+
+# ------------------------------------------------------------- gather/scatter
+
+@pytest.mark.parametrize("case", TINY)
+def test_gather_scatter_roundtrip_bit_exact(oracle_mod, case):
+    T, H, W, tile, heads, d, _ = case
+    q, _, _ = _inputs(T, H, W, tile, heads, d)
+    tiles = oracle_mod.gather(q, 1, heads, d, T, H, W, tile)
+    slots = oracle_mod.tile_slots(T, H, W, tile)
+    # padded slots are zero, valid slots carry the token's row
+    pad = slots < 0
+    assert np.all(tiles[:, :, pad] == 0)
+    back = oracle_mod.scatter(tiles, 1, heads, d, T, H, W, tile)
+    assert np.array_equal(back, oracle_mod.bits(q))
+
+
+# ------------------------------------------------------------------- pooling
+
+def test_pool_tile_constant_is_exact(oracle_mod):
+    """P6: a tile-constant input pools to that constant exactly (valid-count
+    division; dividing by the full tile volume would fail on ragged cubes)."""
+    T, H, W, tile, heads, d = 5, 6, 7, (4, 4, 4), 2, 4
+    cube, nt = twin.cube_of_token(T, H, W, tile)
+    vals = torch.arange(nt * heads * d, dtype=torch.float32).reshape(nt, heads, d) / 8 - 3
+    x = vals[torch.as_tensor(cube)].unsqueeze(0).to(torch.bfloat16)   # [1,N,heads,d]
+    p = oracle_mod.pool(x, 1, heads, d, T, H, W, tile)
+    expect = vals.permute(1, 0, 2).to(torch.bfloat16).to(torch.float64).numpy()[None]
+    assert np.array_equal(p, expect)
+
+
+# ------------------------------------------------------------------ selection
+
+@pytest.mark.parametrize("case", TINY)
+def test_select_matches_numpy_twin(oracle_mod, case):
+    T, H, W, tile, heads, d, k = case
+    q, kk, _ = _inputs(T, H, W, tile, heads, d, seed=3)
+    idx, sc = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile, with_scores=True)
+    tidx, tsc = twin.select(_f64(q), _f64(kk), T, H, W, tile, k)
+    np.testing.assert_allclose(sc, tsc, rtol=0, atol=1e-12)
+    assert np.array_equal(idx, tidx)
+    assert np.all(np.diff(idx, axis=-1) > 0)        # strictly ascending rows
+
+
+def test_topk_is_brute_force_best_subset(oracle_mod):
+    """P2: the kept set maximises the summed coarse score over all C(nt, k)
+    subsets (unique when scores have no ties)."""
+    T, H, W, tile, heads, d = 4, 8, 8, (2, 2, 2), 1, 8
+    q, kk, _ = _inputs(T, H, W, tile, heads, d, seed=11)
+    for k in (1, 2, 3):
+        idx, sc = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile, with_scores=True)
+        nt = sc.shape[-1]
+        for i in range(0, nt, 5):
+            row = sc[0, 0, i]
+            best = max(itertools.combinations(range(nt), k), key=lambda s: row[list(s)].sum())
+            assert tuple(idx[0, 0, i]) == tuple(sorted(best))
+
+
+def test_topk_ties_go_to_lower_tile_id(oracle_mod):
+    scores = np.zeros((1, 1, 6, 6))               # square: nt query x nt key tiles
+    scores[0, 0, 0] = [1, 5, 5, 5, 0, 5]          # four-way tie for the top
+    scores[0, 0, 1] = [2, 2, 2, 2, 2, 2]          # all equal
+    scores[0, 0, 2] = [-1, -2, -3, -4, -5, -6]
+    scores[0, 0, 3] = [0, 0, 0, 0, 0, 9]
+    idx = oracle_mod.topk(scores, 2)
+    assert idx[0, 0, :4].tolist() == [[1, 2], [0, 1], [0, 1], [0, 5]]
+
+
+def test_coarse_probs_are_row_softmax(oracle_mod):
+    rng = np.random.default_rng(0)
+    qp, kp = rng.normal(size=(1, 2, 7, 16)), rng.normal(size=(1, 2, 7, 16))
+    sc, pr = oracle_mod.coarse(qp, kp, with_probs=True)
+    ref = torch.softmax(torch.from_numpy(qp @ kp.transpose(0, 1, 3, 2) / 4.0), -1).numpy()
+    np.testing.assert_allclose(pr, ref, atol=1e-14)
+    np.testing.assert_allclose(sc, qp @ kp.transpose(0, 1, 3, 2) / 4.0, atol=1e-13)
+
+
+# ------------------------------------------------------------------ fine pass
+
+@pytest.mark.parametrize("case", TINY)
+def test_fine_matches_masked_dense_attention(oracle_mod, case):
+    """P2 (fine half): equals dense attention under an explicit N x N block mask."""
+    T, H, W, tile, heads, d, k = case
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=5)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    ref, _ = twin.masked_attention(_f64(q), _f64(kk), _f64(v),
+                                   twin.block_mask(idx, T, H, W, tile))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", [(4, 8, 8, (4, 4, 4), 2, 16), (5, 6, 7, (4, 4, 4), 3, 8)])
+def test_all_tiles_equals_dense_sdpa(oracle_mod, case):
+    """P1: k = nt reduces to dense softmax attention (torch SDPA, fp64 CPU)."""
+    T, H, W, tile, heads, d = case
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=7, amplitude=0.7)
+    nt = oracle_mod.num_tiles(T, H, W, tile)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, nt, tile)
+    assert np.array_equal(idx[0, 0, 0], np.arange(nt))
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    tq, tk, tv = (x.to(torch.float64).permute(0, 2, 1, 3) for x in (q, kk, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+    dense = oracle_mod.dense(q, kk, v, 1, heads, d, T * H * W)
+    np.testing.assert_allclose(dense, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_weights_sum_to_one_and_vanish_off_selection(oracle_mod):
+    """P3: each query's weights sum to one, are zero outside the kept tiles
+    (and hence on padded slots), and reproduce the fine output."""
+    T, H, W, tile, heads, d, k = 5, 6, 7, (4, 4, 4), 2, 16, 3
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=9)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    cube, _ = twin.cube_of_token(T, H, W, tile)
+    for head in range(heads):
+        for n in (0, 17, 101, T * H * W - 1):
+            w = oracle_mod.weights(q, kk, idx, 0, head, n, 1, heads, d, T, H, W, tile)
+            assert abs(w.sum() - 1.0) < 1e-12
+            kept = np.isin(cube, idx[0, head, cube[n]])
+            assert np.all(w[~kept] == 0) and np.all(w[kept] > 0)
+            np.testing.assert_allclose(w @ _f64(v)[0, :, head], out[0, n, head], atol=1e-12)
+
+
+def test_permutation_invariance(oracle_mod):
+    """P5: the order of a row's indices, and the order of tokens inside a key
+    tile, do not change the output."""
+    T, H, W, tile, heads, d, k = 4, 8, 8, (2, 2, 2), 2, 8, 4
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=13)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    rng = np.random.default_rng(1)
+    shuffled = np.take_along_axis(idx, rng.permuted(np.broadcast_to(np.arange(k), idx.shape).copy(), axis=-1), -1)
+    out2 = oracle_mod.fine(q, kk, v, shuffled, 1, heads, d, T, H, W, tile)
+    np.testing.assert_allclose(out, out2, rtol=0, atol=1e-12)
+    # swap two tokens of one cube in k and v: cube membership is unchanged
+    cube, _ = twin.cube_of_token(T, H, W, tile)
+    a, b = np.nonzero(cube == 3)[0][:2]
+    k2, v2 = kk.clone(), v.clone()
+    k2[:, [a, b]] = kk[:, [b, a]]
+    v2[:, [a, b]] = v[:, [b, a]]
+    out3 = oracle_mod.fine(q, k2, v2, idx, 1, heads, d, T, H, W, tile)
+    np.testing.assert_allclose(out, out3, rtol=0, atol=1e-12)
+
+
+def test_topk_one_is_single_tile_softmax(oracle_mod):
+    """P6: with k = 1 each query attends one tile: an explicit small softmax."""
+    T, H, W, tile, heads, d = 4, 8, 8, (4, 4, 4), 1, 16
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=2)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, 1, tile)
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    cube, _ = twin.cube_of_token(T, H, W, tile)
+    qf, kf, vf = _f64(q)[0, :, 0], _f64(kk)[0, :, 0], _f64(v)[0, :, 0]
+    for n in (0, 63, 200):
+        keys = np.nonzero(cube == idx[0, 0, cube[n], 0])[0]
+        s = kf[keys] @ qf[n] / 4.0
+        p = np.exp(s - s.max()); p /= p.sum()
+        np.testing.assert_allclose(out[0, n, 0], p @ vf[keys], atol=1e-12)
+
+
+def test_fine_tiles_sample_matches_full(oracle_mod):
+    T, H, W, tile, heads, d, k = 5, 6, 7, (4, 4, 4), 2, 16, 3
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=4)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    out = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    nt = oracle_mod.num_tiles(T, H, W, tile)
+    rows = np.array([0, nt - 1, nt + 3])
+    part = oracle_mod.fine_tiles(q, kk, v, idx, rows, 1, heads, d, T, H, W, tile)
+    slots = oracle_mod.tile_slots(T, H, W, tile)
+    for r, row in enumerate(rows):
+        head, i = divmod(int(row), nt)
+        for s, n in enumerate(slots[i]):
+            if n >= 0:
+                assert np.array_equal(part[r, s], out[0, n, head])
+            else:
+                assert np.all(part[r, s] == 0)
+
+
+# -------------------------------------------------------------- linear branch
+
+def test_linear_zero_keys_gives_mean_value(oracle_mod):
+    """P7: K = 0 makes phi(k) = 1, so every query's linear output is the mean
+    of V over all tokens."""
+    B, heads, d, T, H, W = 1, 2, 8, 3, 4, 5
+    q, _, v = _inputs(T, H, W, (4, 4, 4), heads, d, seed=6)
+    kk = torch.zeros_like(q)
+    N = T * H * W
+    S, z = oracle_mod.linear_state(kk, v, B, heads, d, N)
+    lin = oracle_mod.linear_apply(q, S, z, B, heads, d, N)
+    mean_v = _f64(v).mean(axis=1)                     # [B, heads, d]
+    np.testing.assert_allclose(lin, np.broadcast_to(mean_v[:, None], lin.shape), atol=1e-12)
+
+
+def test_linear_state_form_matches_quadratic_form(oracle_mod):
+    B, heads, d, T, H, W = 1, 2, 8, 3, 4, 5
+    q, kk, v = _inputs(T, H, W, (4, 4, 4), heads, d, seed=8)
+    N = T * H * W
+    S, z = oracle_mod.linear_state(kk, v, B, heads, d, N)
+    lin = oracle_mod.linear_apply(q, S, z, B, heads, d, N)
+    ref = twin.linear_branch(_f64(q), _f64(kk), _f64(v))
+    np.testing.assert_allclose(lin, ref, rtol=1e-12, atol=1e-12)
+    # phi is elu + 1 (torch's elu is an independent library routine)
+    x = torch.linspace(-5, 5, 101, dtype=torch.float64)
+    np.testing.assert_allclose(twin.phi(x.numpy()), (torch.nn.functional.elu(x) + 1).numpy(),
+                               atol=1e-15)
+
+
+def test_linear_state_matches_torch_einsum(oracle_mod):
+    B, heads, d, T, H, W = 1, 3, 8, 2, 4, 4
+    _, kk, v = _inputs(T, H, W, (4, 4, 4), heads, d, seed=10)
+    S, z = oracle_mod.linear_state(kk, v, B, heads, d, T * H * W)
+    pk = torch.nn.functional.elu(kk.to(torch.float64)) + 1
+    Sref = torch.einsum("bnha,bnhc->bhac", pk, v.to(torch.float64))
+    np.testing.assert_allclose(S, Sref.numpy(), rtol=1e-12)
+    np.testing.assert_allclose(z, pk.sum(1).numpy(), rtol=1e-12)
+
+
+def test_whole_path_matches_numpy_twin(oracle_mod):
+    T, H, W, tile, heads, d, k = 5, 6, 7, (4, 4, 4), 2, 16, 3
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=12)
+    out, idx = oracle_mod.forward(q, kk, v, 1, heads, d, T, H, W, k, tile, linear=True)
+    ref, tidx = twin.forward(_f64(q), _f64(kk), _f64(v), T, H, W, tile, k, linear=True)
+    assert np.array_equal(idx, tidx)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+# ------------------------------------------------------------------ precision
+
+def test_fp32_oracle_far_inside_tolerance(oracle_mod):
+    """P8: the same oracle in fp32 differs from fp64 by far less than the
+    fine-pass tolerance (max-abs 2e-2, relative Frobenius 1e-2)."""
+    T, H, W, tile, heads, d, k = 4, 16, 16, (4, 4, 4), 2, 64, 4
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=1)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    o64 = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    o32 = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile, precision="f32")
+    err = np.abs(o64 - o32).max()
+    rel = np.linalg.norm(o64 - o32) / np.linalg.norm(o64)
+    assert err < 1e-4 and rel < 1e-5
