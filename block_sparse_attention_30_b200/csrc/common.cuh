@@ -1,0 +1,78 @@
+// common.cuh -- shared definitions of the CUDA library: tile geometry,
+// device status word, small math helpers.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace vsa {
+
+// Bits of the device status word (first int of the workspace).
+enum : int {
+    kStatusTimeout = 1,      // a bounded wait gave up
+    kStatusBadIndex = 2,     // a block index outside [0, nt)
+    kStatusMisaligned = 4,   // shared memory not aligned as the kernel needs
+};
+
+// Geometry of the cube tiling of a T x H x W token grid.
+struct Grid {
+    int B, heads, d;
+    int T, H, W;
+    int tt, th, tw;
+    int nT, nh, nw, nt;
+    long long N;
+};
+
+__host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+inline Grid make_grid(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
+    Grid g;
+    g.B = B; g.heads = heads; g.d = d;
+    g.T = T; g.H = H; g.W = W;
+    g.tt = tt; g.th = th; g.tw = tw;
+    g.nT = ceil_div_i(T, tt); g.nh = ceil_div_i(H, th); g.nw = ceil_div_i(W, tw);
+    g.nt = g.nT * g.nh * g.nw;
+    g.N = (long long)T * H * W;
+    return g;
+}
+
+// Cube j -> its first (t, h, w) coordinates and its valid extents.
+struct TileCoord {
+    int t0, h0, w0;      // origin in the grid
+    int vt, vh, vw;      // number of valid layers along each axis
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const Grid& g, int j) {
+    TileCoord c;
+    const int it = j / (g.nh * g.nw);
+    const int ih = (j / g.nw) % g.nh;
+    const int iw = j % g.nw;
+    c.t0 = it * g.tt; c.h0 = ih * g.th; c.w0 = iw * g.tw;
+    c.vt = min(g.tt, g.T - c.t0);
+    c.vh = min(g.th, g.H - c.h0);
+    c.vw = min(g.tw, g.W - c.w0);
+    return c;
+}
+
+// 64-bit mask of the valid slots of a cube (slot s = (dt*th + dh)*tw + dw).
+__device__ __forceinline__ uint64_t valid_slot_mask(const Grid& g, const TileCoord& c) {
+    if (c.vt == g.tt && c.vh == g.th && c.vw == g.tw) return ~0ull;
+    uint64_t m = 0;
+    for (int s = 0; s < 64; ++s) {
+        const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
+        if (dt < c.vt && dh < c.vh && dw < c.vw) m |= 1ull << s;
+    }
+    return m;
+}
+
+__device__ __forceinline__ void report(int* status, int bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// 2^x on the MUFU unit (hardware approximation, ~2 ulp).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+}  // namespace vsa

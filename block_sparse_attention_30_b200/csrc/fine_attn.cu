@@ -1,0 +1,445 @@
+// fine_attn.cu -- the fine pass of block-sparse video attention on sm_100a.
+//
+// Source of the operation: "FastVideo 稀疏蒸馏技术深度解析" (omica.com.cn),
+// section "2. 视频稀疏注意力VSA": only the attention weights of the selected
+// key blocks are evaluated, exactly and Flash-Attention style.  Here a query
+// block is one 64-token cube tile and every kept key block is a cube tile.
+//
+// One CTA owns one query cube (b, head, i) and runs online softmax over its
+// top-k key cubes, two cubes (128 keys) per step:
+//   * warp 4 (one lane) loads Q once and the K / V cube pairs into shared
+//     memory rings with 5-D TMA boxes cut straight from the [B][N][heads][d]
+//     tensors (box = d-chunk x tw x th x tt), so the cube gather costs no
+//     extra pass and ragged edge cubes arrive zero-filled;
+//   * warp 5 (one lane) issues the tensor-core work: S = Q K^T (M=64 queries,
+//     N=128 keys, A and B from shared memory) into TMEM, then, once softmax
+//     has written P as bf16 over S in TMEM, O += P V (A = P from TMEM,
+//     B = V from shared memory, MN-major);
+//   * warps 0-3 (one TMEM sub-partition each; rows 16w..16w+15, each row
+//     split in two 64-column halves over lanes t and t+16) do the fp32 online
+//     softmax in the exp2 domain, rescale O in TMEM only when a row maximum
+//     grows by more than 2^8, and finally write O / l as bf16 in grid order
+//     (the cube scatter, fused), skipping padded slots.
+// Two CTAs share an SM (256 TMEM columns and ~112 KB of shared memory each),
+// so one CTA's softmax overlaps the other's MMAs.
+//
+// Every wait is bounded; on a timeout the CTA records kStatusTimeout in the
+// status word, drains its own copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "fine_attn.h"
+#include "sm100.cuh"
+
+namespace vsa {
+using namespace sm100;
+
+template <int D>
+struct FineCfg {
+    static constexpr int NCH = D / 64;                 // 64-element (128-byte) d chunks
+    static constexpr int Q_BYTES = 64 * D * 2;         // one query cube
+    static constexpr int CUBE_BYTES = 64 * D * 2;      // one key cube (K or V)
+    static constexpr int PAIR_BYTES = 2 * CUBE_BYTES;  // two key cubes
+    static constexpr int CHUNK_STRIDE = 128 * 128;     // bytes between d chunks of a pair
+    static constexpr int NK = (D == 128) ? 2 : 3;      // K pair stages
+    static constexpr int NV = (D == 128) ? 1 : 3;      // V pair stages
+    static constexpr int TMEM_COLS = 256;
+    static constexpr int O_COL = 0;                    // fp32 O, D columns
+    static constexpr int S_COL = 128;                  // fp32 S (128 cols) / bf16 P (64 cols)
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = Q_BYTES + (NK + NV) * PAIR_BYTES + BAR_BYTES;
+};
+
+template <int D>
+struct FineBars {
+    uint64_t q_full;
+    uint64_t k_full[FineCfg<D>::NK], k_empty[FineCfg<D>::NK];
+    uint64_t v_full[FineCfg<D>::NV], v_empty[FineCfg<D>::NV];
+    uint64_t s_full, p_full, o_ready, mma_done, lin_ready, lin_done;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(FineBars<128>) <= FineCfg<128>::BAR_BYTES, "barrier block");
+static_assert(sizeof(FineBars<64>) <= FineCfg<64>::BAR_BYTES, "barrier block");
+
+__device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) return false;
+    return true;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 2)
+fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 const __grid_constant__ CUtensorMap mv, const Grid g,
+                 const int32_t* __restrict__ block_idx, const int topk, const float scale_log2,
+                 const float* __restrict__ lin_S, const float* __restrict__ lin_z,
+                 __nv_bfloat16* __restrict__ out, int* status) {
+    using C = FineCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
+        if (threadIdx.x == 0) report(status, kStatusMisaligned);
+        return;
+    }
+    uint8_t* sQ = smem;
+    uint8_t* sK = smem + C::Q_BYTES;
+    uint8_t* sV = sK + C::NK * C::PAIR_BYTES;
+    FineBars<D>* bars = reinterpret_cast<FineBars<D>*>(sV + C::NV * C::PAIR_BYTES);
+    volatile int* abort_flag = &bars->abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long row_id = blockIdx.x;                 // (b*heads + head)*nt + i
+    const int i = (int)(row_id % g.nt);
+    const int bh = (int)(row_id / g.nt);
+    const int head = bh % g.heads, b = bh / g.heads;
+    const int32_t* my_idx = block_idx + row_id * topk;
+    const int n_pairs = (topk + 1) >> 1;
+    const bool lin = lin_S != nullptr && lin_z != nullptr;
+    // Linear-branch operands reuse the K/V rings once the last PV is done:
+    //   phi(Q) hi / lo  (A, K-major like Q)        at sK, sK + Q_BYTES
+    //   S hi / lo       (B, MN-major like V pairs) at sK + 2*Q_BYTES, + D*D*2
+    uint8_t* sPhiHi = sK;
+    uint8_t* sPhiLo = sK + C::Q_BYTES;
+    uint8_t* sSHi = sK + 2 * C::Q_BYTES;
+    uint8_t* sSLo = sSHi + D * D * 2;
+
+    if (tid == 0) {
+        bars->abort = 0;
+        mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < C::NK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
+        for (int s = 0; s < C::NV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->o_ready, 1);
+        mbar_init(&bars->mma_done, 1);
+        mbar_init(&bars->lin_ready, 128);
+        mbar_init(&bars->lin_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+    if (warp == 4 && lane == 0) { tma_prefetch_desc(&mq); tma_prefetch_desc(&mk); tma_prefetch_desc(&mv); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = bars->tmem_base;
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        report(status, kStatusTimeout);
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int k_issued = 0, v_issued = 0;
+            const TileCoord qc = tile_coord(g, i);
+            mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+            for (int c = 0; c < C::NCH; ++c)
+                tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + 64 * c, qc.w0, qc.h0, qc.t0, b);
+            for (int p = 0; p < n_pairs; ++p) {
+                const int ntl = min(2, topk - 2 * p);
+                int jt[2] = {0, 0};
+                for (int t = 0; t < ntl; ++t) {
+                    int j = __ldg(my_idx + 2 * p + t);
+                    if (j < 0 || j >= g.nt) { report(status, kStatusBadIndex); j = 0; }
+                    jt[t] = j;
+                }
+                const int sk = p % C::NK;
+                if (p >= C::NK && !mbar_wait(&bars->k_empty[sk], ((p / C::NK) - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&bars->k_full[sk], ntl * C::CUBE_BYTES);
+                for (int t = 0; t < ntl; ++t) {
+                    const TileCoord kc = tile_coord(g, jt[t]);
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_5d(sK + sk * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, &mk,
+                                    &bars->k_full[sk], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
+                }
+                ++k_issued;
+                const int sv = p % C::NV;
+                if (p >= C::NV && !mbar_wait(&bars->v_empty[sv], ((p / C::NV) - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&bars->v_full[sv], ntl * C::CUBE_BYTES);
+                for (int t = 0; t < ntl; ++t) {
+                    const TileCoord kc = tile_coord(g, jt[t]);
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_5d(sV + sv * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, &mv,
+                                    &bars->v_full[sv], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
+                }
+                ++v_issued;
+            }
+            if (*abort_flag) {
+                // drain: the last load issued into each stage must land before exit
+                wait_noabort(&bars->q_full, 0);
+                for (int n = max(0, k_issued - C::NK); n < k_issued; ++n)
+                    wait_noabort(&bars->k_full[n % C::NK], (n / C::NK) & 1);
+                for (int n = max(0, v_issued - C::NV); n < v_issued; ++n)
+                    wait_noabort(&bars->v_full[n % C::NV], (n / C::NV) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------- MMA
+        if (lane == 0) {
+            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            const uint32_t tS = tbase + C::S_COL, tO = tbase + C::O_COL;
+            const uint32_t id_pv = idesc_bf16_f32(64, D, false, true);
+            bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
+            for (int p = 0; ok && p < n_pairs; ++p) {
+                const int nkeys = min(2, topk - 2 * p) * 64;
+                const int sk = p % C::NK, sv = p % C::NV;
+                if (!mbar_wait(&bars->k_full[sk], (p / C::NK) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(k_addr + sk * C::PAIR_BYTES + (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32, 16, 1024);
+                    mma_bf16_ss(tS, a, bd, id_s, kk > 0);
+                }
+                mma_commit(&bars->s_full);
+                mma_commit(&bars->k_empty[sk]);
+                if (!mbar_wait(&bars->p_full, p & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&bars->v_full[sv], (p / C::NV) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kk = 0; kk < nkeys / 16; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(v_addr + sv * C::PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
+                    mma_bf16_ts(tO, tS + kk * 8, bd, id_pv, (p > 0 || kk > 0));
+                }
+                mma_commit(&bars->o_ready);
+                mma_commit(&bars->v_empty[sv]);
+            }
+            if (ok && lin) {
+                // Lin = phi(Q) S with S and phi(Q) split into bf16 hi + lo parts:
+                // hi*hi + hi*lo + lo*hi, fp32 accumulation in the S columns.
+                if (mbar_wait(&bars->lin_ready, 0, abort_flag)) {
+                    tc_fence_after();
+                    const uint32_t id_lin = idesc_bf16_f32(64, D, false, true);
+                    const uint32_t a_hi = smem_u32(sPhiHi), a_lo = smem_u32(sPhiLo);
+                    const uint32_t b_hi = smem_u32(sSHi), b_lo = smem_u32(sSLo);
+                    for (int pass = 0; pass < 3; ++pass) {
+                        const uint32_t aa = pass == 2 ? a_lo : a_hi;
+                        const uint32_t bb = pass == 1 ? b_lo : b_hi;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t a = smem_desc_sw128(aa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(bb + kk * 2048, D * 128, 1024);
+                            mma_bf16_ss(tS, a, bd, id_lin, (pass > 0 || kk > 0));
+                        }
+                    }
+                    mma_commit(&bars->lin_done);
+                } else {
+                    ok = false;
+                }
+            }
+            if (!ok) fail();
+            mma_commit(&bars->mma_done);
+            wait_noabort(&bars->mma_done, 0);
+        }
+    } else {
+        // --------------------------------------------------- softmax / epilogue
+        const int r = 16 * warp + (lane & 15), hf = lane >> 4;
+        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const uint32_t tS = tbase + lane_base + C::S_COL, tO = tbase + lane_base + C::O_COL;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int p = 0; p < n_pairs; ++p) {
+            const int ntl = min(2, topk - 2 * p);
+            uint64_t vmask = 0;
+            if (hf < ntl) {
+                int j = __ldg(my_idx + 2 * p + hf);
+                if (j < 0 || j >= g.nt) j = 0;
+                vmask = valid_slot_mask(g, tile_coord(g, j));
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, p & 1, abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            float s[64];
+            tmem_ld_16x32bx2_x16<64>(tS + 0, *reinterpret_cast<float(*)[16]>(&s[0]));
+            tmem_ld_16x32bx2_x16<64>(tS + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+            tmem_ld_16x32bx2_x16<64>(tS + 32, *reinterpret_cast<float(*)[16]>(&s[32]));
+            tmem_ld_16x32bx2_x16<64>(tS + 48, *reinterpret_cast<float(*)[16]>(&s[48]));
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                s[c] = ((vmask >> c) & 1ull) ? s[c] * scale_log2 : -INFINITY;
+                mx = fmaxf(mx, s[c]);
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const bool resc = mx > m_run + 8.f;
+            const float m_new = resc ? mx : m_run;
+            const float alpha = resc ? ex2(m_run - m_new) : 1.f;
+            m_run = m_new;
+            float ls = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float p0 = ex2(s[2 * c] - m_new), p1 = ex2(s[2 * c + 1] - m_new);
+                pk[c] = pack_bf16x2(p0, p1);
+                // normalise by the weights the tensor core will actually use
+                // (bf16-rounded), so O / l is an exactly normalised average
+                ls += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+            }
+            l_run = l_run * alpha + ls;
+            tmem_st_16x32bx2_x32(tS, pk);
+            if (p > 0 && __any_sync(0xffffffffu, resc)) {
+                // O holds PV up to pair p-1: wait for it, then rescale in place
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, (p - 1) & 1, abort_flag))) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                    float o[16];
+                    tmem_ld_16x32bx2_x16<D / 2>(tO + c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] *= alpha;
+                    tmem_st_16x32bx2_x16<D / 2>(tO + c0, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+        }
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, (n_pairs - 1) & 1, abort_flag))) ok = false;
+        // ------------------------------------------------------- linear branch
+        // phi(q) = elu(q) + 1 (SparkDiffusion RoLA / TurboDiffusion SLA linear
+        // branch).  Each thread owns half a query row: D/2 features.
+        float den = 1.f;
+        if (ok && lin) {
+            tc_fence_after();
+            const float* zb = lin_z + (long long)bh * D + hf * (D / 2);
+            const float* Sb = lin_S + (long long)bh * D * D;
+            float dpart = 0.f;
+            // phi(Q) hi/lo: this thread's D/2 features sit in chunk (hf*(D/2))/64
+            // of the Q cube, 16-byte units u0 .. u0 + D/16 - 1 of row r.
+            const int chunk = (hf * (D / 2)) / 64, u0 = ((hf * (D / 2)) % 64) / 8;
+#pragma unroll
+            for (int u = 0; u < D / 16; ++u) {
+                const int uu = u0 + u;
+                const uint32_t off = chunk * 8192 + r * 128 + (((uu) ^ (r & 7)) << 4);
+                const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float q0 = __uint_as_float(w[e] << 16), q1 = __uint_as_float(w[e] & 0xffff0000u);
+                    const float f0 = q0 > 0.f ? q0 + 1.f : __expf(q0);
+                    const float f1 = q1 > 0.f ? q1 + 1.f : __expf(q1);
+                    dpart += f0 * __ldg(zb + u * 8 + 2 * e) + f1 * __ldg(zb + u * 8 + 2 * e + 1);
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+                    const float2 hf2 = __bfloat1622float2(h);
+                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    lo[e] = pack_bf16x2(f0 - hf2.x, f1 - hf2.y);
+                }
+                *reinterpret_cast<uint4*>(sPhiHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sPhiLo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            den = dpart + __shfl_xor_sync(0xffffffffu, dpart, 16);
+            // S hi/lo (B operand, MN-major): row a = input feature, 64-wide
+            // chunks of output features c, 128-byte rows, 128-byte swizzle.
+            for (int unit = tid; unit < D * D / 8; unit += 128) {
+                const int a = unit / (D / 8), cu = unit % (D / 8);      // cu: 8-wide group of c
+                const int ch = cu / 8, uu = cu % 8;
+                const float4 x0 = __ldg(reinterpret_cast<const float4*>(Sb + a * D + cu * 8));
+                const float4 x1 = __ldg(reinterpret_cast<const float4*>(Sb + a * D + cu * 8 + 4));
+                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(xs[2 * e], xs[2 * e + 1]);
+                    const float2 hf2 = __bfloat1622float2(h);
+                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    lo[e] = pack_bf16x2(xs[2 * e] - hf2.x, xs[2 * e + 1] - hf2.y);
+                }
+                const uint32_t off = ch * (D * 128) + a * 128 + ((uu ^ (a & 7)) << 4);
+                *reinterpret_cast<uint4*>(sSHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sSLo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->lin_ready);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->lin_done, 0, abort_flag))) ok = false;
+        }
+        if (!ok) fail();
+        // ------------------------------------------------------------ epilogue
+        if (ok) {
+            tc_fence_after();
+            const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+            const float inv = 1.f / l;
+            const float inv_den = 1.f / den;
+            const TileCoord qc = tile_coord(g, i);
+            const int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
+            const bool valid = dt < qc.vt && dh < qc.vh && dw < qc.vw;
+            const long long n = ((long long)(qc.t0 + dt) * g.H + (qc.h0 + dh)) * g.W + (qc.w0 + dw);
+            __nv_bfloat16* orow = out + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
+#pragma unroll
+            for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                float o[16];
+                tmem_ld_16x32bx2_x16<D / 2>(tO + c0, o);
+                if (lin) {
+                    float li[16];
+                    tmem_ld_16x32bx2_x16<D / 2>(tS + c0, li);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = o[e] * inv + li[e] * inv_den;
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] *= inv;
+                }
+                uint4 w0, w1;
+                w0.x = pack_bf16x2(o[0], o[1]);
+                w0.y = pack_bf16x2(o[2], o[3]);
+                w0.z = pack_bf16x2(o[4], o[5]);
+                w0.w = pack_bf16x2(o[6], o[7]);
+                w1.x = pack_bf16x2(o[8], o[9]);
+                w1.y = pack_bf16x2(o[10], o[11]);
+                w1.z = pack_bf16x2(o[12], o[13]);
+                w1.w = pack_bf16x2(o[14], o[15]);
+                if (valid) {
+                    reinterpret_cast<uint4*>(orow + c0)[0] = w0;
+                    reinterpret_cast<uint4*>(orow + c0)[1] = w1;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int D>
+static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
+    using C = FineCfg<D>;
+    static int configured_device = -1;   // per process: attribute set once per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(fine_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    const long long rows = (long long)a.g.B * a.g.heads * a.g.nt;
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    fine_attn_kernel<D><<<(unsigned)rows, 192, C::SMEM_BYTES, stream>>>(
+        *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, a.lin_S, a.lin_z,
+        reinterpret_cast<__nv_bfloat16*>(a.out), a.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) {
+    if (a.g.d == 128) return launch_fine_impl<128>(a, stream);
+    return launch_fine_impl<64>(a, stream);
+}
+
+int fine_smem_bytes(int d) { return d == 128 ? FineCfg<128>::SMEM_BYTES : FineCfg<64>::SMEM_BYTES; }
+
+}  // namespace vsa

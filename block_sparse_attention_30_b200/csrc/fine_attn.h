@@ -1,0 +1,27 @@
+// fine_attn.h -- internal launch interface of the fine-pass kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace vsa {
+
+struct FineArgs {
+    Grid g;
+    const CUtensorMap* mq;       // 5-D maps over q, k, v (see api.cu)
+    const CUtensorMap* mk;
+    const CUtensorMap* mv;
+    const int32_t* block_idx;    // [B][heads][nt][topk]
+    int topk;
+    const float* lin_S;          // optional linear-branch state [B][heads][d][d]
+    const float* lin_z;          // optional [B][heads][d]
+    void* out;                   // bf16 [B][N][heads][d]
+    int* status;                 // device status word
+};
+
+cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream);
+int fine_smem_bytes(int d);
+
+}  // namespace vsa

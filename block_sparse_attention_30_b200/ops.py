@@ -1,0 +1,131 @@
+"""Python front-end with the C ABI's names: torch tensors in, kernel launches
+out.  PyTorch supplies device memory and the current stream; each function
+only checks dtypes/shapes and forwards raw pointers to libvsa.so.
+"""
+import torch
+
+from . import _lib
+
+_SENTINEL = object()
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _shape(B, heads, head_dim, T, H, W, tile):
+    tt, th, tw = tile
+    return [B, heads, head_dim, T, H, W, tt, th, tw]
+
+
+def _grid_of(x, T, H, W):
+    assert x.dim() == 4 and x.is_contiguous(), "expected a contiguous [B, N, heads, d] tensor"
+    B, N, heads, d = x.shape
+    assert N == T * H * W, f"N={N} does not match grid {T}x{H}x{W}"
+    return B, heads, d
+
+
+def vsa_status_string(code: int) -> str:
+    return _lib.lib().vsa_status_string(code).decode()
+
+
+def vsa_num_tiles(T, H, W, tile=(4, 4, 4)) -> int:
+    return _lib.lib().vsa_num_tiles(T, H, W, *tile)
+
+
+def vsa_workspace_bytes(B, heads, head_dim, T, H, W, topk, tile=(4, 4, 4)) -> int:
+    return _lib.lib().vsa_workspace_bytes(*_shape(B, heads, head_dim, T, H, W, tile), topk)
+
+
+def new_workspace(B, heads, head_dim, T, H, W, topk, tile=(4, 4, 4), device="cuda", stream=None):
+    """Allocate (torch) and initialise a workspace for these shapes."""
+    n = vsa_workspace_bytes(B, heads, head_dim, T, H, W, topk, tile)
+    if n == 0:
+        raise _lib.VSAError("vsa_workspace_bytes", 1)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _lib.check("vsa_workspace_init", _lib.lib().vsa_workspace_init(ws.data_ptr(), n, _stream(stream)))
+    return ws
+
+
+def vsa_gather_tiles(x, x_tiles, T, H, W, tile=(4, 4, 4), stream=None):
+    B, heads, d = _grid_of(x, T, H, W)
+    _lib.check("vsa_gather_tiles", _lib.lib().vsa_gather_tiles(
+        x.data_ptr(), x_tiles.data_ptr(), *_shape(B, heads, d, T, H, W, tile), _stream(stream)))
+
+
+def vsa_scatter_tiles(x_tiles, x, T, H, W, tile=(4, 4, 4), stream=None):
+    B, heads, d = _grid_of(x, T, H, W)
+    _lib.check("vsa_scatter_tiles", _lib.lib().vsa_scatter_tiles(
+        x_tiles.data_ptr(), x.data_ptr(), *_shape(B, heads, d, T, H, W, tile), _stream(stream)))
+
+
+def vsa_select_blocks(q, k, T, H, W, topk, block_idx, workspace, tile=(4, 4, 4), stream=None):
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_select_blocks", _lib.lib().vsa_select_blocks(
+        q.data_ptr(), k.data_ptr(), *_shape(B, heads, d, T, H, W, tile), topk,
+        block_idx.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def vsa_linear_branch_fwd(k, v, lin_S, lin_z, T, H, W, stream=None):
+    B, heads, d = _grid_of(k, T, H, W)
+    _lib.check("vsa_linear_branch_fwd", _lib.lib().vsa_linear_branch_fwd(
+        k.data_ptr(), v.data_ptr(), lin_S.data_ptr(), lin_z.data_ptr(), B, heads, d, T, H, W,
+        _stream(stream)))
+
+
+def vsa_sparse_attn_fwd(q, k, v, block_idx, out, T, H, W, topk, workspace, lin_S=None, lin_z=None,
+                        tile=(4, 4, 4), stream=None):
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_sparse_attn_fwd", _lib.lib().vsa_sparse_attn_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), block_idx.data_ptr(), _ptr(lin_S), _ptr(lin_z),
+        out.data_ptr(), *_shape(B, heads, d, T, H, W, tile), topk, workspace.data_ptr(),
+        workspace.numel(), _stream(stream)))
+
+
+def vsa_device_status(workspace, stream=None) -> int:
+    """Synchronise and return the device status code (0 = VSA_OK)."""
+    return _lib.lib().vsa_device_status(workspace.data_ptr(), _stream(stream))
+
+
+class BlockSparseVideoAttention:
+    """Whole forward pass for one grid shape: select -> (linear state) -> fine.
+
+    Buffers (indices, linear state, workspace) are allocated once by torch and
+    reused by every call; `__call__` only enqueues kernels on the stream.
+    """
+
+    def __init__(self, B, heads, head_dim, T, H, W, topk, tile=(4, 4, 4), linear=False,
+                 device="cuda"):
+        self.shape = (B, heads, head_dim, T, H, W)
+        self.T, self.H, self.W, self.topk, self.tile, self.linear = T, H, W, topk, tuple(tile), linear
+        nt = vsa_num_tiles(T, H, W, tile)
+        self.num_tiles = nt
+        self.block_idx = torch.empty((B, heads, nt, topk), dtype=torch.int32, device=device)
+        self.workspace = new_workspace(B, heads, head_dim, T, H, W, topk, tile, device)
+        if linear:
+            self.lin_S = torch.empty((B, heads, head_dim, head_dim), dtype=torch.float32, device=device)
+            self.lin_z = torch.empty((B, heads, head_dim), dtype=torch.float32, device=device)
+        else:
+            self.lin_S = self.lin_z = None
+
+    def __call__(self, q, k, v, out=None, stream=None):
+        for x in (q, k, v):
+            assert x.dtype == torch.bfloat16 and x.is_cuda and tuple(x.shape[1:]) == (
+                self.T * self.H * self.W, self.shape[1], self.shape[2])
+        if out is None:
+            out = torch.empty_like(q)
+        vsa_select_blocks(q, k, self.T, self.H, self.W, self.topk, self.block_idx, self.workspace,
+                          self.tile, stream)
+        if self.linear:
+            vsa_linear_branch_fwd(k, v, self.lin_S, self.lin_z, self.T, self.H, self.W, stream)
+        vsa_sparse_attn_fwd(q, k, v, self.block_idx, out, self.T, self.H, self.W, self.topk,
+                            self.workspace, self.lin_S, self.lin_z, self.tile, stream)
+        return out
+
+    def status(self, stream=None) -> int:
+        return vsa_device_status(self.workspace, stream)

@@ -1,0 +1,146 @@
+/*
+ * vsa.h -- C ABI of a B200-native (sm_100a) block-sparse video attention
+ * library: VSA-style trainable block-sparse attention with an optional
+ * SLA/RoLA-style linear branch.
+ *
+ * What the method computes (sources, by page title and section):
+ *  - "FastVideo 稀疏蒸馏技术深度解析" (omica.com.cn), section "2. 视频稀疏注意力VSA":
+ *    video sparse attention picks, per block of queries, the key blocks that
+ *    matter and evaluates only 10-20 % of the attention weights (sparsity
+ *    0.8-0.9), staying compatible with exact Flash-Attention-style softmax.
+ *  - SparkDiffusion news item (bazainvestora.ru), paragraphs 2-3: at 97 %
+ *    sparsity 3 % of the blocks remain; RoLA adds a low-rank linear branch
+ *    that keeps global context next to the block-sparse branch.
+ *  - TurboDiffusion article (dolphinsci.com), section "稀疏、蒸馏与全链路量化":
+ *    SLA = trainable sparse attention plus a linear-attention branch.
+ * The pages leave the mechanics open; this library reads them as:
+ *  tokens of a T x H x W latent grid are grouped into tt x th x tw cube tiles
+ *  of 64 tokens (ceiling division; slots outside the grid are padding); each
+ *  cube is mean-pooled over its valid tokens; a query cube i scores every key
+ *  cube j with Qp[i].Kp[j]/sqrt(d) and keeps the top-k (ties -> lower j);
+ *  the fine pass is exact softmax attention (scale 1/sqrt(d)) of each query
+ *  over the valid tokens of its kept cubes; the optional linear branch adds
+ *  phi(q) S / (phi(q).z) with phi = elu + 1, S = sum_n phi(k_n)^T v_n and
+ *  z = sum_n phi(k_n) over all tokens.
+ *
+ * Conventions shared by every entry point
+ *  - Shape arguments: B (batch), heads, head_dim d (64 or 128), grid T, H, W
+ *    (token n = (t*H + h)*W + w, N = T*H*W), tile tt, th, tw with
+ *    tt*th*tw == 64.  Cube j = (it*nh + ih)*nw + iw with nT = ceil(T/tt),
+ *    nh = ceil(H/th), nw = ceil(W/tw), nt = nT*nh*nw; inside a cube, slot
+ *    s = (dt*th + dh)*tw + dw.
+ *  - q, k, v, out: bf16 (raw bit patterns, vsa_bf16), contiguous
+ *    [B][N][heads][d] in device memory.
+ *  - block_idx: int32 [B][heads][nt][topk] in device memory; each row is
+ *    strictly ascending with values in [0, nt).
+ *  - Every device pointer must be 16-byte aligned (TMA requirement).
+ *  - The caller owns every buffer and the stream.  The library never
+ *    allocates device memory, never frees it and never synchronises, except
+ *    vsa_device_status.  It keeps no global state besides a cached driver
+ *    entry point and per-device kernel attributes, and is re-entrant.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream).  Argument errors are reported before any launch;
+ *    launch failures return VSA_ERR_CUDA.  Faults detected on the device
+ *    (a bounded wait that gave up, a block index out of range) are recorded
+ *    in the workspace's status word and reported by vsa_device_status.
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t vsa_bf16;                 /* raw bfloat16 bits            */
+typedef struct CUstream_st* vsa_stream_t;  /* == cudaStream_t              */
+
+typedef enum {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARGUMENT = 1,  /* bad shape, null/misaligned pointer, bad topk */
+    VSA_ERR_UNSUPPORTED = 2,       /* head_dim not in {64,128}, tile volume != 64  */
+    VSA_ERR_WORKSPACE = 3,         /* workspace missing or smaller than required   */
+    VSA_ERR_CUDA = 4,              /* a CUDA runtime/driver call or launch failed  */
+    VSA_ERR_TIMEOUT = 5,           /* a device-side bounded wait gave up           */
+    VSA_ERR_DEVICE_CHECK = 6       /* a device-side range check failed             */
+} vsa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* vsa_status_string(vsa_status status);
+
+/* Number of cube tiles nt of a T x H x W grid cut into tt x th x tw tiles
+ * (ceiling division); 0 if any argument is < 1. */
+int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
+
+/* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
+ * for these shapes: a 256-byte status block followed by the fp64 cube means
+ * of q and k ([2][B][heads][nt][d]).  Returns 0 for invalid shapes.  The
+ * same workspace may be passed to every call of one forward pass; calls that
+ * share a workspace must be ordered on one stream. */
+size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W,
+                           int tt, int th, int tw, int topk);
+
+/* Clear the workspace's status word (enqueued on `stream`).  Call once after
+ * allocating a workspace, before its first use. */
+vsa_status vsa_workspace_init(void* workspace, size_t workspace_bytes, vsa_stream_t stream);
+
+/* Tile gather: grid order x[B][N][heads][d] -> cube-major
+ * x_tiles[B][heads][nt][64][d] (slot order above); padded slots are written
+ * as zeros.  A bit-exact copy (the tiling step of the pages' block selection,
+ * "2. 视频稀疏注意力VSA"). */
+vsa_status vsa_gather_tiles(const vsa_bf16* x, vsa_bf16* x_tiles, int B, int heads,
+                            int head_dim, int T, int H, int W, int tt, int th, int tw,
+                            vsa_stream_t stream);
+
+/* Tile scatter: cube-major x_tiles -> grid order x; only valid slots are
+ * written (padded slots of x_tiles are ignored).  Bit-exact. */
+vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int heads,
+                             int head_dim, int T, int H, int W, int tt, int th, int tw,
+                             vsa_stream_t stream);
+
+/* Block selection ("2. 视频稀疏注意力VSA": pick the key blocks each query block
+ * attends to).  Mean-pools q and k per cube over valid tokens (fp64), scores
+ * C[i][j] = Qp[i].Kp[j]/sqrt(d) in fp64 and writes, per (b, head, i), the
+ * topk key cubes with the largest C (ties -> lower j) in ascending order to
+ * block_idx.  1 <= topk <= nt.  Needs vsa_workspace_bytes() of workspace. */
+vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
+                             int head_dim, int T, int H, int W, int tt, int th, int tw,
+                             int topk, int32_t* block_idx, void* workspace,
+                             size_t workspace_bytes, vsa_stream_t stream);
+
+/* Linear-branch state (SparkDiffusion RoLA, paragraph 3; TurboDiffusion SLA,
+ * "稀疏、蒸馏与全链路量化"): lin_S[B][heads][d][d] = sum_n phi(k_n)^T v_n and
+ * lin_z[B][heads][d] = sum_n phi(k_n) over all N tokens, phi = elu + 1,
+ * fp32 accumulation.  Both outputs are fully overwritten. */
+vsa_status vsa_linear_branch_fwd(const vsa_bf16* k, const vsa_bf16* v, float* lin_S,
+                                 float* lin_z, int B, int heads, int head_dim, int T, int H,
+                                 int W, vsa_stream_t stream);
+
+/* Fine pass ("2. 视频稀疏注意力VSA": evaluate only the weights of the kept
+ * blocks, exactly, Flash-Attention style).  For every valid query token of
+ * cube i: softmax over the valid tokens of cubes block_idx[b][head][i][:] of
+ * q.k/sqrt(d) (fp32 online softmax, bf16 tensor-core products), times v,
+ * written as bf16 to out in grid order.  Padded slots take no part.  When
+ * lin_S and lin_z are both non-NULL (from vsa_linear_branch_fwd) the linear
+ * branch phi(q) S / (phi(q).z) is added in fp32 before rounding; pass both
+ * NULL for the sparse branch alone.  Needs vsa_workspace_bytes() of
+ * workspace (status word only). */
+vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                               const int32_t* block_idx, const float* lin_S,
+                               const float* lin_z, vsa_bf16* out, int B, int heads,
+                               int head_dim, int T, int H, int W, int tt, int th, int tw,
+                               int topk, void* workspace, size_t workspace_bytes,
+                               vsa_stream_t stream);
+
+/* Synchronise `stream`, then report and clear the device status word the
+ * kernels of this workspace wrote: VSA_OK, VSA_ERR_TIMEOUT or
+ * VSA_ERR_DEVICE_CHECK (VSA_ERR_CUDA if the stream itself failed). */
+vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI (no GPU work): the library loads, exports
+every entry point include/vsa.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_30_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vsa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation returns first
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ["vsa_select_blocks", "vsa_sparse_attn_fwd", "vsa_linear_branch_fwd",
+              "vsa_gather_tiles", "vsa_scatter_tiles", "vsa_workspace_bytes",
+              "vsa_device_status", "vsa_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(L):
+    for code, name in _lib.STATUS_NAMES.items():
+        assert L.vsa_status_string(code).decode() == name
+    assert L.vsa_status_string(99).decode() == "VSA_ERR_UNKNOWN"
+
+
+def test_num_tiles_and_workspace(L):
+    assert L.vsa_num_tiles(21, 45, 80, 4, 4, 4) == 1440
+    assert L.vsa_num_tiles(20, 28, 52, 4, 4, 4) == 455
+    assert L.vsa_num_tiles(4, 32, 32, 4, 4, 4) == 64
+    assert L.vsa_num_tiles(0, 4, 4, 4, 4, 4) == 0
+    nt, B, h, d = 455, 1, 40, 128
+    want = 256 + 2 * B * h * nt * d * 8 + B * h * nt * nt * 8
+    assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 46) == want
+    assert L.vsa_workspace_bytes(B, h, 96, 20, 28, 52, 4, 4, 4, 46) == 0       # d unsupported
+    assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
+    assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 0) == 0         # topk < 1
+    assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 456) == 0       # topk > nt
+
+
+SHAPE = [1, 2, 128, 4, 8, 8, 4, 4, 4]       # nt = 4
+
+
+def test_select_argument_validation(L):
+    f = L.vsa_select_blocks
+    big = 1 << 30
+    assert f(FAKE, FAKE, *SHAPE, 0, FAKE, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, *SHAPE, 5, FAKE, FAKE, big, None) == INVALID
+    assert f(None, FAKE, *SHAPE, 2, FAKE, FAKE, big, None) == INVALID
+    assert f(FAKE + 8, FAKE, *SHAPE, 2, FAKE, FAKE, big, None) == INVALID      # misaligned q
+    assert f(FAKE, FAKE, *SHAPE, 2, FAKE, None, big, None) == WORKSPACE
+    assert f(FAKE, FAKE, *SHAPE, 2, FAKE, FAKE, 100, None) == WORKSPACE
+    bad = list(SHAPE); bad[2] = 80
+    assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == UNSUPPORTED
+    bad = list(SHAPE); bad[6] = 2
+    assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == UNSUPPORTED
+    bad = list(SHAPE); bad[3] = 0
+    assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == INVALID
+
+
+def test_fine_argument_validation(L):
+    f = L.vsa_sparse_attn_fwd
+    big = 1 << 20
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *SHAPE, 0, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, *SHAPE, 2, FAKE, big, None) == INVALID  # S w/o z
+    assert f(FAKE, FAKE, FAKE, None, None, None, FAKE, *SHAPE, 2, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE + 2, *SHAPE, 2, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *SHAPE, 2, None, big, None) == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *SHAPE, 2, FAKE, 64, None) == WORKSPACE
+    bad = list(SHAPE); bad[2] = 256
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *bad, 2, FAKE, big, None) == UNSUPPORTED
+
+
+def test_other_entry_points_validate(L):
+    assert L.vsa_gather_tiles(None, FAKE, *SHAPE, None) == INVALID
+    assert L.vsa_scatter_tiles(FAKE, FAKE + 4, *SHAPE, None) == INVALID
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, None, FAKE, 1, 2, 128, 4, 8, 8, None) == INVALID
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 32, 4, 8, 8, None) == UNSUPPORTED
+    assert L.vsa_workspace_init(None, 1024, None) == INVALID
+    assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
+    assert L.vsa_device_status(None, None) == INVALID
+
+
+def test_library_has_no_oracle_dependency():
+    """The product library never links or names the oracle."""
+    with open(_lib.LIB_PATH, "rb") as fh:
+        blob = fh.read()
+    assert b"oracle" not in blob
+    for root, _, files in os.walk(os.path.join(ROOT, "block_sparse_attention_30_b200")):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(root, fn), encoding="utf-8").read()
+                assert "import oracle" not in src and "from oracle" not in src, fn

@@ -1,0 +1,316 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars: block indices bit-exact, except that a cube may differ when its oracle
+coarse score lies within 1e-5 of the row's k-th largest score (a near-tie);
+fine output within max-abs 2e-2 and relative Frobenius 1e-2 of the oracle run
+on the GPU's own indices; cube gather/scatter bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_30_b200 import WORKLOADS, synth
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_FRO, TIE = 2e-2, 1e-2, 1e-5
+
+
+@pytest.fixture(scope="module")
+def ops():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_attention_30_b200 import build, ops
+    build.build()
+    return ops
+
+
+_INPUTS = {}
+
+
+def inputs(name):
+    if name not in _INPUTS:
+        w = WORKLOADS[name]
+        q, k, v = synth.make_workload_inputs(w)
+        _INPUTS[name] = (w, q, k, v, q.cuda(), k.cuda(), v.cuda())
+    return _INPUTS[name]
+
+
+def check_indices(gpu_idx, ref_idx, scores):
+    """Bit-exact, except near-ties (|C - tau| < 1e-5, tau = k-th largest)."""
+    gpu_idx = np.asarray(gpu_idx)
+    assert np.all(np.diff(gpu_idx, axis=-1) > 0), "rows must be strictly ascending"
+    assert gpu_idx.min() >= 0 and gpu_idx.max() < scores.shape[-1]
+    diff_rows = np.nonzero(np.any(gpu_idx != ref_idx, axis=-1))
+    k = gpu_idx.shape[-1]
+    for r in zip(*diff_rows):
+        row = scores[r]
+        tau = np.sort(row)[::-1][k - 1]
+        sym = set(gpu_idx[r].tolist()) ^ set(ref_idx[r].tolist())
+        for j in sym:
+            assert abs(row[j] - tau) < TIE, (r, j, row[j], tau)
+    return len(diff_rows[0])
+
+
+def check_close(got, ref):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref).max()
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err <= MAX_ABS and rel <= REL_FRO, (err, rel)
+    return err, rel
+
+
+def run_select(ops, w, q_d, k_d, topk=None, tile=None):
+    topk = w.topk if topk is None else topk
+    tile = w.tile if tile is None else tile
+    B, N, heads, d = q_d.shape
+    nt = ops.vsa_num_tiles(w.T, w.H, w.W, tile)
+    idx = torch.empty((B, heads, nt, topk), dtype=torch.int32, device="cuda")
+    ws = ops.new_workspace(B, heads, d, w.T, w.H, w.W, topk, tile)
+    ops.vsa_select_blocks(q_d, k_d, w.T, w.H, w.W, topk, idx, ws, tile)
+    assert ops.vsa_device_status(ws) == 0
+    return idx, ws
+
+
+def run_fine(ops, w, q_d, k_d, v_d, idx, ws, tile=None, lin=None):
+    tile = w.tile if tile is None else tile
+    out = torch.full_like(q_d, float("nan"))
+    S, z = lin if lin is not None else (None, None)
+    ops.vsa_sparse_attn_fwd(q_d, k_d, v_d, idx, out, w.T, w.H, w.W, idx.shape[-1], ws, S, z, tile)
+    assert ops.vsa_device_status(ws) == 0
+    return out
+
+
+def to_f64(t):
+    return t.float().cpu().double().numpy()
+
+
+# ------------------------------------------------------------ small grids
+
+class Small:
+    def __init__(self, T, H, W, heads, d, topk, tile=(4, 4, 4), amplitude=1.0, seed=0, B=1):
+        self.T, self.H, self.W, self.heads, self.head_dim, self.topk = T, H, W, heads, d, topk
+        self.tile, self.B = tile, B
+        self.q, self.k, self.v = synth.make_qkv(B, heads, d, T, H, W, tile, amplitude, seed)
+
+
+SMALL = [
+    # T, H, W, heads, d, topk, tile
+    (4, 8, 8, 2, 128, 2, (4, 4, 4)),        # 4 cubes, even k
+    (5, 6, 7, 2, 128, 3, (4, 4, 4)),        # ragged on every axis, odd k
+    (9, 13, 10, 3, 64, 5, (4, 4, 4)),       # ragged, d = 64
+    (8, 16, 16, 2, 128, 1, (4, 4, 4)),      # k = 1
+    (8, 16, 16, 2, 128, 32, (4, 4, 4)),     # k = nt (dense)
+    (8, 12, 20, 2, 64, 7, (2, 4, 8)),       # non-cubic tile shape
+    (6, 10, 9, 2, 128, 9, (4, 4, 4)),       # ragged, several pairs + odd tail
+]
+
+
+@pytest.mark.parametrize("case", SMALL)
+def test_small_grids_select_and_fine(ops, case):
+    T, H, W, heads, d, topk, tile = case
+    c = Small(T, H, W, heads, d, topk, tile, seed=hash(case) % 1000)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    ref_idx, scores = O.select(c.q, c.k, 1, heads, d, T, H, W, topk, tile, with_scores=True)
+    check_indices(idx.cpu().numpy(), ref_idx, scores)
+    out = run_fine(ops, c, qd, kd, vd, idx, ws)
+    ref = O.fine(c.q, c.k, c.v, idx.cpu().numpy(), 1, heads, d, T, H, W, tile)
+    assert not torch.isnan(out).any(), "every valid token must be written"
+    check_close(to_f64(out), ref)
+
+
+def test_dense_limit_matches_sdpa(ops):
+    """k = nt: the fine pass is dense attention (torch SDPA as reference)."""
+    T, H, W, heads, d = 8, 16, 16, 2, 128
+    c = Small(T, H, W, heads, d, 32, seed=21, amplitude=0.7)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    assert torch.equal(idx[0, 0, 0].cpu(), torch.arange(32, dtype=torch.int32))
+    out = run_fine(ops, c, qd, kd, vd, idx, ws)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(x.double().permute(0, 2, 1, 3) for x in (c.q, c.k, c.v))).permute(0, 2, 1, 3)
+    check_close(to_f64(out), ref.numpy())
+
+
+def test_index_order_invariance(ops):
+    """Permuting a row's indices leaves the output unchanged (up to fp32 order)."""
+    c = Small(8, 16, 16, 2, 128, 6, seed=3)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    out1 = run_fine(ops, c, qd, kd, vd, idx, ws)
+    perm = idx.flip(-1).contiguous()
+    out2 = run_fine(ops, c, qd, kd, vd, perm, ws)
+    assert (out1.float() - out2.float()).abs().max().item() < 2e-2
+
+
+def test_bad_index_is_reported_not_faulted(ops):
+    c = Small(4, 8, 8, 2, 128, 2, seed=4)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    bad = idx.clone()
+    bad[0, 1, 2, 1] = 4          # nt == 4: out of range
+    out = torch.empty_like(qd)
+    ops.vsa_sparse_attn_fwd(qd, kd, vd, bad, out, c.T, c.H, c.W, 2, ws)
+    assert ops.vsa_device_status(ws) == 6          # VSA_ERR_DEVICE_CHECK
+    assert ops.vsa_device_status(ws) == 0          # cleared by the read
+
+
+def test_repeated_calls_are_deterministic(ops):
+    c = Small(8, 16, 16, 2, 128, 5, seed=8)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    a = run_fine(ops, c, qd, kd, vd, idx, ws)
+    b = run_fine(ops, c, qd, kd, vd, idx, ws)
+    assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------- gather/scatter
+
+@pytest.mark.parametrize("case", [(5, 6, 7, 2, 128, (4, 4, 4)), (9, 13, 10, 3, 64, (4, 4, 4)),
+                                  (8, 12, 20, 2, 64, (2, 4, 8))])
+def test_gather_scatter_bit_exact(ops, case):
+    T, H, W, heads, d, tile = case
+    q, _, _ = synth.make_qkv(1, heads, d, T, H, W, tile, 1.0, seed=2)
+    nt = ops.vsa_num_tiles(T, H, W, tile)
+    qd = q.cuda()
+    tiles = torch.full((1, heads, nt, 64, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    ops.vsa_gather_tiles(qd, tiles, T, H, W, tile)
+    ref = O.gather(q, 1, heads, d, T, H, W, tile)
+    got = tiles.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    back = torch.zeros_like(qd)
+    ops.vsa_scatter_tiles(tiles, back, T, H, W, tile)
+    assert torch.equal(back.cpu(), q)
+
+
+# ---------------------------------------------------------- named workloads
+
+def sample_rows(nt, heads, B, n, seed, extra=()):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(B * heads * nt, size=min(n, B * heads * nt), replace=False).tolist())
+    rows.update([0, nt - 1, B * heads * nt - 1, *extra])
+    return np.array(sorted(rows), np.int64)
+
+
+def check_fine_sample(out, w, q, k, v, idx_np, rows):
+    part = O.fine_tiles(q, k, v, idx_np, rows, w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.tile)
+    slots = O.tile_slots(w.T, w.H, w.W, w.tile)
+    nt = slots.shape[0]
+    got = []
+    ref = []
+    out_c = out
+    for r, row in enumerate(rows):
+        bh, i = divmod(int(row), nt)
+        b, head = divmod(bh, w.heads)
+        toks = slots[i]
+        valid = toks >= 0
+        sel = out_c[b, torch.as_tensor(toks[valid]), head].float().cpu().double().numpy()
+        got.append(sel)
+        ref.append(part[r][valid])
+    return check_close(np.concatenate(got), np.concatenate(ref))
+
+
+@pytest.mark.parametrize("name", ["tiny_4x32x32"])
+def test_tiny_workload_full(ops, name):
+    w, q, k, v, qd, kd, vd = inputs(name)
+    idx, ws = run_select(ops, w, qd, kd)
+    ref_idx, scores = O.select(q, k, w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                               with_scores=True)
+    check_indices(idx.cpu().numpy(), ref_idx, scores)
+    out = run_fine(ops, w, qd, kd, vd, idx, ws)
+    ref = O.fine(q, k, v, idx.cpu().numpy(), w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.tile)
+    check_close(to_f64(out), ref)
+
+
+@pytest.mark.parametrize("name,heads_sel", [("wan1.3b_480p", None), ("wan14b_480p", None),
+                                            ("wan14b_720p_ragged", (0, 4)),
+                                            ("sparse97_linear_480p", None)])
+def test_workload_selection(ops, name, heads_sel):
+    """Selection on the full-size workloads (a head subset for the largest)."""
+    w, q, k, v, qd, kd, vd = inputs(name)
+    idx, _ = run_select(ops, w, qd, kd)
+    idx = idx.cpu().numpy()
+    if heads_sel is not None:
+        h0, h1 = heads_sel
+        qs, ks = q[:, :, h0:h1].contiguous(), k[:, :, h0:h1].contiguous()
+        idx = idx[:, h0:h1]
+    else:
+        h0, h1, qs, ks = 0, w.heads, q, k
+    ref_idx, scores = O.select(qs, ks, w.B, h1 - h0, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                               with_scores=True)
+    check_indices(idx, ref_idx, scores)
+
+
+@pytest.mark.parametrize("name", ["wan1.3b_480p", "wan14b_480p", "wan14b_720p_ragged"])
+def test_workload_fine_sampled(ops, name):
+    """Full-size fine pass, checked on sampled query cubes (incl. edge cubes)."""
+    w, q, k, v, qd, kd, vd = inputs(name)
+    idx, ws = run_select(ops, w, qd, kd)
+    out = run_fine(ops, w, qd, kd, vd, idx, ws)
+    assert not torch.isnan(out).any(), "every valid token must be written"
+    nt = ops.vsa_num_tiles(w.T, w.H, w.W, w.tile)
+    nT, nh, nw = w.tile_grid
+    corner = (nT - 1) * nh * nw + (nh - 1) * nw + (nw - 1)     # most ragged cube of head 0
+    rows = sample_rows(nt, w.heads, w.B, 24, seed=len(name), extra=(corner,))
+    check_fine_sample(out, w, q, k, v, idx.cpu().numpy(), rows)
+
+
+# -------------------------------------------------------------- linear branch
+
+def test_linear_state_small(ops):
+    c = Small(5, 6, 7, 3, 128, 3, seed=31, amplitude=0.7)
+    kd, vd = c.k.cuda(), c.v.cuda()
+    S = torch.empty((1, 3, 128, 128), dtype=torch.float32, device="cuda")
+    z = torch.empty((1, 3, 128), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, c.T, c.H, c.W)
+    Sr, zr = O.linear_state(c.k, c.v, 1, 3, 128, c.T * c.H * c.W)
+    np.testing.assert_allclose(S.cpu().double().numpy(), Sr, rtol=1e-4, atol=1e-3)
+    np.testing.assert_allclose(z.cpu().double().numpy(), zr, rtol=1e-4, atol=1e-3)
+
+
+@pytest.mark.parametrize("case", [(5, 6, 7, 2, 128, 3), (9, 13, 10, 2, 64, 4)])
+def test_linear_branch_small_full(ops, case):
+    T, H, W, heads, d, topk = case
+    c = Small(T, H, W, heads, d, topk, seed=41, amplitude=0.7)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    S = torch.empty((1, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((1, heads, d), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W)
+    out = run_fine(ops, c, qd, kd, vd, idx, ws, lin=(S, z))
+    N = T * H * W
+    ref = O.fine(c.q, c.k, c.v, idx.cpu().numpy(), 1, heads, d, T, H, W)
+    Sr, zr = O.linear_state(c.k, c.v, 1, heads, d, N)
+    ref = ref + O.linear_apply(c.q, Sr, zr, 1, heads, d, N)
+    check_close(to_f64(out), ref)
+
+
+def test_sparse97_linear_workload_sampled(ops):
+    name = "sparse97_linear_480p"
+    w, q, k, v, qd, kd, vd = inputs(name)
+    from block_sparse_attention_30_b200.ops import BlockSparseVideoAttention
+    attn = BlockSparseVideoAttention(w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                                     linear=True)
+    out = attn(qd, kd, vd)
+    assert attn.status() == 0
+    idx_np = attn.block_idx.cpu().numpy()
+    Sr, zr = O.linear_state(k, v, w.B, w.heads, w.head_dim, w.N)
+    np.testing.assert_allclose(attn.lin_S.cpu().double().numpy(), Sr, rtol=1e-4, atol=2e-2)
+    nt = w.num_tiles
+    rows = sample_rows(nt, w.heads, w.B, 16, seed=7)
+    part = O.fine_tiles(q, k, v, idx_np, rows, w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.tile)
+    slots = O.tile_slots(w.T, w.H, w.W, w.tile)
+    got, ref = [], []
+    for r, row in enumerate(rows):
+        bh, i = divmod(int(row), nt)
+        b, head = divmod(bh, w.heads)
+        toks = slots[i][slots[i] >= 0]
+        qrow = q[b:b + 1, torch.as_tensor(toks), head:head + 1].contiguous()
+        lin = O.linear_apply(qrow, Sr[b:b + 1, head:head + 1], zr[b:b + 1, head:head + 1], 1, 1,
+                             w.head_dim, len(toks))[0, :, 0]
+        ref.append(part[r][slots[i] >= 0] + lin)
+        got.append(out[b, torch.as_tensor(toks), head].float().cpu().double().numpy())
+    check_close(np.concatenate(got), np.concatenate(ref))
