@@ -1,0 +1,340 @@
+"""Benchmark of the block-sparse video attention forward pass on B200.
+
+One step = the whole hot path on one batch: block selection (pool, coarse
+scores, top-k) and the fine pass with its fused cube gather/scatter (plus the
+linear-branch state for workloads that have one), all through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  `value` is the effective fine-pass TFLOP/s of
+the whole step, 4 * N_valid * k * 64 * d * heads * B FLOPs per step (selected
+blocks only), summed over ranks; every rank runs its own copy of the workload
+(weak scaling, no data-path collective).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_30_b200 import HEADLINE, WORKLOADS, synth  # noqa: E402
+
+METRIC = "fine-attn effective TFLOP/s & ms/call (selected blocks), % of B200 BF16 peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(
+        os.environ.get("WORLD_SIZE", 1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_step_fn(w, q, k, v, out, attn, fine_events):
+    """One hot-path pass on the current stream; fine_events brackets the fine kernel."""
+    from block_sparse_attention_30_b200 import ops
+
+    def step(record_fine=False):
+        ops.vsa_select_blocks(q, k, w.T, w.H, w.W, w.topk, attn.block_idx, attn.workspace, w.tile)
+        if w.linear:
+            ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W)
+        if record_fine:
+            fine_events[0].record()
+        ops.vsa_sparse_attn_fwd(q, k, v, attn.block_idx, out, w.T, w.H, w.W, w.topk,
+                                attn.workspace, attn.lin_S, attn.lin_z, w.tile)
+        if record_fine:
+            fine_events[1].record()
+    return step
+
+
+def run_gpu(args):
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from block_sparse_attention_30_b200 import build, ops
+    build.build()
+    w = WORKLOADS[args.workload]
+    q_h, k_h, v_h = synth.make_workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    out = torch.empty_like(q)
+    attn = ops.BlockSparseVideoAttention(w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                                         linear=w.linear, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fine_ev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+    step = gpu_step_fn(w, q, k, v, out, attn, fine_ev)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if attn.status() != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    fine_ms = []
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)                          # let the sampler take its first reading
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 255)                 # evict L2 between steps (outside the events)
+        starts[i].record()
+        step(record_fine=True)
+        ends[i].record()
+        ends[i].synchronize()
+        fine_ms.append(fine_ev[0].elapsed_time(fine_ev[1]))
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    status = attn.status()
+
+    # end to end through the public API: pinned host inputs in, host output back
+    e2e_steps = max(1, min(args.steps, 5))
+    qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
+    out_h = torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        qd = qp.to(dev, non_blocking=True)
+        kd = kp.to(dev, non_blocking=True)
+        vd = vp.to(dev, non_blocking=True)
+        attn(qd, kd, vd, out=out)
+        out_h.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = 3 * q_h.numel() * q_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    stats = torch.tensor([total_ms, e2e_ms, sum(fine_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms, fine_total = stats.tolist()
+
+    if rank == 0:
+        flops = w.fine_flops()
+        ms_per_step = total_ms / args.steps
+        value = world * flops / (ms_per_step * 1e-3) / 1e12
+        fine_avg_ms = fine_total / args.steps
+        fine_tflops = flops / (fine_avg_ms * 1e-3) / 1e12
+        peaks, src = load_peaks()
+        peak = peaks["bf16_tflops"]
+        launches_per_step = 4 + (1 if w.linear else 0)
+        result = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) noise + per-cube N(0,1) offsets, Wan latent shapes)",
+            "config": {
+                "workload": w.name, "B": w.B, "heads": w.heads, "head_dim": w.head_dim,
+                "grid": [w.T, w.H, w.W], "tile": list(w.tile), "num_tiles": w.num_tiles,
+                "topk": w.topk, "sparsity": round(w.sparsity, 4), "linear_branch": w.linear,
+                "fine_flops_per_step": flops,
+                "l2": "256 MiB write between steps (outside the timed events); inputs 3x%.0f MB exceed L2"
+                      % (q_h.numel() * 2 / 1e6),
+                "parallelism": f"replica per GPU x{world}",
+            },
+            "fine_kernel": {"ms_per_call": round(fine_avg_ms, 4), "tflops": round(fine_tflops, 2),
+                            "pct_of_bf16_peak": round(100 * fine_tflops / peak, 2),
+                            "pct_of_bf16_sustained": round(100 * fine_tflops / peaks["bf16_tflops_sustained"], 2)},
+            "pct_of_bf16_peak": round(100 * (value / world) / peak, 2),
+            "roofline": {
+                "bound": "tensor", "kernel": "fine_attn_kernel<%d>" % w.head_dim,
+                "achieved": round(fine_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(fine_tflops / peak, 4),
+                "peak_source": f"{src} bf16_tflops (burst)",
+                "traffic": args.traffic,
+            },
+            "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "device_status": status,
+            "wall_s": round(wall, 3),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, args.cpu_heads)
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# -------------------------------------------------------------------- oracle
+
+def oracle_sample(w, q, k, v, heads):
+    """Select + fine (+ linear) of the oracle on the first `heads` heads (all
+    query cubes of each); returns (seconds, fine FLOPs covered)."""
+    from oracle import oracle as O
+    qs, ks, vs = (x[:, :, :heads].contiguous() for x in (q, k, v))
+    t0 = time.perf_counter()
+    idx = O.select(qs, ks, w.B, heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile)
+    out = O.fine(qs, ks, vs, idx, w.B, heads, w.head_dim, w.T, w.H, w.W, w.tile)
+    if w.linear:
+        S, z = O.linear_state(ks, vs, w.B, heads, w.head_dim, w.N)
+        out = out + O.linear_apply(qs, S, z, w.B, heads, w.head_dim, w.N)
+    dt = time.perf_counter() - t0
+    return dt, w.fine_flops() * heads / w.heads
+
+
+def cpu_baseline(w, q, k, v, heads):
+    from oracle import oracle as O
+    heads = min(heads, w.heads)
+    dt, flops = oracle_sample(w, q, k, v, heads)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": O.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"{heads} of {w.heads} heads, all {w.num_tiles} query cubes each: "
+                      f"fp64 select + fine{' + linear' if w.linear else ''}"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return                                   # rank 0 alone runs the CPU oracle
+    from oracle import oracle as O
+    w = WORKLOADS[args.workload]
+    q, k, v = synth.make_workload_inputs(w)
+    heads = min(args.cpu_heads, w.heads)
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, 1)
+    times = []
+    flops = 0.0
+    for _ in range(args.steps):
+        dt, flops = oracle_sample(w, q, k, v, heads)
+        times.append(dt)
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    cb = {"value": round(value, 6), "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
+          "sample": f"{heads} of {w.heads} heads per step, all {w.num_tiles} query cubes each: "
+                    f"fp64 select + fine{' + linear' if w.linear else ''}"}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "head_dim": w.head_dim,
+                   "grid": [w.T, w.H, w.W], "topk": w.topk, "sample_heads": heads},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per fine launch from an ncu capture (reported as-is)")
+    args = ap.parse_args()
+    _, _, world = dist_env()
+    if world != args.gpus:
+        if args.gpus > 1 and world == 1:
+            sys.exit("for --gpus > 1 launch with torch.distributed.run --nproc-per-node N")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        if not torch.cuda.is_available():
+            sys.exit("bench.py needs a CUDA device for --impl ours")
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
