@@ -30,7 +30,11 @@ SIGNATURES = {
     "vsa_linear_branch_fwd": (_i, [_p, _p, _p, _p] + [_i] * 6 + [_p]),
     "vsa_sparse_attn_fwd": (_i, [_p] * 7 + _SHAPE + [_i, _p, _sz, _p]),
     "vsa_device_status": (_i, [_p, _p]),
+    "vsa_select_blocks_noalloc": (_i, [_p, _p] + _SHAPE + [_i, _p, _p]),
 }
+
+# VSA_NOALLOC_SELECT_SCRATCH_BYTES of include/vsa.h
+NOALLOC_SELECT_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class VSAError(RuntimeError):

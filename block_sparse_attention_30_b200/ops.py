@@ -71,6 +71,15 @@ def vsa_select_blocks(q, k, T, H, W, topk, block_idx, workspace, tile=(4, 4, 4),
         block_idx.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
 
 
+def vsa_select_blocks_noalloc(q, k, T, H, W, topk, block_idx, tile=(4, 4, 4), stream=None):
+    """vsa_select_blocks without a workspace: for callers that cannot allocate
+    device memory.  The library's fixed device array holds the intermediates."""
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_select_blocks_noalloc", _lib.lib().vsa_select_blocks_noalloc(
+        q.data_ptr(), k.data_ptr(), *_shape(B, heads, d, T, H, W, tile), topk,
+        block_idx.data_ptr(), _stream(stream)))
+
+
 def vsa_linear_branch_fwd(k, v, lin_S, lin_z, T, H, W, stream=None):
     B, heads, d = _grid_of(k, T, H, W)
     _lib.check("vsa_linear_branch_fwd", _lib.lib().vsa_linear_branch_fwd(

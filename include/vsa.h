@@ -37,7 +37,8 @@
  *  - The caller owns every buffer and the stream.  The library never
  *    allocates device memory, never frees it and never synchronises, except
  *    vsa_device_status.  It keeps no global state besides a cached driver
- *    entry point and per-device kernel attributes, and is re-entrant.
+ *    entry point, per-device kernel attributes and the fixed device array of
+ *    vsa_select_blocks_noalloc (end of this header), and is re-entrant.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream).  Argument errors are reported before any launch;
  *    launch failures return VSA_ERR_CUDA.  Faults detected on the device
@@ -138,6 +139,37 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
  * kernels of this workspace wrote: VSA_OK, VSA_ERR_TIMEOUT or
  * VSA_ERR_DEVICE_CHECK (VSA_ERR_CUDA if the stream itself failed). */
 vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Allocation-free block selection.
+ *
+ * No counterpart on the pages: this entry point exists for callers that cannot
+ * allocate device memory (no cudaMalloc: a callback or runtime that forbids
+ * allocation, a fixed memory budget, an embedding without an allocator) and
+ * so cannot provide vsa_select_blocks' workspace.  It computes exactly what
+ * vsa_select_blocks computes, with the same kernels, but keeps the
+ * intermediate fp64 cube means and coarse scores in one file-scope device
+ * array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved on every GPU that loads
+ * the library until the process exits.  It allocates and frees nothing.
+ *
+ *  - The caller still passes q, k (device, bf16 [B][N][heads][d]) and
+ *    block_idx (device, int32 [B][heads][nt][topk]), 16-byte aligned.
+ *  - Shapes whose intermediates exceed the array
+ *    (2*B*heads*nt*d*8 + B*heads*nt*nt*8 bytes > the maximum) are rejected
+ *    with VSA_ERR_WORKSPACE before anything is enqueued; argument errors as
+ *    for vsa_select_blocks.
+ *  - All calls share the array, which keeps the last call's contents; every
+ *    call rewrites what it reads, so nothing needs clearing.  Calls that
+ *    overlap on the GPU (other streams, unordered host threads) race on it:
+ *    order them on one stream.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ */
+#define VSA_NOALLOC_SELECT_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+vsa_status vsa_select_blocks_noalloc(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
+                                     int head_dim, int T, int H, int W, int tt, int th, int tw,
+                                     int topk, int32_t* block_idx, vsa_stream_t stream);
 
 #ifdef __cplusplus
 }
