@@ -2,6 +2,7 @@
 // device status word, small math helpers.
 #pragma once
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace vsa {
@@ -53,19 +54,27 @@ __device__ __forceinline__ TileCoord tile_coord(const Grid& g, int j) {
     return c;
 }
 
-// 64-bit mask of the valid slots of a cube (slot s = (dt*th + dh)*tw + dw).
+// 64-bit mask of the valid slots of a cube (slot s = (dt*th + dh)*tw + dw):
+// a row of vw bits, repeated for the vh valid rows, repeated for the vt
+// valid layers.
 __device__ __forceinline__ uint64_t valid_slot_mask(const Grid& g, const TileCoord& c) {
     if (c.vt == g.tt && c.vh == g.th && c.vw == g.tw) return ~0ull;
+    const uint64_t row = (1ull << c.vw) - 1ull;
+    uint64_t layer = 0;
+    for (int dh = 0; dh < c.vh; ++dh) layer |= row << (dh * g.tw);
     uint64_t m = 0;
-    for (int s = 0; s < 64; ++s) {
-        const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
-        if (dt < c.vt && dh < c.vh && dw < c.vw) m |= 1ull << s;
-    }
+    const int layer_bits = g.th * g.tw;
+    for (int dt = 0; dt < c.vt; ++dt) m |= layer << (dt * layer_bits);
     return m;
 }
 
 __device__ __forceinline__ void report(int* status, int bits) {
     if (status) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // 2^x on the MUFU unit (hardware approximation, ~2 ulp).

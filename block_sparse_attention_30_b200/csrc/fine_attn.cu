@@ -32,6 +32,7 @@
 #include "common.cuh"
 #include "fine_attn.h"
 #include "sm100.cuh"
+#include "softmax_step.cuh"
 
 namespace vsa {
 using namespace sm100;
@@ -64,24 +65,12 @@ struct FineBars {
 static_assert(sizeof(FineBars<128>) <= FineCfg<128>::BAR_BYTES, "barrier block");
 static_assert(sizeof(FineBars<64>) <= FineCfg<64>::BAR_BYTES, "barrier block");
 
-__device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) return false;
-    return true;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-template <int D>
-__global__ void __launch_bounds__(192, 2)
+template <int D, bool LIN>
+__global__ void __launch_bounds__(224, 2)
 fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                  const __grid_constant__ CUtensorMap mv, const Grid g,
                  const int32_t* __restrict__ block_idx, const int topk, const float scale_log2,
-                 const float* __restrict__ lin_S, const float* __restrict__ lin_z,
+                 const int ragged, const float* __restrict__ lin_S, const float* __restrict__ lin_z,
                  __nv_bfloat16* __restrict__ out, int* status) {
     using C = FineCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -102,7 +91,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const int head = bh % g.heads, b = bh / g.heads;
     const int32_t* my_idx = block_idx + row_id * topk;
     const int n_pairs = (topk + 1) >> 1;
-    const bool lin = lin_S != nullptr && lin_z != nullptr;
+    constexpr bool lin = LIN;
     // Linear-branch operands reuse the K/V rings once the last PV is done:
     //   phi(Q) hi / lo  (A, K-major like Q)        at sK, sK + Q_BYTES
     //   S hi / lo       (B, MN-major like V pairs) at sK + 2*Q_BYTES, + D*D*2
@@ -136,50 +125,49 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         report(status, kStatusTimeout);
     };
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ producer
+    if (warp == 4 || warp == 6) {
+        // --------------------------------------- producers: Q + K (warp 4), V (warp 6)
+        // Two warps, so that a wait for a free V slot never delays a K load.
         if (lane == 0) {
-            int k_issued = 0, v_issued = 0;
-            const TileCoord qc = tile_coord(g, i);
-            mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-            for (int c = 0; c < C::NCH; ++c)
-                tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + 64 * c, qc.w0, qc.h0, qc.t0, b);
+            const bool is_k = warp == 4;
+            int issued = 0;
+            if (is_k) {
+                const TileCoord qc = tile_coord(g, i);
+                mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+                for (int c = 0; c < C::NCH; ++c)
+                    tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + 64 * c, qc.w0, qc.h0, qc.t0, b);
+            }
+            const int nst = is_k ? C::NK : C::NV;
+            uint64_t* full = is_k ? bars->k_full : bars->v_full;
+            uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+            uint8_t* ring = is_k ? sK : sV;
+            const CUtensorMap* map = is_k ? &mk : &mv;
+            int jn[2] = {__ldg(my_idx), topk > 1 ? __ldg(my_idx + 1) : 0};
             for (int p = 0; p < n_pairs; ++p) {
                 const int ntl = min(2, topk - 2 * p);
-                int jt[2] = {0, 0};
-                for (int t = 0; t < ntl; ++t) {
-                    int j = __ldg(my_idx + 2 * p + t);
-                    if (j < 0 || j >= g.nt) { report(status, kStatusBadIndex); j = 0; }
-                    jt[t] = j;
+                int jt[2] = {jn[0], jn[1]};
+                if (p + 1 < n_pairs) {                      // next pair's cubes, in flight meanwhile
+                    jn[0] = __ldg(my_idx + 2 * p + 2);
+                    jn[1] = 2 * p + 3 < topk ? __ldg(my_idx + 2 * p + 3) : 0;
                 }
-                const int sk = p % C::NK;
-                if (p >= C::NK && !mbar_wait(&bars->k_empty[sk], ((p / C::NK) - 1) & 1, abort_flag)) { fail(); break; }
-                mbar_arrive_expect_tx(&bars->k_full[sk], ntl * C::CUBE_BYTES);
-                for (int t = 0; t < ntl; ++t) {
-                    const TileCoord kc = tile_coord(g, jt[t]);
-                    for (int c = 0; c < C::NCH; ++c)
-                        tma_load_5d(sK + sk * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, &mk,
-                                    &bars->k_full[sk], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
-                }
-                ++k_issued;
-                const int sv = p % C::NV;
-                if (p >= C::NV && !mbar_wait(&bars->v_empty[sv], ((p / C::NV) - 1) & 1, abort_flag)) { fail(); break; }
-                mbar_arrive_expect_tx(&bars->v_full[sv], ntl * C::CUBE_BYTES);
+                for (int t = 0; t < ntl; ++t)
+                    if (jt[t] < 0 || jt[t] >= g.nt) { if (is_k) report(status, kStatusBadIndex); jt[t] = 0; }
+                const int st = p % nst;
+                if (p >= nst && !mbar_wait(&empty[st], ((p / nst) - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&full[st], ntl * C::CUBE_BYTES);
                 for (int t = 0; t < ntl; ++t) {
                     const TileCoord kc = tile_coord(g, jt[t]);
                     for (int c = 0; c < C::NCH; ++c)
-                        tma_load_5d(sV + sv * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, &mv,
-                                    &bars->v_full[sv], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
+                        tma_load_5d(ring + st * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, map,
+                                    &full[st], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
                 }
-                ++v_issued;
+                ++issued;
             }
             if (*abort_flag) {
                 // drain: the last load issued into each stage must land before exit
-                wait_noabort(&bars->q_full, 0);
-                for (int n = max(0, k_issued - C::NK); n < k_issued; ++n)
-                    wait_noabort(&bars->k_full[n % C::NK], (n / C::NK) & 1);
-                for (int n = max(0, v_issued - C::NV); n < v_issued; ++n)
-                    wait_noabort(&bars->v_full[n % C::NV], (n / C::NV) & 1);
+                if (is_k) wait_noabort(&bars->q_full, 0);
+                for (int n = max(0, issued - nst); n < issued; ++n)
+                    wait_noabort(&full[n % nst], (n / nst) & 1);
             }
         }
     } else if (warp == 5) {
@@ -245,12 +233,12 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         const int r = 16 * warp + (lane & 15), hf = lane >> 4;
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
         const uint32_t tS = tbase + lane_base + C::S_COL, tO = tbase + lane_base + C::O_COL;
-        float m_run = -INFINITY, l_run = 0.f;
+        SoftmaxState sm{-INFINITY, 0.f};
         bool ok = true;
         for (int p = 0; p < n_pairs; ++p) {
             const int ntl = min(2, topk - 2 * p);
-            uint64_t vmask = 0;
-            if (hf < ntl) {
+            uint64_t vmask = hf < ntl ? ~0ull : 0ull;   // odd tail: this half has no cube
+            if (ragged && hf < ntl) {                   // edge cubes: mask padded keys
                 int j = __ldg(my_idx + 2 * p + hf);
                 if (j < 0 || j >= g.nt) j = 0;
                 vmask = valid_slot_mask(g, tile_coord(g, j));
@@ -263,28 +251,11 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tmem_ld_16x32bx2_x16<64>(tS + 32, *reinterpret_cast<float(*)[16]>(&s[32]));
             tmem_ld_16x32bx2_x16<64>(tS + 48, *reinterpret_cast<float(*)[16]>(&s[48]));
             tmem_wait_ld();
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                s[c] = ((vmask >> c) & 1ull) ? s[c] * scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[c]);
-            }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const bool resc = mx > m_run + 8.f;
-            const float m_new = resc ? mx : m_run;
-            const float alpha = resc ? ex2(m_run - m_new) : 1.f;
-            m_run = m_new;
-            float ls = 0.f;
             uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(s[2 * c] - m_new), p1 = ex2(s[2 * c + 1] - m_new);
-                pk[c] = pack_bf16x2(p0, p1);
-                // normalise by the weights the tensor core will actually use
-                // (bf16-rounded), so O / l is an exactly normalised average
-                ls += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
-            }
-            l_run = l_run * alpha + ls;
+            bool resc;
+            const bool masked = __any_sync(0xffffffffu, vmask != ~0ull);
+            const float alpha = masked ? softmax_step<true>(s, vmask, scale_log2, sm, resc, pk)
+                                       : softmax_step<false>(s, vmask, scale_log2, sm, resc, pk);
             tmem_st_16x32bx2_x32(tS, pk);
             if (p > 0 && __any_sync(0xffffffffu, resc)) {
                 // O holds PV up to pair p-1: wait for it, then rescale in place
@@ -367,7 +338,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         // ------------------------------------------------------------ epilogue
         if (ok) {
             tc_fence_after();
-            const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+            const float l = sm.l_run + __shfl_xor_sync(0xffffffffu, sm.l_run, 16);
             const float inv = 1.f / l;
             const float inv_den = 1.f / den;
             const TileCoord qc = tile_coord(g, i);
@@ -414,7 +385,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-template <int D>
+template <int D, bool LIN>
 static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     using C = FineCfg<D>;
     static int configured_device = -1;   // per process: attribute set once per device
@@ -422,22 +393,32 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(fine_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(fine_attn_kernel<D, LIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
     const long long rows = (long long)a.g.B * a.g.heads * a.g.nt;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    fine_attn_kernel<D><<<(unsigned)rows, 192, C::SMEM_BYTES, stream>>>(
-        *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, a.lin_S, a.lin_z,
+    const int ragged = (a.g.T % a.g.tt) || (a.g.H % a.g.th) || (a.g.W % a.g.tw);
+    fine_attn_kernel<D, LIN><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
+        *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged, a.lin_S, a.lin_z,
         reinterpret_cast<__nv_bfloat16*>(a.out), a.status);
     return cudaGetLastError();
 }
 
+cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
+    const bool lin = a.lin_S != nullptr;
+    if (a.g.d == 128) return lin ? launch_fine_impl<128, true>(a, stream) : launch_fine_impl<128, false>(a, stream);
+    return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
+}
+
+#ifndef VSA_FINE_USE_PAIR
+#define VSA_FINE_USE_PAIR 0
+#endif
 cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) {
-    if (a.g.d == 128) return launch_fine_impl<128>(a, stream);
-    return launch_fine_impl<64>(a, stream);
+    if (a.lin_S != nullptr || !VSA_FINE_USE_PAIR) return launch_fine_single(a, stream);
+    return launch_fine_pair(a, stream);
 }
 
 int fine_smem_bytes(int d) { return d == 128 ? FineCfg<128>::SMEM_BYTES : FineCfg<64>::SMEM_BYTES; }

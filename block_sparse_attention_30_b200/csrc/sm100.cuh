@@ -66,6 +66,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// Non-blocking probe of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait by polling with test_wait: the thread never sleeps, so it
+// reacts to the phase flip within a few cycles (for the single MMA-issuing
+// thread, whose idle time is tensor-core idle time).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                               const volatile int* abort) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long t0 = clock64();
+    while (true) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) return false;
+    }
+}
+
+// Wait without looking at the abort flag (used to drain in-flight work).
+__device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) return false;
+    return true;
+}
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (tensor core / TMA) reads of the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -105,6 +105,8 @@ SMALL = [
     (8, 16, 16, 2, 128, 32, (4, 4, 4)),     # k = nt (dense)
     (8, 12, 20, 2, 64, 7, (2, 4, 8)),       # non-cubic tile shape
     (6, 10, 9, 2, 128, 9, (4, 4, 4)),       # ragged, several pairs + odd tail
+    (12, 4, 4, 1, 128, 2, (4, 4, 4)),       # odd number of query cubes (3 rows)
+    (12, 4, 4, 1, 64, 3, (4, 4, 4)),        # odd rows, d = 64, k = nt
 ]
 
 
