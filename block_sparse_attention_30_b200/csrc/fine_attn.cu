@@ -7,19 +7,21 @@
 //
 // One CTA owns one query cube (b, head, i) and runs online softmax over its
 // top-k key cubes, two cubes (128 keys) per step:
-//   * warp 4 (one lane) loads Q once and the K / V cube pairs into shared
-//     memory rings with 5-D TMA boxes cut straight from the [B][N][heads][d]
-//     tensors (box = d-chunk x tw x th x tt), so the cube gather costs no
-//     extra pass and ragged edge cubes arrive zero-filled;
+//   * warp 4 (one lane) loads Q once and the K cube pairs, warp 6 (one lane)
+//     the V cube pairs, into shared-memory rings with 5-D TMA boxes cut
+//     straight from the [B][N][heads][d] tensors (box = d-chunk x tw x th x
+//     tt), so the cube gather costs no extra pass and ragged edge cubes arrive
+//     zero-filled;
 //   * warp 5 (one lane) issues the tensor-core work: S = Q K^T (M=64 queries,
 //     N=128 keys, A and B from shared memory) into TMEM, then, once softmax
 //     has written P as bf16 over S in TMEM, O += P V (A = P from TMEM,
 //     B = V from shared memory, MN-major);
 //   * warps 0-3 (one TMEM sub-partition each; rows 16w..16w+15, each row
 //     split in two 64-column halves over lanes t and t+16) do the fp32 online
-//     softmax in the exp2 domain, rescale O in TMEM only when a row maximum
-//     grows by more than 2^8, and finally write O / l as bf16 in grid order
-//     (the cube scatter, fused), skipping padded slots.
+//     softmax in the exp2 domain (softmax_step.cuh), rescale O in TMEM only
+//     when a row maximum grows by more than 2^8, and finally write O / l (+ the
+//     linear-branch term) as bf16 in grid order (the cube scatter, fused),
+//     skipping padded slots.
 // Two CTAs share an SM (256 TMEM columns and ~112 KB of shared memory each),
 // so one CTA's softmax overlaps the other's MMAs.
 //
@@ -413,13 +415,7 @@ cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
 }
 
-#ifndef VSA_FINE_USE_PAIR
-#define VSA_FINE_USE_PAIR 0
-#endif
-cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) {
-    if (a.lin_S != nullptr || !VSA_FINE_USE_PAIR) return launch_fine_single(a, stream);
-    return launch_fine_pair(a, stream);
-}
+cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) { return launch_fine_single(a, stream); }
 
 int fine_smem_bytes(int d) { return d == 128 ? FineCfg<128>::SMEM_BYTES : FineCfg<64>::SMEM_BYTES; }
 

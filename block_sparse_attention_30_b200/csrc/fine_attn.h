@@ -21,12 +21,8 @@ struct FineArgs {
     int* status;                 // device status word
 };
 
-// Dispatch: the two-cube persistent kernel (fine_pair.cu) for the sparse
-// branch alone, the one-cube kernel (fine_attn.cu) when the linear branch is
-// fused into the epilogue.
 cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream);
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream);
-cudaError_t launch_fine_pair(const FineArgs& a, cudaStream_t stream);
 int fine_smem_bytes(int d);
 
 }  // namespace vsa
