@@ -11,8 +11,8 @@
 //   pool_kernel    one CTA per (cube, batch, q|k): 16-byte vector loads of the
 //                  cube's valid token rows (all heads at once), fp64 sums,
 //                  divide by the valid count -> pooled [2][B][heads][nt][d].
-//   coarse_kernel  per (b, head) a 64x64 tile of C = Qp Kp^T / sqrt(d) with a
-//                  4x4 register tile per thread -> scores [B][heads][nt][nt].
+//   coarse_kernel  per (b, head) a 64x64 tile of C = Qp Kp^T / sqrt(d) with an
+//                  8x4 register tile per thread -> scores [B][heads][nt][nt].
 //   topk_kernel    one warp per score row: 8-pass MSD radix select on
 //                  order-preserving 64-bit keys finds the k-th largest score,
 //                  then a ballot sweep in ascending j emits the kept cubes
@@ -27,7 +27,16 @@ namespace vsa {
 
 // ------------------------------------------------------------------ pooling
 
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 raw) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += (double)__uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += (double)__uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+
+__global__ void __launch_bounds__(320)
 pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g,
             double* __restrict__ pooled) {
     const int j = blockIdx.x, b = blockIdx.y, which = blockIdx.z;
@@ -38,26 +47,32 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, cons
     const double count = (double)(vt * vh * vw);
     const int row_elems = g.heads * g.d;              // one token: all heads
     const int nvec = row_elems / 8;
+    const bool full444 = vt == 4 && vh == 4 && vw == 4 && g.tt == 4 && g.th == 4 && g.tw == 4;
     double* out = pooled + ((long long)which * g.B + b) * g.heads * (long long)g.nt * g.d;
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
         double acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-        for (int dt = 0; dt < vt; ++dt)
-            for (int dh = 0; dh < vh; ++dh) {
-                const long long n0 = ((long long)(t0 + dt) * g.H + (h0 + dh)) * g.W + w0;
-                const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)b * g.N + n0) * row_elems) + v;
-#pragma unroll 4
-                for (int dw = 0; dw < vw; ++dw) {
-                    const uint4 raw = __ldg(src + (long long)dw * nvec);
-                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        if (full444) {
+            // all 64 tokens valid: 16 loads in flight per layer
+            for (int dt = 0; dt < 4; ++dt) {
+                uint4 raw[16];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        acc[2 * e] += (double)__uint_as_float(w[e] << 16);
-                        acc[2 * e + 1] += (double)__uint_as_float(w[e] & 0xffff0000u);
-                    }
+                for (int r = 0; r < 16; ++r) {
+                    const long long n = ((long long)(t0 + dt) * g.H + (h0 + (r >> 2))) * g.W + w0 + (r & 3);
+                    raw[r] = __ldg(reinterpret_cast<const uint4*>(x + ((long long)b * g.N + n) * row_elems) + v);
                 }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) add_bf16x8(acc, raw[r]);
             }
+        } else {
+            for (int dt = 0; dt < vt; ++dt)
+                for (int dh = 0; dh < vh; ++dh) {
+                    const long long n0 = ((long long)(t0 + dt) * g.H + (h0 + dh)) * g.W + w0;
+                    const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)b * g.N + n0) * row_elems) + v;
+                    for (int dw = 0; dw < vw; ++dw) add_bf16x8(acc, __ldg(src + (long long)dw * nvec));
+                }
+        }
         const int e0 = v * 8, head = e0 / g.d, c0 = e0 % g.d;
         double* dst = out + ((long long)head * g.nt + j) * g.d + c0;
 #pragma unroll
@@ -67,25 +82,27 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, cons
 
 // ------------------------------------------------------------ coarse scores
 // C[i][j] = (sum_c Qp[i][c] Kp[j][c]) / sqrt(d), per (b, head); 64x64 tiles,
-// 256 threads, 4x4 outputs per thread, operands staged 16 features at a time.
-__global__ void __launch_bounds__(256)
+// 128 threads, 8 (rows) x 4 (cols) fp64 outputs per thread, operands staged
+// 16 features at a time, read back with 16-byte shared loads.  The features
+// are summed in increasing order, as in the exact definition.
+__global__ void __launch_bounds__(128)
 coarse_kernel(const double* __restrict__ qp, const double* __restrict__ kp, const Grid g,
               const double inv_sqrt_d, double* __restrict__ scores) {
-    __shared__ double As[16][64 + 1];
-    __shared__ double Bs[16][64 + 1];
+    __shared__ __align__(16) double As[16][64 + 2];
+    __shared__ __align__(16) double Bs[16][64 + 2];
     const int bh = blockIdx.z;
     const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
     const int nt = g.nt, d = g.d;
     const double* Q = qp + (long long)bh * nt * d;
     const double* K = kp + (long long)bh * nt * d;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    double acc[4][4];
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;     // 16 column groups x 8 row groups
+    double acc[8][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[a][c] = 0.0;
     for (int e0 = 0; e0 < d; e0 += 16) {
-        for (int l = threadIdx.x; l < 64 * 16; l += 256) {
+        for (int l = threadIdx.x; l < 64 * 16; l += 128) {
             const int rr = l / 16, ee = l % 16;
             As[ee][rr] = (i0 + rr < nt) ? Q[(long long)(i0 + rr) * d + e0 + ee] : 0.0;
             Bs[ee][rr] = (j0 + rr < nt) ? K[(long long)(j0 + rr) * d + e0 + ee] : 0.0;
@@ -93,11 +110,19 @@ coarse_kernel(const double* __restrict__ qp, const double* __restrict__ kp, cons
         __syncthreads();
 #pragma unroll
         for (int ee = 0; ee < 16; ++ee) {
-            double a[4], bv[4];
+            double a[8], bv[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) { a[u] = As[ee][ty + 16 * u]; bv[u] = Bs[ee][tx + 16 * u]; }
+            for (int u = 0; u < 4; ++u) {
+                const double2 t2 = *reinterpret_cast<const double2*>(&As[ee][8 * ty + 2 * u]);
+                a[2 * u] = t2.x; a[2 * u + 1] = t2.y;
+            }
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 2; ++u) {
+                const double2 t2 = *reinterpret_cast<const double2*>(&Bs[ee][4 * tx + 2 * u]);
+                bv[2 * u] = t2.x; bv[2 * u + 1] = t2.y;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
 #pragma unroll
                 for (int w = 0; w < 4; ++w) acc[u][w] = fma(a[u], bv[w], acc[u][w]);
         }
@@ -105,12 +130,12 @@ coarse_kernel(const double* __restrict__ qp, const double* __restrict__ kp, cons
     }
     double* S = scores + (long long)bh * nt * nt;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int ii = i0 + ty + 16 * u;
+    for (int u = 0; u < 8; ++u) {
+        const int ii = i0 + 8 * ty + u;
         if (ii >= nt) continue;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            const int jj = j0 + tx + 16 * w;
+            const int jj = j0 + 4 * tx + w;
             if (jj < nt) S[(long long)ii * nt + jj] = acc[u][w] * inv_sqrt_d;
         }
     }
@@ -220,13 +245,13 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     const Grid& g = a.g;
     double* pooled = reinterpret_cast<double*>(a.scratch);
     double* scores = pooled + 2ull * g.B * g.heads * g.nt * g.d;
-    pool_kernel<<<dim3(g.nt, g.B, 2), 256, 0, stream>>>(a.q, a.k, g, pooled);
+    pool_kernel<<<dim3(g.nt, g.B, 2), 320, 0, stream>>>(a.q, a.k, g, pooled);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const double* qp = pooled;
     const double* kp = pooled + (size_t)g.B * g.heads * g.nt * g.d;
     const int tiles = ceil_div_i(g.nt, 64);
-    coarse_kernel<<<dim3(tiles, tiles, g.B * g.heads), 256, 0, stream>>>(qp, kp, g, 1.0 / sqrt((double)g.d), scores);
+    coarse_kernel<<<dim3(tiles, tiles, g.B * g.heads), 128, 0, stream>>>(qp, kp, g, 1.0 / sqrt((double)g.d), scores);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int wpc = topk_warps_per_cta(g.nt);
