@@ -108,7 +108,7 @@ def gpu_step_fn(w, q, k, v, out, attn, fine_events):
     def step(record_fine=False):
         ops.vsa_select_blocks(q, k, w.T, w.H, w.W, w.topk, attn.block_idx, attn.workspace, w.tile)
         if w.linear:
-            ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W)
+            ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W, attn.workspace)
         if record_fine:
             fine_events[0].record()
         ops.vsa_sparse_attn_fwd(q, k, v, attn.block_idx, out, w.T, w.H, w.W, w.topk,

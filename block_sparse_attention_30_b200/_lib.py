@@ -27,7 +27,7 @@ SIGNATURES = {
     "vsa_gather_tiles": (_i, [_p, _p] + _SHAPE + [_p]),
     "vsa_scatter_tiles": (_i, [_p, _p] + _SHAPE + [_p]),
     "vsa_select_blocks": (_i, [_p, _p] + _SHAPE + [_i, _p, _p, _sz, _p]),
-    "vsa_linear_branch_fwd": (_i, [_p, _p, _p, _p] + [_i] * 6 + [_p]),
+    "vsa_linear_branch_fwd": (_i, [_p, _p, _p, _p] + [_i] * 6 + [_p, _sz, _p]),
     "vsa_sparse_attn_fwd": (_i, [_p] * 7 + _SHAPE + [_i, _p, _sz, _p]),
     "vsa_device_status": (_i, [_p, _p]),
     "vsa_select_blocks_noalloc": (_i, [_p, _p] + _SHAPE + [_i, _p, _p]),

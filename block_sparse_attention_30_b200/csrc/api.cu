@@ -146,14 +146,19 @@ vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int he
 
 vsa_status vsa_linear_branch_fwd(const vsa_bf16* k, const vsa_bf16* v, float* lin_S, float* lin_z,
                                  int B, int heads, int head_dim, int T, int H, int W,
-                                 vsa_stream_t stream) {
+                                 void* workspace, size_t workspace_bytes, vsa_stream_t stream) {
     // the tile shape does not enter the linear branch; any valid one will do
     vsa_status s = check_shape(B, heads, head_dim, T, H, W, 4, 4, 4);
     if (s != VSA_OK) return s;
     if (!aligned16(k) || !aligned16(v) || !aligned16(lin_S) || !aligned16(lin_z))
         return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes) return VSA_ERR_WORKSPACE;
+    auto fn = encode_fn();
+    if (!fn) return VSA_ERR_CUDA;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, 4, 4, 4);
-    return from_cuda(vsa::launch_linear_state(g, k, v, lin_S, lin_z, (cudaStream_t)stream));
+    return from_cuda(vsa::launch_linear_state(g, k, v, lin_S, lin_z, static_cast<int*>(workspace),
+                                              (cudaStream_t)stream, fn));
 }
 
 vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,

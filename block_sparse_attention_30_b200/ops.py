@@ -80,11 +80,11 @@ def vsa_select_blocks_noalloc(q, k, T, H, W, topk, block_idx, tile=(4, 4, 4), st
         block_idx.data_ptr(), _stream(stream)))
 
 
-def vsa_linear_branch_fwd(k, v, lin_S, lin_z, T, H, W, stream=None):
+def vsa_linear_branch_fwd(k, v, lin_S, lin_z, T, H, W, workspace, stream=None):
     B, heads, d = _grid_of(k, T, H, W)
     _lib.check("vsa_linear_branch_fwd", _lib.lib().vsa_linear_branch_fwd(
         k.data_ptr(), v.data_ptr(), lin_S.data_ptr(), lin_z.data_ptr(), B, heads, d, T, H, W,
-        _stream(stream)))
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
 
 
 def vsa_sparse_attn_fwd(q, k, v, block_idx, out, T, H, W, topk, workspace, lin_S=None, lin_z=None,
@@ -131,7 +131,8 @@ class BlockSparseVideoAttention:
         vsa_select_blocks(q, k, self.T, self.H, self.W, self.topk, self.block_idx, self.workspace,
                           self.tile, stream)
         if self.linear:
-            vsa_linear_branch_fwd(k, v, self.lin_S, self.lin_z, self.T, self.H, self.W, stream)
+            vsa_linear_branch_fwd(k, v, self.lin_S, self.lin_z, self.T, self.H, self.W,
+                                  self.workspace, stream)
         vsa_sparse_attn_fwd(q, k, v, self.block_idx, out, self.T, self.H, self.W, self.topk,
                             self.workspace, self.lin_S, self.lin_z, self.tile, stream)
         return out

@@ -114,10 +114,13 @@ vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int he
 /* Linear-branch state (SparkDiffusion RoLA, paragraph 3; TurboDiffusion SLA,
  * "稀疏、蒸馏与全链路量化"): lin_S[B][heads][d][d] = sum_n phi(k_n)^T v_n and
  * lin_z[B][heads][d] = sum_n phi(k_n) over all N tokens, phi = elu + 1,
- * fp32 accumulation.  Both outputs are fully overwritten. */
+ * fp32 accumulation (phi split into bf16 hi + lo parts on the tensor cores).
+ * Both outputs are fully overwritten.  The workspace (vsa_workspace_bytes()
+ * of any tile shape, only its status word is used) receives device faults. */
 vsa_status vsa_linear_branch_fwd(const vsa_bf16* k, const vsa_bf16* v, float* lin_S,
                                  float* lin_z, int B, int heads, int head_dim, int T, int H,
-                                 int W, vsa_stream_t stream);
+                                 int W, void* workspace, size_t workspace_bytes,
+                                 vsa_stream_t stream);
 
 /* Fine pass ("2. 视频稀疏注意力VSA": evaluate only the weights of the kept
  * blocks, exactly, Flash-Attention style).  For every valid query token of

@@ -98,8 +98,9 @@ def test_fine_argument_validation(L):
 def test_other_entry_points_validate(L):
     assert L.vsa_gather_tiles(None, FAKE, *SHAPE, None) == INVALID
     assert L.vsa_scatter_tiles(FAKE, FAKE + 4, *SHAPE, None) == INVALID
-    assert L.vsa_linear_branch_fwd(FAKE, FAKE, None, FAKE, 1, 2, 128, 4, 8, 8, None) == INVALID
-    assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 32, 4, 8, 8, None) == UNSUPPORTED
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, None, FAKE, 1, 2, 128, 4, 8, 8, FAKE, 1024, None) == INVALID
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 32, 4, 8, 8, FAKE, 1024, None) == UNSUPPORTED
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 128, 4, 8, 8, None, 1024, None) == WORKSPACE
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID

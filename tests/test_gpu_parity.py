@@ -267,7 +267,9 @@ def test_linear_state_small(ops):
     kd, vd = c.k.cuda(), c.v.cuda()
     S = torch.empty((1, 3, 128, 128), dtype=torch.float32, device="cuda")
     z = torch.empty((1, 3, 128), dtype=torch.float32, device="cuda")
-    ops.vsa_linear_branch_fwd(kd, vd, S, z, c.T, c.H, c.W)
+    ws = ops.new_workspace(1, 3, 128, c.T, c.H, c.W, 1)
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, c.T, c.H, c.W, ws)
+    assert ops.vsa_device_status(ws) == 0
     Sr, zr = O.linear_state(c.k, c.v, 1, 3, 128, c.T * c.H * c.W)
     np.testing.assert_allclose(S.cpu().double().numpy(), Sr, rtol=1e-4, atol=1e-3)
     np.testing.assert_allclose(z.cpu().double().numpy(), zr, rtol=1e-4, atol=1e-3)
@@ -281,7 +283,7 @@ def test_linear_branch_small_full(ops, case):
     idx, ws = run_select(ops, c, qd, kd)
     S = torch.empty((1, heads, d, d), dtype=torch.float32, device="cuda")
     z = torch.empty((1, heads, d), dtype=torch.float32, device="cuda")
-    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W)
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
     out = run_fine(ops, c, qd, kd, vd, idx, ws, lin=(S, z))
     N = T * H * W
     ref = O.fine(c.q, c.k, c.v, idx.cpu().numpy(), 1, heads, d, T, H, W)
