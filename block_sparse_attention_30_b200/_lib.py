@@ -31,6 +31,7 @@ SIGNATURES = {
     "vsa_sparse_attn_fwd": (_i, [_p] * 7 + _SHAPE + [_i, _p, _sz, _p]),
     "vsa_device_status": (_i, [_p, _p]),
     "vsa_select_blocks_noalloc": (_i, [_p, _p] + _SHAPE + [_i, _p, _p]),
+    "vsa_selftest_wait_timeout": (_i, [_p, _sz, ctypes.c_uint, _p]),
 }
 
 # VSA_NOALLOC_SELECT_SCRATCH_BYTES of include/vsa.h

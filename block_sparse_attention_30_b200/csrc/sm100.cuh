@@ -53,17 +53,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false when
-// the wait gave up after VSA_WAIT_LIMIT_CYCLES (or immediately if *abort is
-// already set by another role of the CTA).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort) {
+// the wait gave up after `limit` SM clock cycles (or as soon as *abort is set
+// by another role of the CTA).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
+                                              const volatile int* abort,
+                                              unsigned long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) return false;
+        if (clock64() - t0 > limit) return false;
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* abort) {
+    return mbar_wait_for(bar, parity, abort, VSA_WAIT_LIMIT_CYCLES);
 }
 
 // Non-blocking probe of a phase (never suspends the thread).

@@ -138,6 +138,15 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
                                int topk, void* workspace, size_t workspace_bytes,
                                vsa_stream_t stream);
 
+/* Self-test of the device failure path (no counterpart on the pages): a
+ * one-warp kernel waits on a barrier nobody arrives at, gives up after
+ * `limit_cycles` SM clock cycles exactly as the library's kernels do, and
+ * records VSA_ERR_TIMEOUT in the workspace status word, which
+ * vsa_device_status then returns.  No fault, trap or hang is involved; the
+ * context stays usable.  limit_cycles > 0. */
+vsa_status vsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                     unsigned int limit_cycles, vsa_stream_t stream);
+
 /* Synchronise `stream`, then report and clear the device status word the
  * kernels of this workspace wrote: VSA_OK, VSA_ERR_TIMEOUT or
  * VSA_ERR_DEVICE_CHECK (VSA_ERR_CUDA if the stream itself failed). */

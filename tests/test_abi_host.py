@@ -104,6 +104,8 @@ def test_other_entry_points_validate(L):
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID
+    assert L.vsa_selftest_wait_timeout(None, 1024, 1000, None) == WORKSPACE
+    assert L.vsa_selftest_wait_timeout(FAKE, 1024, 0, None) == INVALID
 
 
 def test_library_has_no_oracle_dependency():

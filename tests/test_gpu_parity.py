@@ -124,6 +124,27 @@ def test_small_grids_select_and_fine(ops, case):
     check_close(to_f64(out), ref)
 
 
+@pytest.mark.parametrize("case", [(5, 6, 7, 3, 128, 3), (4, 8, 12, 2, 64, 4)])
+def test_batch_of_two(ops, case):
+    """B = 2: batch indexing of the pooled means, TMA boxes and outputs."""
+    T, H, W, heads, d, topk = case
+    c = Small(T, H, W, heads, d, topk, seed=17, B=2)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    ref_idx, scores = O.select(c.q, c.k, 2, heads, d, T, H, W, topk, c.tile, with_scores=True)
+    check_indices(idx.cpu().numpy(), ref_idx, scores)
+    S = torch.empty((2, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((2, heads, d), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
+    for lin in (None, (S, z)):
+        out = run_fine(ops, c, qd, kd, vd, idx, ws, lin=lin)
+        ref = O.fine(c.q, c.k, c.v, idx.cpu().numpy(), 2, heads, d, T, H, W, c.tile)
+        if lin is not None:
+            Sr, zr = O.linear_state(c.k, c.v, 2, heads, d, T * H * W)
+            ref = ref + O.linear_apply(c.q, Sr, zr, 2, heads, d, T * H * W)
+        check_close(to_f64(out), ref)
+
+
 def test_dense_limit_matches_sdpa(ops):
     """k = nt: the fine pass is dense attention (torch SDPA as reference)."""
     T, H, W, heads, d = 8, 16, 16, 2, 128
@@ -158,6 +179,23 @@ def test_bad_index_is_reported_not_faulted(ops):
     ops.vsa_sparse_attn_fwd(qd, kd, vd, bad, out, c.T, c.H, c.W, 2, ws)
     assert ops.vsa_device_status(ws) == 6          # VSA_ERR_DEVICE_CHECK
     assert ops.vsa_device_status(ws) == 0          # cleared by the read
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(ops):
+    """The device failure path: a wait nobody satisfies gives up after its
+    bound, the status word says VSA_ERR_TIMEOUT, and the next call works."""
+    from block_sparse_attention_30_b200 import _lib
+    c = Small(4, 8, 8, 2, 128, 2, seed=6)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = _lib.lib().vsa_selftest_wait_timeout(ws.data_ptr(), ws.numel(), 2_000_000, stream)
+    assert rc == 0
+    assert ops.vsa_device_status(ws) == 5          # VSA_ERR_TIMEOUT
+    assert ops.vsa_device_status(ws) == 0          # cleared by the read
+    out = run_fine(ops, c, qd, kd, vd, idx, ws)    # context still usable
+    ref = O.fine(c.q, c.k, c.v, idx.cpu().numpy(), 1, 2, 128, c.T, c.H, c.W)
+    check_close(to_f64(out), ref)
 
 
 def test_repeated_calls_are_deterministic(ops):
