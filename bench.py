@@ -41,6 +41,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+FINE_SOURCES = ["fine_attn.cu", "softmax_step.cuh", "sm100.cuh", "common.cuh"]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "fine_attn_wan1.3b_480p.md")
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per fine launch from the committed ncu summary, or None when
+    the summary lacks this workload or the kernel sources changed since."""
+    import hashlib
+    import re
+    if not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    text = open(TRAFFIC_PROFILE, encoding="utf-8").read()
+    m_hash = re.search(r"^sources_sha256: ([0-9a-f]+)$", text, re.M)
+    m_val = re.search(r"^traffic_bytes_per_launch\[%s\]: (\d+)$" % re.escape(workload), text, re.M)
+    if not m_hash or not m_val:
+        return None
+    csrc = os.path.join(ROOT, "block_sparse_attention_30_b200", "csrc")
+    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in FINE_SOURCES))
+    return int(m_val.group(1)) if h.hexdigest()[:16] == m_hash.group(1) else None
+
+
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(
         os.environ.get("WORLD_SIZE", 1))
@@ -235,7 +256,9 @@ def run_gpu(args):
                 "achieved": round(fine_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(fine_tflops / peak, 4),
                 "peak_source": f"{src} bf16_tflops (burst)",
-                "traffic": args.traffic,
+                "traffic": args.traffic if args.traffic is not None else profiled_traffic(w.name),
+                "traffic_unit": "bytes per launch (ncu dram read+write)",
+                "algorithmic_bytes": 4 * w.B * w.N * w.heads * w.head_dim * 2,
             },
             "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                     "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
