@@ -299,6 +299,75 @@ def run_gpu(args):
         torch.distributed.destroy_process_group()
 
 
+# ------------------------------------------------------------ per-kernel lines
+
+def run_kernels(args):
+    """One JSON line per hot-path kernel on one workload: its time (CUDA
+    events, median of `steps` calls, L2 flushed before each) against its own
+    roofline -- HBM GB/s for the copies, pooling and the linear state, tensor
+    TFLOP/s for the fine pass."""
+    from block_sparse_attention_30_b200 import build, ops
+    build.build()
+    dev = torch.device("cuda", 0)
+    w = WORKLOADS[args.workload]
+    q_h, k_h, v_h = synth.make_workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    attn = ops.BlockSparseVideoAttention(w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                                         linear=True, device=dev)
+    out = torch.empty_like(q)
+    nt = w.num_tiles
+    tiles = torch.empty((w.B, w.heads, nt, 64, w.head_dim), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks, src = load_peaks()
+    elem = w.B * w.N * w.heads * w.head_dim * 2            # bytes of one [B][N][heads][d] tensor
+    tile_bytes = tiles.numel() * 2
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(max(args.steps, 3)):
+            flush.fill_(i & 255)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2]
+
+    rows = [
+        ("gather_tiles (a1)", lambda: ops.vsa_gather_tiles(q, tiles, w.T, w.H, w.W, w.tile),
+         "hbm", elem + tile_bytes),
+        ("scatter_tiles (a7)", lambda: ops.vsa_scatter_tiles(tiles, out, w.T, w.H, w.W, w.tile),
+         "hbm", 2 * elem),
+        ("select_blocks (a2-a4)", lambda: ops.vsa_select_blocks(q, k, w.T, w.H, w.W, w.topk,
+                                                                  attn.block_idx, attn.workspace, w.tile),
+         "hbm", 2 * elem + w.B * w.heads * nt * w.topk * 4),
+        ("linear_branch_fwd (a6 state)", lambda: ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W,
+                                                                           attn.workspace),
+         "hbm", 2 * elem),
+        ("sparse_attn_fwd (a1+a5+a7 fused)", lambda: ops.vsa_sparse_attn_fwd(q, k, v, attn.block_idx, out, w.T, w.H, w.W,
+                                                                            w.topk, attn.workspace, tile=w.tile),
+         "tensor", w.fine_flops()),
+        ("sparse_attn_fwd + linear apply (a5+a6)", lambda: ops.vsa_sparse_attn_fwd(
+            q, k, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, attn.lin_S, attn.lin_z, w.tile),
+         "tensor", w.fine_flops()),
+    ]
+    for name, fn, bound, units in rows:
+        ms = timed(fn)
+        if bound == "hbm":
+            achieved, peak, unit = units / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            achieved, peak, unit = units / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        print(json.dumps({"kernel": name, "workload": w.name, "ms": round(ms, 4), "bound": bound,
+                          "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                          "frac": round(achieved / peak, 4), "peak_source": src,
+                          "algorithmic": units}), flush=True)
+    if attn.status() != 0:
+        raise RuntimeError("device status not OK")
+
+
 # -------------------------------------------------------------------- oracle
 
 def oracle_sample(w, q, k, v, heads):
@@ -368,6 +437,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels", action="store_true",
+                    help="print one roofline line per hot-path kernel instead of the step line")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per fine launch from an ncu capture (reported as-is)")
     args = ap.parse_args()
@@ -377,6 +448,10 @@ def main():
             sys.exit("for --gpus > 1 launch with torch.distributed.run --nproc-per-node N")
     if args.impl == "reference":
         run_reference(args)
+    elif args.kernels:
+        if not torch.cuda.is_available():
+            sys.exit("bench.py --kernels needs a CUDA device")
+        run_kernels(args)
     else:
         if not torch.cuda.is_available():
             sys.exit("bench.py needs a CUDA device for --impl ours")

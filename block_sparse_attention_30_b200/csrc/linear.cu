@@ -15,7 +15,8 @@
 // layout, and accumulate z in fp32; one thread issues
 //     S(TMEM, M = d features a, N = d features c) += phi_hi^T V + phi_lo^T V
 // (A = phi(K)^T and B = V, both read MN-major from shared memory, M = 128).
-// Three stages keep two steps of loads in flight while step t is computed.  At the
+// Four 48 KB stages (phi hi overwrites K in place) keep three steps of loads
+// in flight while step t is computed.  At the
 // end each CTA adds its partial S (read from TMEM) and z into the zeroed
 // outputs with fp32 atomics, so the summation order across CTAs varies from
 // run to run at the fp32 rounding level.
@@ -33,8 +34,8 @@ template <int D>
 struct LinCfg {
     static constexpr int NCH = D / 64;                    // 64-feature chunks
     static constexpr int TILE = 64 * D * 2;               // one 64-token tile (bf16)
-    static constexpr int STAGE = 4 * TILE;                // K staging, V, phi hi, phi lo
-    static constexpr int NST = 3;
+    static constexpr int STAGE = 3 * TILE;                // K -> phi hi (in place), V, phi lo
+    static constexpr int NST = 4;
     static constexpr int BAR_BYTES = 128;
     static constexpr int SMEM_BYTES = NST * STAGE + BAR_BYTES;
     static constexpr int TMEM_COLS = D < 32 ? 32 : D;     // fp32 accumulator, D columns
@@ -117,13 +118,13 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(stage_ptr(s, 1));
 #pragma unroll
-                for (int part = 2; part < 4; ++part) {
+                for (int part = 0; part < 3; part += 2) {     // phi hi (part 0), phi lo (part 2)
                     const uint32_t a_addr = smem_u32(stage_ptr(s, part));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {         // 16 tokens per MMA
                         const uint64_t a = smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
                         const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, 8192, 1024);
-                        mma_bf16_ss(tbase, a, bd, id, (t > 0 || part > 2 || kk > 0));
+                        mma_bf16_ss(tbase, a, bd, id, (t > 0 || part > 0 || kk > 0));
                     }
                 }
                 mma_commit(&bars->done[s]);
@@ -154,8 +155,8 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->full[s], (t / C::NST) & 1, abort_flag))) { ok = false; break; }
             const int valid = (int)min(64ll, n_end - (n_begin + 64ll * t));
             const uint8_t* kt = stage_ptr(s, 0);
-            uint8_t* hi = stage_ptr(s, 2);
-            uint8_t* lo = stage_ptr(s, 3);
+            uint8_t* hi = stage_ptr(s, 0);                  // in place: each thread rewrites its own units
+            uint8_t* lo = stage_ptr(s, 2);
             for (int r = r0; r < 64; r += rows_per_pass) {
                 const uint32_t off = chunk * 8192 + r * 128 + ((uu ^ (r & 7)) << 4);
                 uint4 raw = *reinterpret_cast<const uint4*>(kt + off);

@@ -7,9 +7,7 @@
 // layouts -- its TMA boxes cut cubes straight out of grid order -- but the
 // copies are part of the library for callers that keep cube-major tensors.
 //
-// One thread moves one 16-byte vector (8 bf16); consecutive threads walk the
-// d axis of one slot, then the slots of a cube, so every warp reads and writes
-// whole 128-byte lines of both layouts.  HBM-bound.
+// HBM-bound copies: every byte is read once and written once.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -17,57 +15,71 @@
 
 namespace vsa {
 
-template <bool GATHER>
+// One CTA per (cube j, batch b).  For each of the cube's slots the token row
+// -- all heads, heads*d bf16, contiguous in grid order -- is copied with
+// 16-byte vectors; in cube-major order the same vector lands in row
+// ((b*heads + head)*nt + j)*vol + slot.  Consecutive threads take consecutive
+// vectors of one row, so reads cover whole 128-byte lines of grid order and
+// writes whole d-wide rows of cube-major order.  Four slots are in flight per
+// thread.
+template <bool GATHER, int VPR>     // VPR: 16-byte vectors per (slot, head) row = d/8
 __global__ void __launch_bounds__(256)
-tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const Grid g,
-                 const long long total_vec) {
-    const int vpr = g.d / 8;                     // vectors per (slot, head) row
+tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const Grid g) {
+    const int j = blockIdx.x, b = blockIdx.y;
     const int vol = g.tt * g.th * g.tw;
-    for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < total_vec;
-         v += (long long)gridDim.x * blockDim.x) {
-        // cube-major index: (((b*heads + head)*nt + j)*vol + s)*vpr + c
-        const int c = (int)(v % vpr);
-        long long rest = v / vpr;
-        const int s = (int)(rest % vol); rest /= vol;
-        const int j = (int)(rest % g.nt); rest /= g.nt;
-        const int head = (int)(rest % g.heads);
-        const int b = (int)(rest / g.heads);
-        const int it = j / (g.nh * g.nw), ih = (j / g.nw) % g.nh, iw = j % g.nw;
-        const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
-        const int t = it * g.tt + dt, h = ih * g.th + dh, w = iw * g.tw + dw;
-        const bool valid = t < g.T && h < g.H && w < g.W;
-        const long long n = ((long long)t * g.H + h) * g.W + w;
-        const long long gi = (((long long)b * g.N + n) * g.heads + head) * vpr + c;
-        if (GATHER) {
-            dst[v] = valid ? __ldg(src + gi) : make_uint4(0, 0, 0, 0);
-        } else if (valid) {
-            dst[gi] = __ldg(src + v);
+    const int it = j / (g.nh * g.nw), ih = (j / g.nw) % g.nh, iw = j % g.nw;
+    const int row_vec = g.heads * VPR;                       // vectors per token row
+    for (int s0 = 0; s0 < vol; s0 += 4) {
+        long long n[4];
+        bool valid[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
+            const int t = it * g.tt + dt, h = ih * g.th + dh, w = iw * g.tw + dw;
+            valid[u] = s < vol && t < g.T && h < g.H && w < g.W;
+            n[u] = ((long long)t * g.H + h) * g.W + w;
+        }
+        for (int v = threadIdx.x; v < row_vec; v += blockDim.x) {
+            const int head = v / VPR, c = v % VPR;
+            const long long tile_row = (((long long)b * g.heads + head) * g.nt + j) * vol;
+            uint4 val[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const long long gi = ((long long)b * g.N + n[u]) * row_vec + v;
+                const long long ti = (tile_row + s0 + u) * VPR + c;
+                if (GATHER) val[u] = valid[u] ? __ldg(src + gi) : make_uint4(0, 0, 0, 0);
+                else val[u] = valid[u] ? __ldg(src + ti) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (s0 + u >= vol) continue;
+                const long long gi = ((long long)b * g.N + n[u]) * row_vec + v;
+                const long long ti = (tile_row + s0 + u) * VPR + c;
+                if (GATHER) dst[ti] = val[u];
+                else if (valid[u]) dst[gi] = val[u];
+            }
         }
     }
 }
 
-static unsigned copy_blocks(long long total_vec) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long want = (total_vec + 255) / 256;
-    const long long cap = (long long)sms * 8;     // 8 resident CTAs of 256 threads per SM
-    return (unsigned)(want < cap ? want : cap);
+template <bool GATHER>
+static cudaError_t launch_copy(const Grid& g, const void* src, void* dst, cudaStream_t stream) {
+    if ((long long)g.B * g.nt == 0) return cudaSuccess;
+    const dim3 grid(g.nt, g.B);
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    if (g.d == 128) tile_copy_kernel<GATHER, 16><<<grid, 256, 0, stream>>>(s, d, g);
+    else tile_copy_kernel<GATHER, 8><<<grid, 256, 0, stream>>>(s, d, g);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const Grid& g, const void* x, void* x_tiles, cudaStream_t stream) {
-    const long long total = (long long)g.B * g.heads * g.nt * (g.tt * g.th * g.tw) * (g.d / 8);
-    if (total == 0) return cudaSuccess;
-    tile_copy_kernel<true><<<copy_blocks(total), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(x_tiles), g, total);
-    return cudaGetLastError();
+    return launch_copy<true>(g, x, x_tiles, stream);
 }
 
 cudaError_t launch_scatter(const Grid& g, const void* x_tiles, void* x, cudaStream_t stream) {
-    const long long total = (long long)g.B * g.heads * g.nt * (g.tt * g.th * g.tw) * (g.d / 8);
-    if (total == 0) return cudaSuccess;
-    tile_copy_kernel<false><<<copy_blocks(total), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x_tiles), reinterpret_cast<uint4*>(x), g, total);
-    return cudaGetLastError();
+    return launch_copy<false>(g, x_tiles, x, stream);
 }
 
 }  // namespace vsa
