@@ -248,7 +248,8 @@ def run_gpu(args):
         fine_tflops = flops / (fine_avg_ms * 1e-3) / 1e12
         peaks, src = load_peaks()
         peak = peaks["bf16_tflops"]
-        launches_per_step = 4 + (1 if w.linear else 0)
+        # pool, coarse, top-k, fine; + linear state and the (S, z) operand pack
+        launches_per_step = 4 + (2 if w.linear else 0)
         result = {
             "metric": METRIC,
             "value": round(value, 2),

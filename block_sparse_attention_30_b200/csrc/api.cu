@@ -36,6 +36,11 @@ vsa::Grid grid_of(int B, int heads, int d, int T, int H, int W, int tt, int th, 
     return vsa::make_grid(B, heads, d, T, H, W, tt, th, tw);
 }
 
+// Workspace scratch the linear-branch apply needs: one operand image per (b, head).
+size_t lin_image_bytes(const vsa::Grid& g) {
+    return (size_t)g.B * g.heads * (size_t)vsa::linear_image_bytes(g.d);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -96,7 +101,9 @@ size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W, 
     if (check_shape(B, heads, head_dim, T, H, W, tt, th, tw) != VSA_OK) return 0;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return 0;
-    return kStatusBytes + vsa::select_scratch_bytes(g);
+    const size_t select = vsa::select_scratch_bytes(g);
+    const size_t image = lin_image_bytes(g);
+    return kStatusBytes + (select > image ? select : image);
 }
 
 vsa_status vsa_workspace_init(void* workspace, size_t workspace_bytes, vsa_stream_t stream) {
@@ -175,7 +182,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     if ((lin_S == nullptr) != (lin_z == nullptr)) return VSA_ERR_INVALID_ARGUMENT;
     if (lin_S && (!aligned16(lin_S) || !aligned16(lin_z))) return VSA_ERR_INVALID_ARGUMENT;
     if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
-    if (workspace_bytes < kStatusBytes) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes + (lin_S ? lin_image_bytes(g) : 0)) return VSA_ERR_WORKSPACE;
     CUtensorMap mq, mk, mv;
     if (!encode_grid_map(&mq, q, g) || !encode_grid_map(&mk, k, g) || !encode_grid_map(&mv, v, g))
         return VSA_ERR_CUDA;
@@ -186,10 +193,16 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     a.mv = &mv;
     a.block_idx = block_idx;
     a.topk = topk;
-    a.lin_S = lin_S;
-    a.lin_z = lin_z;
+    a.lin_image = nullptr;
     a.out = out;
     a.status = static_cast<int*>(workspace);
+    if (lin_S) {
+        // the bf16 hi/lo operand image of (S, z) goes into the workspace scratch
+        a.lin_image = static_cast<uint8_t*>(workspace) + kStatusBytes;
+        cudaError_t e = vsa::launch_linear_pack(g, lin_S, lin_z, const_cast<void*>(a.lin_image),
+                                                (cudaStream_t)stream);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
     return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
 }
 

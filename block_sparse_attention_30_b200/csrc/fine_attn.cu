@@ -52,7 +52,10 @@ struct FineCfg {
     static constexpr int O_COL = 0;                    // fp32 O, D columns
     static constexpr int S_COL = 128;                  // fp32 S (128 cols) / bf16 P (64 cols)
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = Q_BYTES + (NK + NV) * PAIR_BYTES + BAR_BYTES;
+    static constexpr int Z_BYTES = D * 4;              // linear branch: z (fp32)
+    static constexpr int SMEM_BYTES = Q_BYTES + (NK + NV) * PAIR_BYTES + BAR_BYTES + Z_BYTES;
+    // the linear branch's S hi + lo image must fit the K ring, phi(Q) lo the V ring
+    static_assert(4 * D * D <= NK * PAIR_BYTES && Q_BYTES <= NV * PAIR_BYTES, "linear operands");
 };
 
 template <int D>
@@ -60,7 +63,7 @@ struct FineBars {
     uint64_t q_full;
     uint64_t k_full[FineCfg<D>::NK], k_empty[FineCfg<D>::NK];
     uint64_t v_full[FineCfg<D>::NV], v_empty[FineCfg<D>::NV];
-    uint64_t s_full, p_full, o_ready, mma_done, lin_ready, lin_done;
+    uint64_t s_full, p_full, o_ready, mma_done, lin_full, lin_ready, lin_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(224, 2)
 fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                  const __grid_constant__ CUtensorMap mv, const Grid g,
                  const int32_t* __restrict__ block_idx, const int topk, const float scale_log2,
-                 const int ragged, const float* __restrict__ lin_S, const float* __restrict__ lin_z,
+                 const int ragged, const uint8_t* __restrict__ lin_image,
                  __nv_bfloat16* __restrict__ out, int* status) {
     using C = FineCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -94,13 +97,16 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const int32_t* my_idx = block_idx + row_id * topk;
     const int n_pairs = (topk + 1) >> 1;
     constexpr bool lin = LIN;
-    // Linear-branch operands reuse the K/V rings once the last PV is done:
-    //   phi(Q) hi / lo  (A, K-major like Q)        at sK, sK + Q_BYTES
-    //   S hi / lo       (B, MN-major like V pairs) at sK + 2*Q_BYTES, + D*D*2
-    uint8_t* sPhiHi = sK;
-    uint8_t* sPhiLo = sK + C::Q_BYTES;
-    uint8_t* sSHi = sK + 2 * C::Q_BYTES;
-    uint8_t* sSLo = sSHi + D * D * 2;
+    // Linear-branch operands reuse the buffers of the sparse pass:
+    //   S hi / lo (B, MN-major) + z: one bulk copy of the (b, head) image into
+    //     the K ring once the last Q K^T is done, z into its own 512 bytes;
+    //   phi(Q) hi / lo (A, K-major like Q): hi over Q in place, lo in the V
+    //     ring, once the last P V is done.
+    uint8_t* sPhiHi = sQ;
+    uint8_t* sPhiLo = sV;
+    uint8_t* sSHi = sK;
+    uint8_t* sSLo = sK + D * D * 2;
+    float* sZ = reinterpret_cast<float*>(sV + C::NV * C::PAIR_BYTES + C::BAR_BYTES);
 
     if (tid == 0) {
         bars->abort = 0;
@@ -111,6 +117,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         mbar_init(&bars->p_full, 128);
         mbar_init(&bars->o_ready, 1);
         mbar_init(&bars->mma_done, 1);
+        mbar_init(&bars->lin_full, 1);
         mbar_init(&bars->lin_ready, 128);
         mbar_init(&bars->lin_done, 1);
         fence_barrier_init();
@@ -165,11 +172,30 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 }
                 ++issued;
             }
+            bool lin_issued = false;
+            if (lin && is_k && issued == n_pairs && !*abort_flag) {
+                // the (S, z) image goes into the K ring once the last Q K^T
+                // MMAs (each stage's last use) are done
+                bool free = true;
+                for (int p = max(0, n_pairs - nst); p < n_pairs && free; ++p)
+                    free = mbar_wait(&empty[p % nst], (p / nst) & 1, abort_flag);
+                if (free) {
+                    const uint8_t* img = lin_image + (long long)bh * (4 * D * D + 4 * D);
+                    mbar_arrive_expect_tx(&bars->lin_full, 4 * D * D + 4 * D);
+                    for (int off = 0; off < 4 * D * D; off += 16384)
+                        bulk_load(sSHi + off, img + off, min(16384, 4 * D * D - off), &bars->lin_full);
+                    bulk_load(sZ, img + 4 * D * D, 4 * D, &bars->lin_full);
+                    lin_issued = true;
+                } else {
+                    fail();
+                }
+            }
             if (*abort_flag) {
                 // drain: the last load issued into each stage must land before exit
                 if (is_k) wait_noabort(&bars->q_full, 0);
                 for (int n = max(0, issued - nst); n < issued; ++n)
                     wait_noabort(&full[n % nst], (n / nst) & 1);
+                if (lin_issued) wait_noabort(&bars->lin_full, 0);
             }
         }
     } else if (warp == 5) {
@@ -206,7 +232,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             if (ok && lin) {
                 // Lin = phi(Q) S with S and phi(Q) split into bf16 hi + lo parts:
                 // hi*hi + hi*lo + lo*hi, fp32 accumulation in the S columns.
-                if (mbar_wait(&bars->lin_ready, 0, abort_flag)) {
+                if (mbar_wait(&bars->lin_full, 0, abort_flag) && mbar_wait(&bars->lin_ready, 0, abort_flag)) {
                     tc_fence_after();
                     const uint32_t id_lin = idesc_bf16_f32(64, D, false, true);
                     const uint32_t a_hi = smem_u32(sPhiHi), a_lo = smem_u32(sPhiLo);
@@ -282,19 +308,23 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         // phi(q) = elu(q) + 1 (SparkDiffusion RoLA / TurboDiffusion SLA linear
         // branch).  Each thread owns half a query row: D/2 features.
         float den = 1.f;
+        if (ok && lin && !__all_sync(0xffffffffu, mbar_wait(&bars->lin_full, 0, abort_flag))) ok = false;
         if (ok && lin) {
             tc_fence_after();
-            const float* zb = lin_z + (long long)bh * D + hf * (D / 2);
-            const float* Sb = lin_S + (long long)bh * D * D;
+            const float* zb = sZ + hf * (D / 2);
             float dpart = 0.f;
             // phi(Q) hi/lo: this thread's D/2 features sit in chunk (hf*(D/2))/64
-            // of the Q cube, 16-byte units u0 .. u0 + D/16 - 1 of row r.
+            // of the Q cube, 16-byte units u0 .. u0 + D/16 - 1 of row r; hi
+            // replaces q in place, lo goes to the same offset in the V ring.
             const int chunk = (hf * (D / 2)) / 64, u0 = ((hf * (D / 2)) % 64) / 8;
 #pragma unroll
             for (int u = 0; u < D / 16; ++u) {
                 const int uu = u0 + u;
                 const uint32_t off = chunk * 8192 + r * 128 + (((uu) ^ (r & 7)) << 4);
                 const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
+                const float4 z0 = reinterpret_cast<const float4*>(zb + u * 8)[0];
+                const float4 z1 = reinterpret_cast<const float4*>(zb + u * 8)[1];
+                const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
                 uint32_t hi[4], lo[4];
 #pragma unroll
@@ -302,36 +332,14 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     const float q0 = __uint_as_float(w[e] << 16), q1 = __uint_as_float(w[e] & 0xffff0000u);
                     const float f0 = q0 > 0.f ? q0 + 1.f : __expf(q0);
                     const float f1 = q1 > 0.f ? q1 + 1.f : __expf(q1);
-                    dpart += f0 * __ldg(zb + u * 8 + 2 * e) + f1 * __ldg(zb + u * 8 + 2 * e + 1);
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
-                    const float2 hf2 = __bfloat1622float2(h);
-                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    lo[e] = pack_bf16x2(f0 - hf2.x, f1 - hf2.y);
+                    dpart += f0 * zz[2 * e] + f1 * zz[2 * e + 1];
+                    hi[e] = pack_bf16x2(f0, f1);
+                    lo[e] = pack_bf16x2(f0 - __uint_as_float(hi[e] << 16), f1 - __uint_as_float(hi[e] & 0xffff0000u));
                 }
                 *reinterpret_cast<uint4*>(sPhiHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4*>(sPhiLo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
             den = dpart + __shfl_xor_sync(0xffffffffu, dpart, 16);
-            // S hi/lo (B operand, MN-major): row a = input feature, 64-wide
-            // chunks of output features c, 128-byte rows, 128-byte swizzle.
-            for (int unit = tid; unit < D * D / 8; unit += 128) {
-                const int a = unit / (D / 8), cu = unit % (D / 8);      // cu: 8-wide group of c
-                const int ch = cu / 8, uu = cu % 8;
-                const float4 x0 = __ldg(reinterpret_cast<const float4*>(Sb + a * D + cu * 8));
-                const float4 x1 = __ldg(reinterpret_cast<const float4*>(Sb + a * D + cu * 8 + 4));
-                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(xs[2 * e], xs[2 * e + 1]);
-                    const float2 hf2 = __bfloat1622float2(h);
-                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    lo[e] = pack_bf16x2(xs[2 * e] - hf2.x, xs[2 * e + 1] - hf2.y);
-                }
-                const uint32_t off = ch * (D * 128) + a * 128 + ((uu ^ (a & 7)) << 4);
-                *reinterpret_cast<uint4*>(sSHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(sSLo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
             fence_proxy_async_smem();
             mbar_arrive(&bars->lin_ready);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->lin_done, 0, abort_flag))) ok = false;
@@ -404,13 +412,13 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (a.g.T % a.g.tt) || (a.g.H % a.g.th) || (a.g.W % a.g.tw);
     fine_attn_kernel<D, LIN><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
-        *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged, a.lin_S, a.lin_z,
-        reinterpret_cast<__nv_bfloat16*>(a.out), a.status);
+        *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged,
+        static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
-    const bool lin = a.lin_S != nullptr;
+    const bool lin = a.lin_image != nullptr;
     if (a.g.d == 128) return lin ? launch_fine_impl<128, true>(a, stream) : launch_fine_impl<128, false>(a, stream);
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
 }

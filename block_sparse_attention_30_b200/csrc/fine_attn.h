@@ -15,8 +15,8 @@ struct FineArgs {
     const CUtensorMap* mv;
     const int32_t* block_idx;    // [B][heads][nt][topk]
     int topk;
-    const float* lin_S;          // optional linear-branch state [B][heads][d][d]
-    const float* lin_z;          // optional [B][heads][d]
+    const void* lin_image;       // optional linear-branch operand images, one per
+                                 // (b, head) (linear_image_bytes(d) each, see linear.h)
     void* out;                   // bf16 [B][N][heads][d]
     int* status;                 // device status word
 };

@@ -35,22 +35,28 @@ struct LinCfg {
     static constexpr int NCH = D / 64;                    // 64-feature chunks
     static constexpr int TILE = 64 * D * 2;               // one 64-token tile (bf16)
     static constexpr int STAGE = 3 * TILE;                // K -> phi hi (in place), V, phi lo
-    static constexpr int NST = 4;
-    static constexpr int BAR_BYTES = 128;
+    static constexpr int NST = D == 128 ? 4 : 8;          // 192 KB of stages
+    static constexpr int NTW = 8;                         // transform warps
+    static constexpr int THREADS = 32 * (NTW + 1);        // + one TMA / MMA warp
+    static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_BYTES = NST * STAGE + BAR_BYTES;
     static constexpr int TMEM_COLS = D < 32 ? 32 : D;     // fp32 accumulator, D columns
+    static constexpr int UPR = D / 8;                     // 16-byte units per token row
+    static constexpr int ROWS_PER_PASS = 32 * NTW / UPR;  // token rows one pass covers
 };
 
 template <int D>
 struct LinBars {
     uint64_t full[LinCfg<D>::NST];       // K and V of a stage landed
-    uint64_t ready[LinCfg<D>::NST];      // phi hi/lo written (128 arrivals)
+    uint64_t ready[LinCfg<D>::NST];      // phi hi/lo written (transform threads)
     uint64_t done[LinCfg<D>::NST];       // MMAs of a stage finished
+    uint64_t seg_done;                   // MMAs of one (b, head) segment finished
+    uint64_t mma_idle;                   // every MMA of the CTA finished
     uint32_t tmem_base;
     int abort;
 };
-
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+static_assert(sizeof(LinBars<64>) <= LinCfg<64>::BAR_BYTES, "barrier block");
+static_assert(sizeof(LinBars<128>) <= LinCfg<128>::BAR_BYTES, "barrier block");
 
 // Fire-and-forget vector add of four floats into global memory (16-byte aligned).
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
@@ -59,12 +65,23 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
-// grid: (chunks, B*heads); 160 threads: warps 0-3 transform K, warp 4 = TMA + MMA.
+// Where 64-token step gs of the flattened (b*heads, step) space lives.
+struct LinStep {
+    int bh, st;       // (b, head) pair and 64-token step within it
+    bool first, last; // first / last step of this CTA's segment of bh
+};
+
+// grid: one CTA per slice of the flattened (b*heads, 64-token step) space;
+// warps 0..NTW-1 transform K, warp NTW = TMA + MMA.  A CTA's slice may cross
+// (b, head) boundaries: at the end of each (b, head) segment the transform
+// warps read the accumulator out of TMEM and add it to S (and z) with
+// vector reductions, and the next segment starts a fresh accumulation.
 template <int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(LinCfg<D>::THREADS, 1)
 linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-                    const Grid g, const int tokens_per_cta, float* __restrict__ S,
-                    float* __restrict__ z, int* status) {
+                    const Grid g, const int steps_per_head, const long long total_steps,
+                    const int steps_per_cta, float* __restrict__ S, float* __restrict__ z,
+                    int* status) {
     using C = LinCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {
@@ -74,21 +91,30 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
     LinBars<D>* bars = reinterpret_cast<LinBars<D>*>(smem + C::NST * C::STAGE);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.y, b = bh / g.heads, head = bh % g.heads;
-    const long long n_begin = (long long)blockIdx.x * tokens_per_cta;
-    const long long n_end = min(n_begin + tokens_per_cta, g.N);
-    const int n_steps = (int)((n_end - n_begin + 63) / 64);
+    const long long gs0 = (long long)blockIdx.x * steps_per_cta;
+    const int n_steps = (int)max(0ll, min((long long)steps_per_cta, total_steps - gs0));
+    auto step_of = [&](int t) {
+        LinStep x;
+        const long long gs = gs0 + t;
+        x.bh = (int)(gs / steps_per_head);
+        x.st = (int)(gs - (long long)x.bh * steps_per_head);
+        x.first = t == 0 || x.st == 0;
+        x.last = t == n_steps - 1 || x.st == steps_per_head - 1;
+        return x;
+    };
 
     if (tid == 0) {
         bars->abort = 0;
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->ready[s], 128);
+            mbar_init(&bars->ready[s], 32 * C::NTW);
             mbar_init(&bars->done[s], 1);
         }
+        mbar_init(&bars->seg_done, 1);
+        mbar_init(&bars->mma_idle, 1);
         fence_barrier_init();
     }
-    if (warp == 4) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+    if (warp == C::NTW) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -96,25 +122,28 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
     auto stage_ptr = [&](int s, int part) { return smem + s * C::STAGE + part * C::TILE; };
     auto fail = [&]() { *abort_flag = 1; report(status, kStatusTimeout); };
 
-    if (warp == 4) {
+    if (warp == C::NTW) {
         if (lane == 0) {
             // ------------------------------------------------- loads + MMAs
             const uint32_t id = idesc_bf16_f32(D, D, true, true);
             bool ok = true;
+            int issued = 0;
             auto load = [&](int t) {
                 const int s = t % C::NST;
-                const int n0 = (int)(n_begin + 64ll * t);
+                const LinStep x = step_of(t);
+                const int b = x.bh / g.heads, head = x.bh % g.heads;
                 mbar_arrive_expect_tx(&bars->full[s], 2 * C::TILE);
                 for (int c = 0; c < C::NCH; ++c) {
-                    tma_load_3d(stage_ptr(s, 0) + c * 8192, &mk, &bars->full[s], head * D + 64 * c, n0, b);
-                    tma_load_3d(stage_ptr(s, 1) + c * 8192, &mv, &bars->full[s], head * D + 64 * c, n0, b);
+                    tma_load_3d(stage_ptr(s, 0) + c * 8192, &mk, &bars->full[s], head * D + 64 * c, 64 * x.st, b);
+                    tma_load_3d(stage_ptr(s, 1) + c * 8192, &mv, &bars->full[s], head * D + 64 * c, 64 * x.st, b);
                 }
+                ++issued;
             };
             for (int t = 0; t < min(C::NST, n_steps); ++t) load(t);
             for (int t = 0; t < n_steps && ok; ++t) {
                 const int s = t % C::NST;
-                const uint32_t ph = (uint32_t)((t / C::NST) & 1);
-                if (!mbar_wait_spin(&bars->ready[s], ph, abort_flag)) { ok = false; break; }
+                const LinStep x = step_of(t);
+                if (!mbar_wait_spin(&bars->ready[s], (uint32_t)((t / C::NST) & 1), abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(stage_ptr(s, 1));
 #pragma unroll
@@ -124,10 +153,11 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
                     for (int kk = 0; kk < 4; ++kk) {         // 16 tokens per MMA
                         const uint64_t a = smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
                         const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, 8192, 1024);
-                        mma_bf16_ss(tbase, a, bd, id, (t > 0 || part > 0 || kk > 0));
+                        mma_bf16_ss(tbase, a, bd, id, !(x.first && part == 0 && kk == 0));
                     }
                 }
                 mma_commit(&bars->done[s]);
+                if (x.last) mma_commit(&bars->seg_done);
                 // refill the stage of step t-1 (its MMAs ran before these) with step t-1+NST
                 const int tr = t - 1 + C::NST;
                 if (t >= 1 && tr < n_steps) {
@@ -136,81 +166,113 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
                     load(tr);
                 }
             }
-            if (!ok) fail();
-            // all MMAs done (the last commit covers every earlier MMA)
-            if (n_steps > 0) wait_noabort(&bars->done[(n_steps - 1) % C::NST], ((n_steps - 1) / C::NST) & 1);
+            if (!ok) {
+                fail();
+                // drain: the last load issued into each stage must land before exit
+                for (int n = max(0, issued - C::NST); n < issued; ++n)
+                    wait_noabort(&bars->full[n % C::NST], (n / C::NST) & 1);
+            }
+            mma_commit(&bars->mma_idle);
+            wait_noabort(&bars->mma_idle, 0);
         }
     } else {
         // ------------------------------------------- phi(K) hi/lo and z (fp32)
-        // thread -> 16-byte column unit u (8 features) and token rows r0 + 8i
-        const int u = tid % (D / 8), r0 = tid / (D / 8);
-        const int rows_per_pass = 128 / (D / 8);           // 8 for D = 128, 16 for D = 64
+        // thread -> 16-byte column unit u (8 features) and token rows r0 + k*ROWS_PER_PASS
+        const int u = tid % C::UPR, r0 = tid / C::UPR;
         const int chunk = u / 8, uu = u % 8;
         float zacc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+        const uint64_t one2 = f32x2(1.f, 1.f);
+        const float log2e = 1.4426950408889634f;
         bool ok = true;
+        int seg = 0;
         for (int t = 0; t < n_steps; ++t) {
             const int s = t % C::NST;
+            const LinStep x = step_of(t);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->full[s], (t / C::NST) & 1, abort_flag))) { ok = false; break; }
-            const int valid = (int)min(64ll, n_end - (n_begin + 64ll * t));
-            const uint8_t* kt = stage_ptr(s, 0);
-            uint8_t* hi = stage_ptr(s, 0);                  // in place: each thread rewrites its own units
+            const int valid = (int)min(64ll, g.N - 64ll * x.st);
+            uint8_t* kt = stage_ptr(s, 0);                  // phi hi is written in place
             uint8_t* lo = stage_ptr(s, 2);
-            for (int r = r0; r < 64; r += rows_per_pass) {
+#pragma unroll
+            for (int k = 0; k < 64 / C::ROWS_PER_PASS; ++k) {
+                const int r = r0 + k * C::ROWS_PER_PASS;
                 const uint32_t off = chunk * 8192 + r * 128 + ((uu ^ (r & 7)) << 4);
-                uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
+                const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
                 uint32_t h[4], l[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    // rows past the end of the grid hold zero-filled K: phi(0) = 1
-                    // must not count, so their phi is forced to 0
-                    const float f0 = r < valid ? phi_elu1(__uint_as_float(w[e] << 16)) : 0.f;
-                    const float f1 = r < valid ? phi_elu1(__uint_as_float(w[e] & 0xffff0000u)) : 0.f;
+                    // phi(x) = elu(x) + 1 = max(x + 1, e^min(x, 0)), because
+                    // e^x >= 1 + x everywhere; zero-filled rows past the end
+                    // of the grid would give phi(0) = 1 and are forced to 0
+                    const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+                    float p0, p1;
+                    unf32x2(add_f32x2(f32x2(x0, x1), one2), p0, p1);
+                    float f0 = fmaxf(p0, ex2(fminf(x0, 0.f) * log2e));
+                    float f1 = fmaxf(p1, ex2(fminf(x1, 0.f) * log2e));
+                    if (r >= valid) { f0 = 0.f; f1 = 0.f; }
                     zacc[2 * e] += f0;
                     zacc[2 * e + 1] += f1;
                     const uint32_t ph = pack_bf16x2(f0, f1);
                     h[e] = ph;
-                    l[e] = pack_bf16x2(f0 - __uint_as_float(ph << 16), f1 - __uint_as_float(ph & 0xffff0000u));
+                    float d0, d1;
+                    unf32x2(add_f32x2(f32x2(f0, f1), f32x2(-__uint_as_float(ph << 16), -__uint_as_float(ph & 0xffff0000u))), d0, d1);
+                    l[e] = pack_bf16x2(d0, d1);
                 }
-                *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4*>(kt + off) = make_uint4(h[0], h[1], h[2], h[3]);
                 *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&bars->ready[s]);
-            // the MMA thread reuses stage s only after its MMAs finished
-        }
-        if (!ok) fail();
-        // z: add this thread's 8 partial sums
-        float* zb = z + (long long)bh * D + u * 8;
+            if (x.last) {
+                // z of this segment: lanes with the same unit u sum first
 #pragma unroll
-        for (int e = 0; e < 8; ++e) atomicAdd(zb + e, zacc[e]);
-        // S partial from TMEM: warp w reads lanes 32w..32w+31 (= feature a)
-        if (ok && n_steps > 0) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->done[(n_steps - 1) % C::NST], ((n_steps - 1) / C::NST) & 1, abort_flag))) ok = false;
-        }
-        if (ok && n_steps > 0) {
-            // M = 128: feature a in lane a; M = 64: feature a in lane (a % 16) + 32 (a / 16)
-            tc_fence_after();
-            const int a = D == 128 ? 32 * warp + lane : 16 * warp + lane;
-            const bool mine = D == 128 || lane < 16;
-            float* Sb = S + ((long long)bh * D + a) * D;
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float vals[16];
-                tmem_ld_32x32b_x16(tbase + ((uint32_t)(32 * warp) << 16) + c0, vals);
-                tmem_wait_ld();
-                if (mine) {
-#pragma unroll
-                    for (int e = 0; e < 16; e += 4) red_add_v4(Sb + c0 + e, vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+                for (int e = 0; e < 8; ++e) {
+                    float v = zacc[e];
+                    for (int m = C::UPR; m < 32; m <<= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+                    zacc[e] = v;
                 }
+                if (lane < C::UPR) {
+                    float* zb = z + (long long)x.bh * D + u * 8;
+                    red_add_v4(zb, zacc[0], zacc[1], zacc[2], zacc[3]);
+                    red_add_v4(zb + 4, zacc[4], zacc[5], zacc[6], zacc[7]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+            }
+            mbar_arrive(&bars->ready[s]);
+            if (x.last) {
+                // the segment's accumulator: wait for its MMAs, add it to S
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->seg_done, seg & 1, abort_flag))) { ok = false; break; }
+                ++seg;
+                tc_fence_after();
+                // M = 128: feature a in lane a; M = 64: feature a in lane (a % 16) + 32 (a / 16).
+                // Warps w and w + 4 share sub-partition w % 4 and split the columns.
+                const int sp = warp % 4, part = warp / 4;
+                const int a = D == 128 ? 32 * sp + lane : 16 * sp + lane;
+                const bool mine = D == 128 || lane < 16;
+                float* Sb = S + ((long long)x.bh * D + a) * D;
+                constexpr int COLS = D / (C::NTW / 4);
+#pragma unroll
+                for (int c0 = part * COLS; c0 < (part + 1) * COLS; c0 += 16) {
+                    float vals[16];
+                    tmem_ld_32x32b_x16(tbase + ((uint32_t)(32 * sp) << 16) + c0, vals);
+                    tmem_wait_ld();
+                    if (mine) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4) red_add_v4(Sb + c0 + e, vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+                    }
+                }
+                // TMEM reads complete before the next segment's first MMA overwrites
+                tc_fence_before();
             }
         }
+        if (!ok) fail();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) tmem_dealloc(tbase, C::TMEM_COLS);
+    if (warp == C::NTW) tmem_dealloc(tbase, C::TMEM_COLS);
 }
 
 // 3-D view (heads*d, N, B) of a [B][N][heads][d] bf16 tensor; box = 64
@@ -251,14 +313,62 @@ static cudaError_t launch_linear_impl(const Grid& g, const void* k, const void* 
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(z, 0, sizeof(float) * g.B * g.heads * g.d, stream);
     if (e != cudaSuccess) return e;
-    // at most one wave (one CTA per SM) over all (b, head), whole 64-token steps per CTA
+    // one wave (one CTA per SM): the flattened (b*heads, 64-token step)
+    // space cut into equal slices of whole steps
+    const int steps_per_head = (int)((g.N + 63) / 64);
+    const long long total = (long long)g.B * g.heads * steps_per_head;
+    const long long per = (total + sms - 1) / sms;
+    const long long ctas = (total + per - 1) / per;
+    linear_state_kernel<D><<<(unsigned)ctas, C::THREADS, C::SMEM_BYTES, stream>>>(
+        mk, mv, g, steps_per_head, total, (int)per, S, z, status);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------ operand image of (S, z)
+// The fine kernel applies the branch as phi(Q) S on the tensor cores with S
+// split into bf16 hi + lo parts (S = hi + lo to ~2^-17 relative).  This
+// kernel writes, per (b, head), the shared-memory image the fine kernel
+// copies in one piece:
+//   [S hi | S lo | z], S parts as the MN-major B operand with a 128-byte
+//   swizzle: 64-wide chunks of output features c, in each chunk one
+//   128-byte row per input feature a, 16-byte unit u of row a stored at
+//   unit position u ^ (a & 7); z as d fp32 values.
+// One thread per 16-byte unit of S (8 consecutive c of one row a).
+__global__ void __launch_bounds__(256)
+linear_pack_kernel(const float* __restrict__ S, const float* __restrict__ z, uint8_t* __restrict__ image,
+                   int d, long long bh_count) {
+    const long long units_per_bh = (long long)d * d / 8;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long bh = gid / units_per_bh;
+    if (bh >= bh_count) return;
+    const int unit = (int)(gid % units_per_bh);
+    const int a = unit / (d / 8), cu = unit % (d / 8);
+    const int ch = cu / 8, uu = cu % 8;
+    const float* src = S + (bh * d + a) * d + cu * 8;
+    const float4 x0 = __ldg(reinterpret_cast<const float4*>(src));
+    const float4 x1 = __ldg(reinterpret_cast<const float4*>(src + 4));
+    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        hi[e] = pack_bf16x2(xs[2 * e], xs[2 * e + 1]);
+        lo[e] = pack_bf16x2(xs[2 * e] - __uint_as_float(hi[e] << 16),
+                            xs[2 * e + 1] - __uint_as_float(hi[e] & 0xffff0000u));
+    }
+    uint8_t* img = image + bh * linear_image_bytes(d);
+    const int off = ch * (d * 128) + a * 128 + ((uu ^ (a & 7)) << 4);
+    *reinterpret_cast<uint4*>(img + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(img + d * d * 2 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    if (unit < d / 4)       // z: d floats = d/4 16-byte units
+        reinterpret_cast<float4*>(img + 4 * d * d)[unit] = __ldg(reinterpret_cast<const float4*>(z + bh * d) + unit);
+}
+
+cudaError_t launch_linear_pack(const Grid& g, const float* S, const float* z, void* image,
+                               cudaStream_t stream) {
     const long long bh = (long long)g.B * g.heads;
-    long long chunks = sms / bh > 0 ? sms / bh : 1;
-    long long per = (g.N + chunks - 1) / chunks;
-    per = ((per + 63) / 64) * 64;
-    chunks = (g.N + per - 1) / per;
-    linear_state_kernel<D><<<dim3((unsigned)chunks, (unsigned)bh), 160, C::SMEM_BYTES, stream>>>(
-        mk, mv, g, (int)per, S, z, status);
+    const long long threads = bh * g.d * g.d / 8;
+    linear_pack_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
+        S, z, static_cast<uint8_t*>(image), g.d, bh);
     return cudaGetLastError();
 }
 

@@ -76,8 +76,11 @@ const char* vsa_status_string(vsa_status status);
 int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
 
 /* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
- * for these shapes: a 256-byte status block followed by the fp64 cube means
- * of q and k ([2][B][heads][nt][d]).  Returns 0 for invalid shapes.  The
+ * for these shapes: a 256-byte status block followed by a scratch area that
+ * holds either the selection's fp64 cube means of q and k
+ * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the
+ * linear branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is
+ * larger.  Returns 0 for invalid shapes.  The
  * same workspace may be passed to every call of one forward pass; calls that
  * share a workspace must be ordered on one stream. */
 size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W,
@@ -129,8 +132,12 @@ vsa_status vsa_linear_branch_fwd(const vsa_bf16* k, const vsa_bf16* v, float* li
  * written as bf16 to out in grid order.  Padded slots take no part.  When
  * lin_S and lin_z are both non-NULL (from vsa_linear_branch_fwd) the linear
  * branch phi(q) S / (phi(q).z) is added in fp32 before rounding; pass both
- * NULL for the sparse branch alone.  Needs vsa_workspace_bytes() of
- * workspace (status word only). */
+ * NULL for the sparse branch alone.  Without the linear branch only the
+ * workspace's status word is used; with it the call also writes a bf16 hi/lo
+ * copy of (lin_S, lin_z) into the workspace scratch (B*heads*(4*d*d + 4*d)
+ * bytes, within vsa_workspace_bytes()), so the scratch of an earlier
+ * vsa_select_blocks on the same workspace is overwritten (block_idx is not).
+ * Returns VSA_ERR_WORKSPACE when the workspace is smaller than that. */
 vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                                const int32_t* block_idx, const float* lin_S,
                                const float* lin_z, vsa_bf16* out, int B, int heads,

@@ -60,6 +60,9 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 0) == 0         # topk < 1
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 456) == 0       # topk > nt
+    # tiny grids: the linear branch's operand image (4*d*d + 4*d bytes per
+    # (b, head)) is larger than the selection scratch and sets the size
+    assert L.vsa_workspace_bytes(1, 2, 128, 4, 8, 8, 4, 4, 4, 2) == 256 + 2 * (4 * 128 * 128 + 4 * 128)
 
 
 SHAPE = [1, 2, 128, 4, 8, 8, 4, 4, 4]       # nt = 4
@@ -93,6 +96,9 @@ def test_fine_argument_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *SHAPE, 2, FAKE, 64, None) == WORKSPACE
     bad = list(SHAPE); bad[2] = 256
     assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, *bad, 2, FAKE, big, None) == UNSUPPORTED
+    # with the linear branch the workspace must hold the (S, z) operand image
+    image = 2 * (4 * 128 * 128 + 4 * 128)
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, *SHAPE, 2, FAKE, 256 + image - 16, None) == WORKSPACE
 
 
 def test_other_entry_points_validate(L):
