@@ -15,7 +15,12 @@
 //   * warp 5 (one lane) issues the tensor-core work: S = Q K^T (M=64 queries,
 //     N=128 keys, A and B from shared memory) into TMEM, then, once softmax
 //     has written P as bf16 over S in TMEM, O += P V (A = P from TMEM,
-//     B = V from shared memory, MN-major);
+//     B = V from shared memory, MN-major).  S and O are double-buffered by
+//     pair parity without extra TMEM columns: an M=64 accumulator fills only
+//     lanes 0-15 of each 32-lane sub-partition, so buffer 1 lives in lanes
+//     16-31 of the same columns.  S of pair p+2 is issued right after P V of
+//     pair p, so softmax finds the next S ready; the output is
+//     O(even pairs) + O(odd pairs);
 //   * warps 0-3 (one TMEM sub-partition each; rows 16w..16w+15, each row
 //     split in two 64-column halves over lanes t and t+16) do the fp32 online
 //     softmax in the exp2 domain (softmax_step.cuh), rescale O in TMEM only
@@ -63,7 +68,8 @@ struct FineBars {
     uint64_t q_full;
     uint64_t k_full[FineCfg<D>::NK], k_empty[FineCfg<D>::NK];
     uint64_t v_full[FineCfg<D>::NV], v_empty[FineCfg<D>::NV];
-    uint64_t s_full, p_full, o_ready, mma_done, lin_full, lin_ready, lin_done;
+    uint64_t s_full[2], p_full[2], o_ready[2];   // per S / O buffer (pair parity)
+    uint64_t mma_done, lin_full, lin_ready, lin_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -113,9 +119,11 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         mbar_init(&bars->q_full, 1);
         for (int s = 0; s < C::NK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
         for (int s = 0; s < C::NV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->o_ready, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_full[x], 128);
+            mbar_init(&bars->o_ready[x], 1);
+        }
         mbar_init(&bars->mma_done, 1);
         mbar_init(&bars->lin_full, 1);
         mbar_init(&bars->lin_ready, 128);
@@ -202,32 +210,43 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            const uint32_t tS = tbase + C::S_COL, tO = tbase + C::O_COL;
+            // pair p uses S buffer p & 1 and O buffer p & 1: the M = 64
+            // accumulators sit in TMEM lanes 0-15 (buffer 0) or 16-31 (buffer 1)
+            // of the same columns
+            auto tS = [&](int x) { return tbase + C::S_COL + ((uint32_t)x << 20); };   // lane 16 x
+            auto tO = [&](int x) { return tbase + C::O_COL + ((uint32_t)x << 20); };
             const uint32_t id_pv = idesc_bf16_f32(64, D, false, true);
-            bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
-            for (int p = 0; ok && p < n_pairs; ++p) {
+            auto issue_qk = [&](int p) -> bool {
                 const int nkeys = min(2, topk - 2 * p) * 64;
-                const int sk = p % C::NK, sv = p % C::NV;
-                if (!mbar_wait(&bars->k_full[sk], (p / C::NK) & 1, abort_flag)) { ok = false; break; }
+                const int sk = p % C::NK;
+                if (!mbar_wait(&bars->k_full[sk], (p / C::NK) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(k_addr + sk * C::PAIR_BYTES + (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32, 16, 1024);
-                    mma_bf16_ss(tS, a, bd, id_s, kk > 0);
+                    mma_bf16_ss(tS(p & 1), a, bd, id_s, kk > 0);
                 }
-                mma_commit(&bars->s_full);
+                mma_commit(&bars->s_full[p & 1]);
                 mma_commit(&bars->k_empty[sk]);
-                if (!mbar_wait(&bars->p_full, p & 1, abort_flag)) { ok = false; break; }
+                return true;
+            };
+            // S of pair p + 2 is computed while softmax works on pair p + 1
+            bool ok = mbar_wait(&bars->q_full, 0, abort_flag) && issue_qk(0) && (n_pairs < 2 || issue_qk(1));
+            for (int p = 0; ok && p < n_pairs; ++p) {
+                const int nkeys = min(2, topk - 2 * p) * 64;
+                const int sv = p % C::NV, x = p & 1;
+                if (!mbar_wait(&bars->p_full[x], (p >> 1) & 1, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(&bars->v_full[sv], (p / C::NV) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int kk = 0; kk < nkeys / 16; ++kk) {
                     const uint64_t bd = smem_desc_sw128(v_addr + sv * C::PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
-                    mma_bf16_ts(tO, tS + kk * 8, bd, id_pv, (p > 0 || kk > 0));
+                    mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
                 }
-                mma_commit(&bars->o_ready);
+                mma_commit(&bars->o_ready[x]);
                 mma_commit(&bars->v_empty[sv]);
+                if (p + 2 < n_pairs && !issue_qk(p + 2)) { ok = false; break; }
             }
             if (ok && lin) {
                 // Lin = phi(Q) S with S and phi(Q) split into bf16 hi + lo parts:
@@ -244,7 +263,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint64_t a = smem_desc_sw128(aa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
                             const uint64_t bd = smem_desc_sw128(bb + kk * 2048, D * 128, 1024);
-                            mma_bf16_ss(tS, a, bd, id_lin, (pass > 0 || kk > 0));
+                            mma_bf16_ss(tS(0), a, bd, id_lin, (pass > 0 || kk > 0));
                         }
                     }
                     mma_commit(&bars->lin_done);
@@ -259,8 +278,10 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     } else {
         // --------------------------------------------------- softmax / epilogue
         const int r = 16 * warp + (lane & 15), hf = lane >> 4;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        const uint32_t tS = tbase + lane_base + C::S_COL, tO = tbase + lane_base + C::O_COL;
+        // buffer x of this warp's rows: TMEM lanes 32*warp + 16*x .. + 15
+        const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
+        auto tS = [&](int x) { return lane_base + C::S_COL + ((uint32_t)x << 20); };
+        auto tO = [&](int x) { return lane_base + C::O_COL + ((uint32_t)x << 20); };
         SoftmaxState sm{-INFINITY, 0.f};
         bool ok = true;
         for (int p = 0; p < n_pairs; ++p) {
@@ -271,39 +292,43 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 if (j < 0 || j >= g.nt) j = 0;
                 vmask = valid_slot_mask(g, tile_coord(g, j));
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, p & 1, abort_flag))) { ok = false; break; }
+            const int x = p & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x], (p >> 1) & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
             float s[64];
-            tmem_ld_16x32bx2_x16<64>(tS + 0, *reinterpret_cast<float(*)[16]>(&s[0]));
-            tmem_ld_16x32bx2_x16<64>(tS + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
-            tmem_ld_16x32bx2_x16<64>(tS + 32, *reinterpret_cast<float(*)[16]>(&s[32]));
-            tmem_ld_16x32bx2_x16<64>(tS + 48, *reinterpret_cast<float(*)[16]>(&s[48]));
+            tmem_ld_16x32bx2_x16<64>(tS(x) + 0, *reinterpret_cast<float(*)[16]>(&s[0]));
+            tmem_ld_16x32bx2_x16<64>(tS(x) + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+            tmem_ld_16x32bx2_x16<64>(tS(x) + 32, *reinterpret_cast<float(*)[16]>(&s[32]));
+            tmem_ld_16x32bx2_x16<64>(tS(x) + 48, *reinterpret_cast<float(*)[16]>(&s[48]));
             tmem_wait_ld();
             uint32_t pk[32];
             bool resc;
             const bool masked = __any_sync(0xffffffffu, vmask != ~0ull);
             const float alpha = masked ? softmax_step<true>(s, vmask, scale_log2, sm, resc, pk)
                                        : softmax_step<false>(s, vmask, scale_log2, sm, resc, pk);
-            tmem_st_16x32bx2_x32(tS, pk);
+            tmem_st_16x32bx2_x32(tS(x), pk);
             if (p > 0 && __any_sync(0xffffffffu, resc)) {
-                // O holds PV up to pair p-1: wait for it, then rescale in place
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, (p - 1) & 1, abort_flag))) { ok = false; break; }
+                // the two O buffers hold PV up to pair p-1 (the completion of
+                // PV(p-1) implies that of every earlier MMA): rescale in place
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_ready[(p - 1) & 1], ((p - 1) >> 1) & 1, abort_flag))) { ok = false; break; }
                 tc_fence_after();
+                for (int ob = 0; ob < min(p, 2); ++ob) {
 #pragma unroll
-                for (int c0 = 0; c0 < D / 2; c0 += 16) {
-                    float o[16];
-                    tmem_ld_16x32bx2_x16<D / 2>(tO + c0, o);
-                    tmem_wait_ld();
+                    for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                        float o[16];
+                        tmem_ld_16x32bx2_x16<D / 2>(tO(ob) + c0, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] *= alpha;
-                    tmem_st_16x32bx2_x16<D / 2>(tO + c0, o);
+                        for (int e = 0; e < 16; ++e) o[e] *= alpha;
+                        tmem_st_16x32bx2_x16<D / 2>(tO(ob) + c0, o);
+                    }
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_full[x]);
         }
-        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, (n_pairs - 1) & 1, abort_flag))) ok = false;
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_ready[(n_pairs - 1) & 1], ((n_pairs - 1) >> 1) & 1, abort_flag))) ok = false;
         // ------------------------------------------------------- linear branch
         // phi(q) = elu(q) + 1 (SparkDiffusion RoLA / TurboDiffusion SLA linear
         // branch).  Each thread owns half a query row: D/2 features.
@@ -359,10 +384,17 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 #pragma unroll
             for (int c0 = 0; c0 < D / 2; c0 += 16) {
                 float o[16];
-                tmem_ld_16x32bx2_x16<D / 2>(tO + c0, o);
+                tmem_ld_16x32bx2_x16<D / 2>(tO(0) + c0, o);
+                if (n_pairs > 1) {                     // O = O(even pairs) + O(odd pairs)
+                    float o1[16];
+                    tmem_ld_16x32bx2_x16<D / 2>(tO(1) + c0, o1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] += o1[e];
+                }
                 if (lin) {
                     float li[16];
-                    tmem_ld_16x32bx2_x16<D / 2>(tS + c0, li);
+                    tmem_ld_16x32bx2_x16<D / 2>(tS(0) + c0, li);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o[e] = o[e] * inv + li[e] * inv_den;
