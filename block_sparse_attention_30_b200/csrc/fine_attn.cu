@@ -54,6 +54,14 @@ struct FineCfg {
     static constexpr int NK = (D == 128) ? 2 : 3;      // K pair stages
     static constexpr int NV = (D == 128) ? 1 : 3;      // V pair stages
     static constexpr int TMEM_COLS = 256;
+    // A ring slot is free once the MMAs reading it are done.  With two K stages
+    // the stage of pair p is the S buffer p & 1, so the K producer can wait on
+    // s_full (the completion of Q K^T of pair p-2); with one V stage, on
+    // o_ready (P V of pair p-1).  Neither barrier can run two phases ahead of
+    // such a waiter, because its next completion needs the very load the
+    // producer has not issued yet.  Deeper rings keep their own barriers.
+    static constexpr bool K_ON_S = NK == 2;
+    static constexpr bool V_ON_O = NV == 1;
     static constexpr int O_COL = 0;                    // fp32 O, D columns
     static constexpr int S_COL = 128;                  // fp32 S (128 cols) / bf16 P (64 cols)
     static constexpr int BAR_BYTES = 256;
@@ -170,7 +178,13 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 for (int t = 0; t < ntl; ++t)
                     if (jt[t] < 0 || jt[t] >= g.nt) { if (is_k) report(status, kStatusBadIndex); jt[t] = 0; }
                 const int st = p % nst;
-                if (p >= nst && !mbar_wait(&empty[st], ((p / nst) - 1) & 1, abort_flag)) { fail(); break; }
+                if (p >= nst) {
+                    uint64_t* bar = &empty[st];
+                    uint32_t par = ((p / nst) - 1) & 1;
+                    if (is_k && C::K_ON_S) { bar = &bars->s_full[p & 1]; par = ((p >> 1) - 1) & 1; }
+                    if (!is_k && C::V_ON_O) { bar = &bars->o_ready[(p - 1) & 1]; par = ((p - 1) >> 1) & 1; }
+                    if (!mbar_wait(bar, par, abort_flag)) { fail(); break; }
+                }
                 mbar_arrive_expect_tx(&full[st], ntl * C::CUBE_BYTES);
                 for (int t = 0; t < ntl; ++t) {
                     const TileCoord kc = tile_coord(g, jt[t]);
@@ -186,7 +200,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 // MMAs (each stage's last use) are done
                 bool free = true;
                 for (int p = max(0, n_pairs - nst); p < n_pairs && free; ++p)
-                    free = mbar_wait(&empty[p % nst], (p / nst) & 1, abort_flag);
+                    free = C::K_ON_S ? mbar_wait(&bars->s_full[p & 1], (p >> 1) & 1, abort_flag)
+                                     : mbar_wait(&empty[p % nst], (p / nst) & 1, abort_flag);
                 if (free) {
                     const uint8_t* img = lin_image + (long long)bh * (4 * D * D + 4 * D);
                     mbar_arrive_expect_tx(&bars->lin_full, 4 * D * D + 4 * D);
@@ -229,7 +244,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     mma_bf16_ss(tS(p & 1), a, bd, id_s, kk > 0);
                 }
                 mma_commit(&bars->s_full[p & 1]);
-                mma_commit(&bars->k_empty[sk]);
+                if (!C::K_ON_S) mma_commit(&bars->k_empty[sk]);
                 return true;
             };
             // S of pair p + 2 is computed while softmax works on pair p + 1
@@ -245,7 +260,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
                 }
                 mma_commit(&bars->o_ready[x]);
-                mma_commit(&bars->v_empty[sv]);
+                if (!C::V_ON_O) mma_commit(&bars->v_empty[sv]);
                 if (p + 2 < n_pairs && !issue_qk(p + 2)) { ok = false; break; }
             }
             if (ok && lin) {
