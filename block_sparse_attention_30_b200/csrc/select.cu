@@ -11,8 +11,8 @@
 //   pool_kernel    one CTA per (cube, batch, q|k): 16-byte vector loads of the
 //                  cube's valid token rows (all heads at once), fp64 sums,
 //                  divide by the valid count -> pooled [2][B][heads][nt][d].
-//   coarse_kernel  per (b, head) a 64x64 tile of C = Qp Kp^T / sqrt(d) with an
-//                  8x4 register tile per thread -> scores [B][heads][nt][nt].
+//   coarse_kernel  per (b, head) a 64x64 tile of C = Qp Kp^T / sqrt(d) on the
+//                  fp64 tensor cores -> scores [B][heads][nt][nt].
 //   topk_kernel    one warp per score row: 8-pass MSD radix select on
 //                  order-preserving 64-bit keys finds the k-th largest score,
 //                  then a ballot sweep in ascending j emits the kept cubes
@@ -81,62 +81,77 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, cons
 }
 
 // ------------------------------------------------------------ coarse scores
-// C[i][j] = (sum_c Qp[i][c] Kp[j][c]) / sqrt(d), per (b, head); 64x64 tiles,
-// 128 threads, 8 (rows) x 4 (cols) fp64 outputs per thread, operands staged
-// 16 features at a time, read back with 16-byte shared loads.  The features
-// are summed in increasing order, as in the exact definition.
+// C[i][j] = (sum_c Qp[i][c] Kp[j][c]) / sqrt(d), per (b, head), in fp64 on
+// the fp64 tensor cores (mma.sync m8n8k4, exact products, fp64 accumulation;
+// tcgen05 has no fp64 kind).  64x64 tiles of C per CTA, 4 warps of 32x32
+// (4x4 MMA tiles), operands staged 32 features at a time in shared memory.
+// The summation order differs from a sequential dot product only at the fp64
+// rounding level, far inside the near-tie tolerance of the selection.
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
+}
+
+constexpr int kCoarseChunk = 32;                 // features staged per step
+constexpr int kCoarseStride = kCoarseChunk + 4;  // doubles per smem row: 8-byte loads of a
+                                                 // half-warp (4 rows x 4 features) hit distinct banks
+
 __global__ void __launch_bounds__(128)
 coarse_kernel(const double* __restrict__ qp, const double* __restrict__ kp, const Grid g,
               const double inv_sqrt_d, double* __restrict__ scores) {
-    __shared__ __align__(16) double As[16][64 + 2];
-    __shared__ __align__(16) double Bs[16][64 + 2];
+    __shared__ __align__(16) double As[64 * kCoarseStride];
+    __shared__ __align__(16) double Bs[64 * kCoarseStride];
     const int bh = blockIdx.z;
     const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
     const int nt = g.nt, d = g.d;
     const double* Q = qp + (long long)bh * nt * d;
     const double* K = kp + (long long)bh * nt * d;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;     // 16 column groups x 8 row groups
-    double acc[8][4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wm = warp >> 1, wn = warp & 1;         // warp tile: rows 32*wm.., cols 32*wn..
+    const int gr = lane >> 2, tq = lane & 3;         // MMA fragment coordinates
+    double acc[4][4][2];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = 0.0;
-    for (int e0 = 0; e0 < d; e0 += 16) {
-        for (int l = threadIdx.x; l < 64 * 16; l += 128) {
-            const int rr = l / 16, ee = l % 16;
-            As[ee][rr] = (i0 + rr < nt) ? Q[(long long)(i0 + rr) * d + e0 + ee] : 0.0;
-            Bs[ee][rr] = (j0 + rr < nt) ? K[(long long)(j0 + rr) * d + e0 + ee] : 0.0;
+        for (int c = 0; c < 4; ++c) acc[a][c][0] = acc[a][c][1] = 0.0;
+    for (int e0 = 0; e0 < d; e0 += kCoarseChunk) {
+        // 64 rows x 32 features of each operand, 16-byte loads, zero rows past nt
+        for (int l = threadIdx.x; l < 64 * kCoarseChunk / 2; l += 128) {
+            const int rr = l / (kCoarseChunk / 2), cc = 2 * (l % (kCoarseChunk / 2));
+            const double2 qa = i0 + rr < nt ? *reinterpret_cast<const double2*>(Q + (long long)(i0 + rr) * d + e0 + cc)
+                                            : make_double2(0.0, 0.0);
+            const double2 kb = j0 + rr < nt ? *reinterpret_cast<const double2*>(K + (long long)(j0 + rr) * d + e0 + cc)
+                                            : make_double2(0.0, 0.0);
+            *reinterpret_cast<double2*>(&As[rr * kCoarseStride + cc]) = qa;
+            *reinterpret_cast<double2*>(&Bs[rr * kCoarseStride + cc]) = kb;
         }
         __syncthreads();
 #pragma unroll
-        for (int ee = 0; ee < 16; ++ee) {
-            double a[8], bv[4];
+        for (int ks = 0; ks < kCoarseChunk / 4; ++ks) {
+            double a[4], b[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const double2 t2 = *reinterpret_cast<const double2*>(&As[ee][8 * ty + 2 * u]);
-                a[2 * u] = t2.x; a[2 * u + 1] = t2.y;
+            for (int t = 0; t < 4; ++t) {
+                a[t] = As[(32 * wm + 8 * t + gr) * kCoarseStride + 4 * ks + tq];   // A[row][k]
+                b[t] = Bs[(32 * wn + 8 * t + gr) * kCoarseStride + 4 * ks + tq];   // B[k][col] = Kp[col][k]
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const double2 t2 = *reinterpret_cast<const double2*>(&Bs[ee][4 * tx + 2 * u]);
-                bv[2 * u] = t2.x; bv[2 * u + 1] = t2.y;
-            }
+            for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) acc[u][w] = fma(a[u], bv[w], acc[u][w]);
+                for (int ct = 0; ct < 4; ++ct) dmma_8x8x4(acc[rt][ct][0], acc[rt][ct][1], a[rt], b[ct]);
         }
         __syncthreads();
     }
     double* S = scores + (long long)bh * nt * nt;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const int ii = i0 + 8 * ty + u;
+    for (int rt = 0; rt < 4; ++rt) {
+        const int ii = i0 + 32 * wm + 8 * rt + gr;
         if (ii >= nt) continue;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const int jj = j0 + 4 * tx + w;
-            if (jj < nt) S[(long long)ii * nt + jj] = acc[u][w] * inv_sqrt_d;
+        for (int ct = 0; ct < 4; ++ct) {
+            const int jj = j0 + 32 * wn + 8 * ct + 2 * tq;
+            if (jj < nt) S[(long long)ii * nt + jj] = acc[rt][ct][0] * inv_sqrt_d;
+            if (jj + 1 < nt) S[(long long)ii * nt + jj + 1] = acc[rt][ct][1] * inv_sqrt_d;
         }
     }
 }
