@@ -178,14 +178,31 @@ topk_kernel(const double* __restrict__ scores, const int nt, const int k, const 
     for (int j = lane; j < nt; j += 32) keys[j] = ordered_key(src[j]);
     __syncwarp();
 
-    unsigned long long prefix = 0, mask = 0;
+    // Skip the leading bytes every key shares (for scores of one magnitude
+    // the sign and exponent byte): start at the highest byte where the
+    // smallest and largest keys differ.
+    unsigned long long kmin = ~0ull, kmax = 0ull;
+    for (int j = lane; j < nt; j += 32) { kmin = min(kmin, keys[j]); kmax = max(kmax, keys[j]); }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+    }
+    const unsigned long long diff = kmin ^ kmax;
+    const int top_shift = diff ? ((63 - __clzll(diff)) / 8) * 8 : -8;
+    unsigned long long mask = top_shift >= 56 ? 0ull : (~0ull << (top_shift + 8));
+    unsigned long long prefix = kmin & mask;        // the common leading bytes
     int remaining = k;                                 // how many still to place at/below prefix
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int shift = top_shift; shift >= 0; shift -= 8) {
         for (int h = lane; h < 256; h += 32) hist[h] = 0;
         __syncwarp();
-        for (int j = lane; j < nt; j += 32) {
-            const unsigned long long u = keys[j];
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1u);
+        for (int j0 = 0; j0 < nt; j0 += 32) {
+            const int j = j0 + lane;
+            const unsigned long long u = j < nt ? keys[j] : 0ull;
+            const int bin = (j < nt && (u & mask) == prefix) ? (int)((u >> shift) & 255) : 256;
+            // one atomic per distinct bin of the warp (keys cluster in few bins)
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
         }
         __syncwarp();
         // lane l owns digits 255-8l .. 248-8l (descending); inclusive scan from the top
@@ -203,31 +220,34 @@ topk_kernel(const double* __restrict__ scores, const int nt, const int k, const 
         // whose inclusive count reaches `remaining`
         const unsigned ball = __ballot_sync(0xffffffffu, incl >= remaining);
         const int owner = __ffs(ball) - 1;
-        int digit = 0, above = 0;
+        int digit = 0, above = 0, bucket = 0;
         if (lane == owner) {
             int run = excl;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                if (run + cnt[e] >= remaining) { digit = 255 - 8 * lane - e; above = run; break; }
+                if (run + cnt[e] >= remaining) { digit = 255 - 8 * lane - e; above = run; bucket = cnt[e]; break; }
                 run += cnt[e];
             }
         }
         digit = __shfl_sync(0xffffffffu, digit, owner);
         above = __shfl_sync(0xffffffffu, above, owner);
+        bucket = __shfl_sync(0xffffffffu, bucket, owner);
         remaining -= above;
         prefix |= (unsigned long long)digit << shift;
         mask |= 255ull << shift;
         __syncwarp();
+        if (bucket == remaining) break;                // the whole bucket is kept: done
     }
-    // prefix is the k-th largest key; take every larger key and the first
-    // `remaining` keys equal to it, sweeping j upward (ascending output).
+    // Every key whose masked value exceeds prefix is kept, and of the keys
+    // equal to it under the mask the first `remaining` in ascending j (all of
+    // them when the loop stopped early; equal full keys go lowest j first).
     int32_t* out = idx + row * k;
     int base = 0, eq_seen = 0;
     const unsigned lt_mask = (1u << lane) - 1u;
     for (int j0 = 0; j0 < nt; j0 += 32) {
         const int j = j0 + lane;
         const bool in = j < nt;
-        const unsigned long long u = in ? keys[j] : 0ull;
+        const unsigned long long u = in ? (keys[j] & mask) : 0ull;
         const bool gt = in && u > prefix;
         const bool eq = in && u == prefix;
         const unsigned eqb = __ballot_sync(0xffffffffu, eq);

@@ -124,6 +124,26 @@ def test_small_grids_select_and_fine(ops, case):
     check_close(to_f64(out), ref)
 
 
+@pytest.mark.parametrize("d,topk", [(128, 5), (64, 12)])
+def test_exact_ties_take_lowest_cube_ids(ops, d, topk):
+    """Key cubes in three classes of identical tokens give exactly three
+    distinct scores per row: the selection must follow the tie rule (larger
+    score first, then lower cube id) exactly, not only up to near-ties."""
+    T, H, W, heads = 8, 16, 16, 2                       # 2 x 4 x 4 = 32 cubes
+    c = Small(T, H, W, heads, d, topk, seed=5)
+    g = torch.Generator().manual_seed(123)
+    levels = torch.randn(3, heads, d, generator=g).to(torch.bfloat16)
+    slots = O.tile_slots(T, H, W, (4, 4, 4))            # [nt, 64] token ids
+    k = c.k.clone()
+    for j in range(slots.shape[0]):
+        toks = torch.as_tensor(slots[j][slots[j] >= 0])
+        k[0, toks] = levels[j % 3]
+    qd, kd = c.q.cuda(), k.cuda()
+    idx, _ = run_select(ops, c, qd, kd)
+    ref_idx, _ = O.select(c.q, k, 1, heads, d, T, H, W, topk, (4, 4, 4), with_scores=True)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+
+
 @pytest.mark.parametrize("case", [(5, 6, 7, 3, 128, 3), (4, 8, 12, 2, 64, 4)])
 def test_batch_of_two(ops, case):
     """B = 2: batch indexing of the pooled means, TMA boxes and outputs."""
