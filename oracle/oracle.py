@@ -134,6 +134,19 @@ def fine(q, k, v, idx, B, heads, d, T, H, W, tile=(4, 4, 4), precision="f64") ->
     return out
 
 
+def fine_bwd(q, k, v, dout, idx, B, heads, d, T, H, W, tile=(4, 4, 4), precision="f64"):
+    """Gradients (dq, dk, dv), each [B][N][heads][d], of the fine pass with the
+    selection idx held fixed, for the output gradient dout (bf16 like q)."""
+    qb, kb, vb, gb = bits(q), bits(k), bits(v), bits(dout)
+    idx = np.ascontiguousarray(idx, np.int32)
+    R = _real(precision)
+    dq, dk, dv = (np.empty((B, T * H * W, heads, d), R) for _ in range(3))
+    lib(precision).oracle_fine_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(idx), _c_int(B),
+                                   _c_int(heads), _c_int(d), *_grid_args(T, H, W, tile),
+                                   _c_int(idx.shape[-1]), _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
 def fine_tiles(q, k, v, idx, rows, B, heads, d, T, H, W, tile=(4, 4, 4),
                precision="f64") -> np.ndarray:
     """Fine pass for a sample of query tiles; rows[r] = (b*heads + head)*nt + i.

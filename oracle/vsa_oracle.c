@@ -405,6 +405,94 @@ void oracle_weights(const uint16_t *q, const uint16_t *kk, const int32_t *idx,
  * q and k (no projection, weight one).  The state sums run over ALL valid
  * tokens:  S = sum_n phi(k_n)^T v_n  (d x d),  z = sum_n phi(k_n)  (d).
  * lin_n = phi(q_n) S / (phi(q_n) . z). */
+/* ------------------------------------------------------ fine pass, backward
+ * Gradients of the fine pass (trainable sparse attention: "FastVideo
+ * 稀疏蒸馏技术深度解析", section "2. 视频稀疏注意力VSA", and the TurboDiffusion
+ * article, section "稀疏、蒸馏与全链路量化", train the sparse branch).  The
+ * selection is a fixed input here, as in the forward fine pass.  For each
+ * valid query token n with kept keys m (valid tokens of its selected tiles),
+ * given the output gradient dO_n, straight from the chain rule through
+ * s_m = q_n.k_m / sqrt(d), p = softmax(s), o_n = sum_m p_m v_m:
+ *     dv_m += p_m dO_n
+ *     dp_m  = dO_n . v_m
+ *     ds_m  = p_m (dp_m - sum_m' p_m' dp_m')
+ *     dq_n  = sum_m ds_m k_m / sqrt(d)
+ *     dk_m += ds_m q_n / sqrt(d)
+ * dout is bf16 (bit patterns, like q, k, v); dq, dk, dv are REAL, fully
+ * overwritten.  One (b, head) per OpenMP iteration, so the dk / dv sums of a
+ * key never race. */
+void oracle_fine_bwd(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
+                     const uint16_t *dout, const int32_t *idx, int B, int heads, int d,
+                     int T, int H, int W, int tt, int th, int tw, int k,
+                     REAL *dq, REAL *dk, REAL *dv)
+{
+    grid_t g = make_grid(T, H, W, tt, th, tw);
+    REAL inv_sqrt_d = (REAL)1 / ORACLE_SQRT((REAL)d);
+    size_t total = (size_t)B * g.N * heads * d;
+    memset(dq, 0, sizeof(REAL) * total);
+    memset(dk, 0, sizeof(REAL) * total);
+    memset(dv, 0, sizeof(REAL) * total);
+#pragma omp parallel
+    {
+        int64_t *tok = (int64_t *)malloc(sizeof(int64_t) * (size_t)k * g.vol);
+        REAL *p = (REAL *)malloc(sizeof(REAL) * (size_t)k * g.vol);
+        REAL *dp = (REAL *)malloc(sizeof(REAL) * (size_t)k * g.vol);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < (int64_t)B * heads; ++bh) {
+            int b = (int)(bh / heads), hd = (int)(bh % heads);
+            for (int i = 0; i < g.nt; ++i) {
+                const int32_t *sel = idx + (bh * g.nt + i) * k;
+                int nk = 0;
+                for (int a = 0; a < k; ++a)
+                    for (int s = 0; s < g.vol; ++s) {
+                        int64_t m = slot_token(&g, sel[a], s);
+                        if (m >= 0) tok[nk++] = m;
+                    }
+                for (int s = 0; s < g.vol; ++s) {
+                    int64_t n = slot_token(&g, i, s);
+                    if (n < 0) continue;
+                    const uint16_t *qr = row_ptr(q, g.N, heads, d, b, n, hd);
+                    const uint16_t *gr = row_ptr(dout, g.N, heads, d, b, n, hd);
+                    /* p = softmax(s) */
+                    REAL mx = -INFINITY;
+                    for (int m = 0; m < nk; ++m) {
+                        const uint16_t *kr = row_ptr(kk, g.N, heads, d, b, tok[m], hd);
+                        REAL acc = 0;
+                        for (int c = 0; c < d; ++c) acc += bf16_to_real(qr[c]) * bf16_to_real(kr[c]);
+                        p[m] = acc * inv_sqrt_d;
+                        if (p[m] > mx) mx = p[m];
+                    }
+                    REAL sum = 0;
+                    for (int m = 0; m < nk; ++m) { p[m] = ORACLE_EXP(p[m] - mx); sum += p[m]; }
+                    for (int m = 0; m < nk; ++m) p[m] /= sum;
+                    /* dp_m = dO_n . v_m and the row term sum_m p_m dp_m */
+                    REAL row = 0;
+                    for (int m = 0; m < nk; ++m) {
+                        const uint16_t *vr = row_ptr(v, g.N, heads, d, b, tok[m], hd);
+                        REAL acc = 0;
+                        for (int c = 0; c < d; ++c) acc += bf16_to_real(gr[c]) * bf16_to_real(vr[c]);
+                        dp[m] = acc;
+                        row += p[m] * acc;
+                    }
+                    REAL *dqr = dq + (((int64_t)b * g.N + n) * heads + hd) * d;
+                    for (int m = 0; m < nk; ++m) {
+                        REAL ds = p[m] * (dp[m] - row);
+                        const uint16_t *kr = row_ptr(kk, g.N, heads, d, b, tok[m], hd);
+                        REAL *dkr = dk + (((int64_t)b * g.N + tok[m]) * heads + hd) * d;
+                        REAL *dvr = dv + (((int64_t)b * g.N + tok[m]) * heads + hd) * d;
+                        for (int c = 0; c < d; ++c) {
+                            dqr[c] += ds * bf16_to_real(kr[c]) * inv_sqrt_d;
+                            dkr[c] += ds * bf16_to_real(qr[c]) * inv_sqrt_d;
+                            dvr[c] += p[m] * bf16_to_real(gr[c]);
+                        }
+                    }
+                }
+            }
+        }
+        free(tok); free(p); free(dp);
+    }
+}
+
 static REAL phi(REAL x) { return x > 0 ? x + 1 : ORACLE_EXP(x); }
 
 void oracle_linear_state(const uint16_t *kk, const uint16_t *v, int B, int heads,

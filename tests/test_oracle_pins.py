@@ -295,3 +295,68 @@ def test_fp32_oracle_far_inside_tolerance(oracle_mod):
     err = np.abs(o64 - o32).max()
     rel = np.linalg.norm(o64 - o32) / np.linalg.norm(o64)
     assert err < 1e-4 and rel < 1e-5
+
+
+# ------------------------------------------------------------ fine backward
+
+def _dout(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (0.5 * torch.randn(shape, generator=g)).to(torch.bfloat16)
+
+
+def _torch_masked_attention(q, k, v, mask):
+    """Dense attention restricted by mask, in torch fp64 (autograd-able)."""
+    d = q.shape[-1]
+    s = torch.einsum("bnhd,bmhd->bhnm", q, k) / np.sqrt(d)
+    s = s.masked_fill(~mask, float("-inf"))
+    return torch.einsum("bhnm,bmhd->bnhd", torch.softmax(s, -1), v)
+
+
+@pytest.mark.parametrize("case", TINY)
+def test_fine_bwd_matches_autograd_of_masked_dense(oracle_mod, case):
+    """P9: the backward equals torch autograd (fp64) of dense attention under
+    the explicit N x N block mask -- an independent differentiation path."""
+    T, H, W, tile, heads, d, k = case
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=11, amplitude=0.7)
+    dout = _dout(q.shape, seed=12)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    dq, dk, dv = oracle_mod.fine_bwd(q, kk, v, dout, idx, 1, heads, d, T, H, W, tile)
+    tq, tk, tv = (x.to(torch.float64).requires_grad_() for x in (q, kk, v))
+    mask = torch.as_tensor(twin.block_mask(idx, T, H, W, tile))
+    out = _torch_masked_attention(tq, tk, tv, mask)
+    out.backward(dout.to(torch.float64))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_fine_bwd_all_tiles_equals_sdpa_autograd(oracle_mod):
+    """P9 (dense limit): k = nt gives the gradients of torch SDPA (fp64)."""
+    T, H, W, tile, heads, d = 4, 8, 8, (4, 4, 4), 2, 16
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=13, amplitude=0.7)
+    dout = _dout(q.shape, seed=14)
+    nt = oracle_mod.num_tiles(T, H, W, tile)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, nt, tile)
+    dq, dk, dv = oracle_mod.fine_bwd(q, kk, v, dout, idx, 1, heads, d, T, H, W, tile)
+    tq, tk, tv = (x.to(torch.float64).permute(0, 2, 1, 3).contiguous().requires_grad_() for x in (q, kk, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)
+    out.backward(dout.to(torch.float64).permute(0, 2, 1, 3))
+    for mine, ref in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(mine, ref.grad.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-11)
+
+
+def test_fine_bwd_dv_is_weights_times_dout(oracle_mod):
+    """P9: dv_m = sum_n p(n, m) dO_n, with p from the oracle's per-query
+    weights (a separate function) -- and keys of tiles nobody keeps get 0."""
+    T, H, W, tile, heads, d, k = 5, 6, 7, (4, 4, 4), 1, 8, 2
+    q, kk, v = _inputs(T, H, W, tile, heads, d, seed=15)
+    dout = _dout(q.shape, seed=16)
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    dq, dk, dv = oracle_mod.fine_bwd(q, kk, v, dout, idx, 1, heads, d, T, H, W, tile)
+    N = T * H * W
+    P = np.stack([oracle_mod.weights(q, kk, idx, 0, 0, n, 1, heads, d, T, H, W, tile) for n in range(N)])
+    ref = P.T @ dout[0, :, 0].to(torch.float64).numpy()
+    np.testing.assert_allclose(dv[0, :, 0], ref, rtol=0, atol=1e-12)
+    never = P.sum(0) == 0
+    assert never.any(), "case should leave some key tiles unselected"
+    assert np.all(dk[0, never] == 0) and np.all(dv[0, never] == 0)
