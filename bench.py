@@ -355,6 +355,22 @@ def run_kernels(args):
             q, k, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, attn.lin_S, attn.lin_z, w.tile),
          "tensor", w.fine_flops()),
     ]
+    # backward pass (trainable sparse branch): the training forward (with the
+    # per-row lse) and the backward; algorithmic FLOPs of the backward are
+    # the five products S, dP, dV, dQ, dK per kept (query, key) cube pair
+    lse = torch.empty((w.B, w.heads, nt, 64), dtype=torch.float32, device=dev)
+    out32 = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    g_out = torch.randn(q.shape, device=dev).mul_(0.5).to(torch.bfloat16)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    rows += [
+        ("sparse_attn_fwd_train (training forward)", lambda: ops.vsa_sparse_attn_fwd_train(
+            q, k, v, attn.block_idx, out, out32, lse, w.T, w.H, w.W, w.topk, attn.workspace, w.tile),
+         "tensor", w.fine_flops()),
+        ("sparse_attn_bwd (backward)", lambda: ops.vsa_sparse_attn_bwd(
+            q, k, v, out32, g_out, attn.block_idx, lse, dq, dk, dv, w.T, w.H, w.W, w.topk,
+            attn.workspace, w.tile),
+         "tensor", 2.5 * w.fine_flops()),
+    ]
     for name, fn, bound, units in rows:
         ms = timed(fn)
         if bound == "hbm":

@@ -14,6 +14,7 @@
 #include "linear.h"
 #include "select.h"
 #include "tiles.h"
+#include "fine_bwd.h"
 
 namespace {
 
@@ -101,9 +102,12 @@ size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W, 
     if (check_shape(B, heads, head_dim, T, H, W, tt, th, tw) != VSA_OK) return 0;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return 0;
-    const size_t select = vsa::select_scratch_bytes(g);
+    size_t scratch = vsa::select_scratch_bytes(g);
     const size_t image = lin_image_bytes(g);
-    return kStatusBytes + (select > image ? select : image);
+    const size_t bwd = vsa::bwd_scratch_bytes(g, topk);
+    if (image > scratch) scratch = image;
+    if (bwd > scratch) scratch = bwd;
+    return kStatusBytes + scratch;
 }
 
 vsa_status vsa_workspace_init(void* workspace, size_t workspace_bytes, vsa_stream_t stream) {
@@ -195,6 +199,8 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     a.topk = topk;
     a.lin_image = nullptr;
     a.out = out;
+    a.out32 = nullptr;
+    a.lse = nullptr;
     a.status = static_cast<int*>(workspace);
     if (lin_S) {
         // the bf16 hi/lo operand image of (S, z) goes into the workspace scratch
@@ -204,6 +210,77 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
         if (e != cudaSuccess) return from_cuda(e);
     }
     return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
+}
+
+vsa_status vsa_sparse_attn_fwd_train(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                                     const int32_t* block_idx, vsa_bf16* out, float* out_f32,
+                                     float* lse, int B, int heads, int head_dim, int T, int H, int W,
+                                     int tt, int th, int tw, int topk, void* workspace,
+                                     size_t workspace_bytes, vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (s != VSA_OK) return s;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_idx) || !aligned16(out) ||
+        !aligned16(out_f32) || !aligned16(lse))
+        return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes) return VSA_ERR_WORKSPACE;
+    CUtensorMap mq, mk, mv;
+    if (!encode_grid_map(&mq, q, g) || !encode_grid_map(&mk, k, g) || !encode_grid_map(&mv, v, g))
+        return VSA_ERR_CUDA;
+    vsa::FineArgs a;
+    a.g = g;
+    a.mq = &mq;
+    a.mk = &mk;
+    a.mv = &mv;
+    a.block_idx = block_idx;
+    a.topk = topk;
+    a.lin_image = nullptr;
+    a.out = out;
+    a.out32 = out_f32;
+    a.lse = lse;
+    a.status = static_cast<int*>(workspace);
+    return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
+}
+
+vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                               const float* out_f32, const vsa_bf16* dout, const int32_t* block_idx,
+                               const float* lse, vsa_bf16* dq, vsa_bf16* dk, vsa_bf16* dv, int B,
+                               int heads, int head_dim, int T, int H, int W, int tt, int th, int tw,
+                               int topk, void* workspace, size_t workspace_bytes,
+                               vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (s != VSA_OK) return s;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
+    for (const void* p : {(const void*)q, (const void*)k, (const void*)v, (const void*)out_f32,
+                          (const void*)dout, (const void*)block_idx, (const void*)lse, (const void*)dq,
+                          (const void*)dk, (const void*)dv})
+        if (!aligned16(p)) return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes + vsa::bwd_scratch_bytes(g, topk)) return VSA_ERR_WORKSPACE;
+    CUtensorMap mq, mk, mv, mg;
+    if (!encode_grid_map(&mq, q, g) || !encode_grid_map(&mk, k, g) || !encode_grid_map(&mv, v, g) ||
+        !encode_grid_map(&mg, dout, g))
+        return VSA_ERR_CUDA;
+    vsa::BwdArgs a;
+    a.g = g;
+    a.mq = &mq;
+    a.mk = &mk;
+    a.mv = &mv;
+    a.mg = &mg;
+    a.block_idx = block_idx;
+    a.topk = topk;
+    a.out32 = out_f32;
+    a.dout = dout;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.scratch = static_cast<uint8_t*>(workspace) + kStatusBytes;
+    a.status = static_cast<int*>(workspace);
+    return from_cuda(vsa::launch_fine_bwd(a, (cudaStream_t)stream));
 }
 
 vsa_status vsa_device_status(void* workspace, vsa_stream_t stream) {

@@ -90,7 +90,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                  const __grid_constant__ CUtensorMap mv, const Grid g,
                  const int32_t* __restrict__ block_idx, const int topk, const float scale_log2,
                  const int ragged, const uint8_t* __restrict__ lin_image,
-                 __nv_bfloat16* __restrict__ out, int* status) {
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ out32, float* __restrict__ lse,
+                 int* status) {
     using C = FineCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
@@ -396,6 +397,9 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             const bool valid = dt < qc.vt && dh < qc.vh && dw < qc.vw;
             const long long n = ((long long)(qc.t0 + dt) * g.H + (qc.h0 + dh)) * g.W + (qc.w0 + dw);
             __nv_bfloat16* orow = out + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
+            // log2 of the softmax normaliser of the scaled scores (for the
+            // backward pass); +inf marks padded query slots (zero weight there)
+            if (lse && hf == 0) lse[row_id * 64 + r] = valid ? sm.m_run + __log2f(l) : INFINITY;
 #pragma unroll
             for (int c0 = 0; c0 < D / 2; c0 += 16) {
                 float o[16];
@@ -430,6 +434,13 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 if (valid) {
                     reinterpret_cast<uint4*>(orow + c0)[0] = w0;
                     reinterpret_cast<uint4*>(orow + c0)[1] = w1;
+                    if (out32) {                       // fp32 copy for the backward pass
+                        float4* o4 = reinterpret_cast<float4*>(
+                            out32 + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2) + c0);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o4[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                    }
                 }
             }
         }
@@ -460,7 +471,7 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     const int ragged = (a.g.T % a.g.tt) || (a.g.H % a.g.th) || (a.g.W % a.g.tw);
     fine_attn_kernel<D, LIN><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
         *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged,
-        static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.status);
+        static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.out32, a.lse, a.status);
     return cudaGetLastError();
 }
 

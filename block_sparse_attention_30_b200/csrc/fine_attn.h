@@ -18,6 +18,9 @@ struct FineArgs {
     const void* lin_image;       // optional linear-branch operand images, one per
                                  // (b, head) (linear_image_bytes(d) each, see linear.h)
     void* out;                   // bf16 [B][N][heads][d]
+    float* out32;                // optional fp32 copy of out (for the backward pass)
+    float* lse;                  // optional [B][heads][nt][64]: log2 softmax normaliser
+                                 // of the scaled scores per cube slot (+inf if padded)
     int* status;                 // device status word
 };
 

@@ -1,0 +1,621 @@
+// fine_bwd.cu -- backward pass of the fine block-sparse attention on sm_100a.
+//
+// The sparse branch is trainable ("FastVideo 稀疏蒸馏技术深度解析",
+// omica.com.cn, section "2. 视频稀疏注意力VSA"; TurboDiffusion article,
+// dolphinsci.com, section "稀疏、蒸馏与全链路量化").  With the selection held
+// fixed and P the softmax of the scaled scores over the kept keys,
+//     dV = P^T dO,   dP = dO V^T,   dS = P o (dP - D),   D = rowsum(dO o O),
+//     dQ = dS K / sqrt(d),          dK = dS^T Q / sqrt(d).
+// P is recomputed from the forward's per-row log2 normaliser (lse).
+//
+// Kernels:
+//   delta_kernel   D per cube slot, fp32 (0 for padded slots).
+//   csr_*          the transpose of the block index: for every key cube the
+//                  ascending list of query cubes that kept it (deterministic).
+//   dq_kernel      one CTA per query cube: per kept key-cube pair, S = Q K^T
+//                  (TMEM lanes 0-15) and dP = dO V^T (lanes 16-31 of the same
+//                  columns) on the tensor cores, dS written as bf16 over S by
+//                  the softmax warps, then dQ += dS K (A = dS from TMEM).
+//   dkdv_kernel    one CTA per key cube: per pair of query cubes that kept it,
+//                  S^T = K Q^T and dP^T = V dO^T, P^T and dS^T written as bf16
+//                  over them, then dV += P^T dO (lanes 0-15) and
+//                  dK += dS^T Q (lanes 16-31) accumulate in TMEM.
+// One K/Q tile serves as the K-major operand of one product and the MN-major
+// operand of the other, as V does in the forward.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "fine_bwd.h"
+#include "sm100.cuh"
+
+namespace vsa {
+using namespace sm100;
+
+// ------------------------------------------------------------------ delta
+// One warp per cube slot: D = sum_c dO[n][c] O[n][c] over the slot's token row,
+// with the forward's fp32 output (its bf16 rounding, 2^-9 relative, would
+// otherwise enter dQ as -dD sum_m P_m k_m / sqrt(d), which does not shrink
+// with dQ when the kept keys share a large common component).
+__global__ void __launch_bounds__(256)
+delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout, const Grid g,
+             float* __restrict__ delta) {
+    const long long slot = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)g.B * g.heads * g.nt;
+    if (slot >= rows * 64) return;
+    const long long row = slot / 64;
+    const int s = (int)(slot % 64);
+    const int i = (int)(row % g.nt), bh = (int)(row / g.nt);
+    const int head = bh % g.heads, b = bh / g.heads;
+    const TileCoord c = tile_coord(g, i);
+    const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
+    float acc = 0.f;
+    if (dt < c.vt && dh < c.vh && dw < c.vw) {
+        const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
+        const long long base = (((long long)b * g.N + n) * g.heads + head) * g.d;
+        for (int e = lane * 2; e < g.d; e += 64) {
+            const float2 x = *reinterpret_cast<const float2*>(o + base + e);
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + base + e));
+            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) delta[slot] = acc;
+}
+
+// ---------------------------------------------------------------- transpose
+// One thread per (b*heads, key cube j): count (pass 0) or list (pass 1) the
+// query cubes i whose ascending block-index row contains j, in increasing i.
+__device__ __forceinline__ bool row_has(const int32_t* row, int k, int j) {
+    int lo = 0, hi = k - 1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int x = __ldg(row + mid);
+        if (x == j) return true;
+        if (x < j) lo = mid + 1; else hi = mid - 1;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(256)
+csr_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, const int pass,
+           int32_t* __restrict__ off, int32_t* __restrict__ entries) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long bhs = (long long)g.B * g.heads;
+    if (t >= bhs * g.nt) return;
+    const long long bh = t / g.nt;
+    const int j = (int)(t % g.nt);
+    const int32_t* rows = idx + bh * g.nt * k;
+    int32_t* o = off + bh * (g.nt + 1);
+    if (pass == 0) {
+        int cnt = 0;
+        for (int i = 0; i < g.nt; ++i) cnt += row_has(rows + (long long)i * k, k, j);
+        o[j + 1] = cnt;                                   // counts; scanned by csr_scan_kernel
+    } else {
+        int32_t* e = entries + bh * g.nt * k + o[j];
+        int c = 0;
+        for (int i = 0; i < g.nt; ++i)
+            if (row_has(rows + (long long)i * k, k, j)) e[c++] = i;
+    }
+}
+
+// One CTA per b*heads: off[0] = 0, off[j+1] = sum of the counts up to j.
+__global__ void __launch_bounds__(1024)
+csr_scan_kernel(const Grid g, int32_t* __restrict__ off) {
+    __shared__ int32_t carry;
+    int32_t* o = off + (long long)blockIdx.x * (g.nt + 1);
+    if (threadIdx.x == 0) { carry = 0; o[0] = 0; }
+    __syncthreads();
+    for (int base = 0; base < g.nt; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        int v = j < g.nt ? o[j + 1] : 0;
+        // inclusive scan of this block of counts
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        __shared__ int32_t wsum[32];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, d);
+            if (lane >= d) v += y;
+        }
+        if (lane == 31) wsum[warp] = v;
+        __syncthreads();
+        if (warp == 0) {
+            int w = wsum[lane];
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, d);
+                if (lane >= d) w += y;
+            }
+            wsum[lane] = w;
+        }
+        __syncthreads();
+        const int incl = v + (warp > 0 ? wsum[warp - 1] : 0) + carry;
+        if (j < g.nt) o[j + 1] = incl;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = incl;
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------- shared layout
+template <int D>
+struct BwdCfg {
+    static constexpr int NCH = D / 64;
+    static constexpr int CUBE_BYTES = 64 * D * 2;        // one cube of one tensor (bf16)
+    static constexpr int PAIR_BYTES = 2 * CUBE_BYTES;
+    static constexpr int CHUNK_STRIDE = 128 * 128;       // bytes between d chunks of a pair
+    static constexpr int TMEM_COLS = 256;
+    static constexpr int ACC_COL = 0;                    // dQ | dV (lanes 0-15), dK (lanes 16-31)
+    static constexpr int S_COL = 128;                    // S / P (lanes 0-15), dP / dS (lanes 16-31)
+};
+
+struct BwdBars {
+    uint64_t a_full;                 // the CTA's own cube(s): Q + dO, or K + V
+    uint64_t x_full, x_empty;        // pair ring 1 (K pairs / Q pairs)
+    uint64_t y_full, y_empty;        // pair ring 2 (V pairs / dO pairs)
+    uint64_t s_full, ds_full, mma_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Loads one key/query cube pair (cubes jt[0..ntl)) of the tensor behind `map`
+// into a pair buffer: chunk c of cube t at c * CHUNK_STRIDE + t * 8192.
+template <int D>
+__device__ __forceinline__ void load_pair(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const Grid& g,
+                                          const int* jt, int ntl, int head, int b) {
+    using C = BwdCfg<D>;
+    for (int t = 0; t < ntl; ++t) {
+        const TileCoord kc = tile_coord(g, jt[t]);
+        for (int ch = 0; ch < C::NCH; ++ch)
+            tma_load_5d(dst + ch * C::CHUNK_STRIDE + t * 8192, map, bar, head * D + 64 * ch, kc.w0, kc.h0, kc.t0, b);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void load_cube(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const Grid& g,
+                                          int j, int head, int b) {
+    const TileCoord c = tile_coord(g, j);
+    for (int ch = 0; ch < D / 64; ++ch)
+        tma_load_5d(dst + ch * 8192, map, bar, head * D + 64 * ch, c.w0, c.h0, c.t0, b);
+}
+
+// Writes half a row (D/2 features) of an fp32 TMEM accumulator, times `scale`,
+// as bf16 to grid order.
+template <int D>
+__device__ __forceinline__ void store_half_row(uint32_t taddr, float scale, __nv_bfloat16* dst, bool valid) {
+#pragma unroll
+    for (int c0 = 0; c0 < D / 2; c0 += 16) {
+        float o[16];
+        tmem_ld_16x32bx2_x16<D / 2>(taddr + c0, o);
+        tmem_wait_ld();
+        uint4 w0, w1;
+        w0.x = pack_bf16x2(o[0] * scale, o[1] * scale);
+        w0.y = pack_bf16x2(o[2] * scale, o[3] * scale);
+        w0.z = pack_bf16x2(o[4] * scale, o[5] * scale);
+        w0.w = pack_bf16x2(o[6] * scale, o[7] * scale);
+        w1.x = pack_bf16x2(o[8] * scale, o[9] * scale);
+        w1.y = pack_bf16x2(o[10] * scale, o[11] * scale);
+        w1.z = pack_bf16x2(o[12] * scale, o[13] * scale);
+        w1.w = pack_bf16x2(o[14] * scale, o[15] * scale);
+        if (valid) {
+            reinterpret_cast<uint4*>(dst + c0)[0] = w0;
+            reinterpret_cast<uint4*>(dst + c0)[1] = w1;
+        }
+    }
+}
+
+__device__ __forceinline__ void store_zero_half_row(int half, __nv_bfloat16* dst, bool valid) {
+    if (!valid) return;
+    for (int c = 0; c < half; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);
+}
+
+// -------------------------------------------------------------------- dQ
+// 224 threads: warps 0-3 softmax (rows 16w..16w+15, each row split in two
+// 64-key halves over lanes t and t+16), warp 4 Q + dO + K pairs, warp 5 MMA,
+// warp 6 V pairs.
+template <int D>
+__global__ void __launch_bounds__(224, 2)
+dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+          const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg, const Grid g,
+          const int32_t* __restrict__ block_idx, const int topk, const float scale_log2, const int ragged,
+          const float* __restrict__ lse, const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq,
+          int* status) {
+    using C = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) report(status, kStatusMisaligned);
+        return;
+    }
+    uint8_t* sQ = smem;
+    uint8_t* sG = sQ + C::CUBE_BYTES;
+    uint8_t* sK = sG + C::CUBE_BYTES;
+    uint8_t* sV = sK + C::PAIR_BYTES;
+    BwdBars* bars = reinterpret_cast<BwdBars*>(sV + C::PAIR_BYTES);
+    volatile int* abort_flag = &bars->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long row_id = blockIdx.x;
+    const int i = (int)(row_id % g.nt);
+    const int bh = (int)(row_id / g.nt);
+    const int head = bh % g.heads, b = bh / g.heads;
+    const int32_t* my_idx = block_idx + row_id * topk;
+    const int n_pairs = (topk + 1) >> 1;
+
+    if (tid == 0) {
+        bars->abort = 0;
+        mbar_init(&bars->a_full, 1);
+        mbar_init(&bars->x_full, 1); mbar_init(&bars->x_empty, 1);
+        mbar_init(&bars->y_full, 1); mbar_init(&bars->y_empty, 1);
+        mbar_init(&bars->s_full, 1); mbar_init(&bars->ds_full, 128); mbar_init(&bars->mma_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = bars->tmem_base;
+    auto fail = [&]() { *abort_flag = 1; report(status, kStatusTimeout); };
+
+    if (warp == 4 || warp == 6) {
+        if (lane == 0) {
+            const bool is_k = warp == 4;
+            uint64_t* full = is_k ? &bars->x_full : &bars->y_full;
+            uint64_t* empty = is_k ? &bars->x_empty : &bars->y_empty;
+            uint8_t* ring = is_k ? sK : sV;
+            const CUtensorMap* map = is_k ? &mk : &mv;
+            if (is_k) {
+                mbar_arrive_expect_tx(&bars->a_full, 2 * C::CUBE_BYTES);
+                load_cube<D>(sQ, &mq, &bars->a_full, g, i, head, b);
+                load_cube<D>(sG, &mg, &bars->a_full, g, i, head, b);
+            }
+            int issued = 0;
+            for (int p = 0; p < n_pairs; ++p) {
+                const int ntl = min(2, topk - 2 * p);
+                int jt[2] = {__ldg(my_idx + 2 * p), ntl > 1 ? __ldg(my_idx + 2 * p + 1) : 0};
+                for (int t = 0; t < ntl; ++t)
+                    if (jt[t] < 0 || jt[t] >= g.nt) { if (is_k) report(status, kStatusBadIndex); jt[t] = 0; }
+                if (p >= 1 && !mbar_wait(empty, (p - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(full, ntl * C::CUBE_BYTES);
+                load_pair<D>(ring, map, full, g, jt, ntl, head, b);
+                ++issued;
+            }
+            if (*abort_flag) {
+                if (is_k) wait_noabort(&bars->a_full, 0);
+                if (issued > 0) wait_noabort(full, (issued - 1) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            const uint32_t q_addr = smem_u32(sQ), g_addr = smem_u32(sG);
+            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            const uint32_t tS = tbase + C::S_COL, tP = tbase + C::S_COL + (16u << 16), tAcc = tbase + C::ACC_COL;
+            const uint32_t id_acc = idesc_bf16_f32(64, D, false, true);
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
+            for (int p = 0; ok && p < n_pairs; ++p) {
+                const int nkeys = min(2, topk - 2 * p) * 64;
+                if (!mbar_wait(&bars->x_full, p & 1, abort_flag) || !mbar_wait(&bars->y_full, p & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // S = Q K^T and dP = dO V^T (K-major)
+                    const uint32_t ao = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32;
+                    mma_bf16_ss(tS, smem_desc_sw128(q_addr + ao, 16, 1024), smem_desc_sw128(k_addr + bo, 16, 1024), id_s, kk > 0);
+                    mma_bf16_ss(tP, smem_desc_sw128(g_addr + ao, 16, 1024), smem_desc_sw128(v_addr + bo, 16, 1024), id_s, kk > 0);
+                }
+                mma_commit(&bars->s_full);
+                mma_commit(&bars->y_empty);                  // V read by dP only
+                if (!mbar_wait(&bars->ds_full, p & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kk = 0; kk < nkeys / 16; ++kk) {    // dQ += dS K (K as MN-major B)
+                    const uint64_t bd = smem_desc_sw128(k_addr + kk * 2048, C::CHUNK_STRIDE, 1024);
+                    mma_bf16_ts(tAcc, tS + kk * 8, bd, id_acc, (p > 0 || kk > 0));
+                }
+                mma_commit(&bars->x_empty);
+            }
+            if (!ok) fail();
+            mma_commit(&bars->mma_done);
+            wait_noabort(&bars->mma_done, 0);
+        }
+    } else {
+        // softmax warps: P = exp2(s * scale_log2 - lse), dS = P (dP - D)
+        const int r = 16 * warp + (lane & 15), hf = lane >> 4;
+        const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
+        const uint32_t tS = lane_base + C::S_COL, tP = lane_base + C::S_COL + (16u << 16);
+        const float l2 = __ldg(lse + row_id * 64 + r);
+        const float dl = __ldg(delta + row_id * 64 + r);
+        bool ok = true;
+        for (int p = 0; p < n_pairs; ++p) {
+            const int ntl = min(2, topk - 2 * p);
+            uint64_t vmask = hf < ntl ? ~0ull : 0ull;
+            if (ragged && hf < ntl) {
+                int j = __ldg(my_idx + 2 * p + hf);
+                if (j < 0 || j >= g.nt) j = 0;
+                vmask = valid_slot_mask(g, tile_coord(g, j));
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, p & 1, abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            float s[64], dp[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 16) {
+                tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
+                tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
+            }
+            tmem_wait_ld();
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const bool v0 = (vmask >> (2 * e)) & 1ull, v1 = (vmask >> (2 * e + 1)) & 1ull;
+                const float p0 = v0 ? ex2(fmaf(s[2 * e], scale_log2, -l2)) : 0.f;
+                const float p1 = v1 ? ex2(fmaf(s[2 * e + 1], scale_log2, -l2)) : 0.f;
+                pk[e] = pack_bf16x2(p0 * (dp[2 * e] - dl), p1 * (dp[2 * e + 1] - dl));
+            }
+            tmem_st_16x32bx2_x32(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_full);
+        }
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag))) ok = false;
+        if (!ok) fail();
+        if (ok) {
+            tc_fence_after();
+            const TileCoord qc = tile_coord(g, i);
+            const int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
+            const bool valid = dt < qc.vt && dh < qc.vh && dw < qc.vw;
+            const long long n = ((long long)(qc.t0 + dt) * g.H + (qc.h0 + dh)) * g.W + (qc.w0 + dw);
+            __nv_bfloat16* drow = dq + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
+            // scale_log2 / log2(e) = 1/sqrt(d)
+            store_half_row<D>(lane_base + C::ACC_COL, scale_log2 * 0.6931471805599453f, drow, valid);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ dK, dV
+// One CTA per key cube: warps 0-3 softmax (key rows 16w..16w+15; lanes t and
+// t+16 hold query cube 0 and 1 of the pair), warp 4 K + V cubes and the Q
+// pairs (+ their lse), warp 5 MMA, warp 6 the dO pairs (+ their D).
+template <int D>
+__global__ void __launch_bounds__(224, 2)
+dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+            const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg, const Grid g,
+            const int topk, const float scale_log2, const int32_t* __restrict__ off,
+            const int32_t* __restrict__ entries, const float* __restrict__ lse,
+            const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+            int* status) {
+    using C = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) report(status, kStatusMisaligned);
+        return;
+    }
+    uint8_t* sK = smem;
+    uint8_t* sV = sK + C::CUBE_BYTES;
+    uint8_t* sQ = sV + C::CUBE_BYTES;         // pair of query cubes
+    uint8_t* sG = sQ + C::PAIR_BYTES;         // pair of dO cubes
+    float* sL = reinterpret_cast<float*>(sG + C::PAIR_BYTES);   // lse of the pair's 128 query slots
+    float* sD = sL + 128;                                         // D of the pair's 128 query slots
+    BwdBars* bars = reinterpret_cast<BwdBars*>(sD + 128);
+    volatile int* abort_flag = &bars->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long row_id = blockIdx.x;          // (b*heads + head)*nt + j
+    const int j = (int)(row_id % g.nt);
+    const int bh = (int)(row_id / g.nt);
+    const int head = bh % g.heads, b = bh / g.heads;
+    const int32_t* o = off + (long long)bh * (g.nt + 1);
+    const int e0 = __ldg(o + j), nq = __ldg(o + j + 1) - e0;
+    const int32_t* my_q = entries + (long long)bh * g.nt * topk + e0;    // ascending query cubes
+    const int n_steps = (nq + 1) >> 1;
+    const long long qrow0 = (long long)bh * g.nt;                          // row id of query cube 0
+
+    if (tid == 0) {
+        bars->abort = 0;
+        mbar_init(&bars->a_full, 1);
+        mbar_init(&bars->x_full, 1); mbar_init(&bars->x_empty, 1);
+        mbar_init(&bars->y_full, 1); mbar_init(&bars->y_empty, 1);
+        mbar_init(&bars->s_full, 1); mbar_init(&bars->ds_full, 128); mbar_init(&bars->mma_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = bars->tmem_base;
+    auto fail = [&]() { *abort_flag = 1; report(status, kStatusTimeout); };
+
+    if (warp == 4 || warp == 6) {
+        if (lane == 0) {
+            const bool is_q = warp == 4;
+            uint64_t* full = is_q ? &bars->x_full : &bars->y_full;
+            uint64_t* empty = is_q ? &bars->x_empty : &bars->y_empty;
+            uint8_t* ring = is_q ? sQ : sG;
+            float* side = is_q ? sL : sD;
+            const float* side_src = is_q ? lse : delta;
+            const CUtensorMap* map = is_q ? &mq : &mg;
+            if (is_q) {
+                mbar_arrive_expect_tx(&bars->a_full, 2 * C::CUBE_BYTES);
+                load_cube<D>(sK, &mk, &bars->a_full, g, j, head, b);
+                load_cube<D>(sV, &mv, &bars->a_full, g, j, head, b);
+            }
+            int issued = 0;
+            for (int st = 0; st < n_steps; ++st) {
+                const int ntl = min(2, nq - 2 * st);
+                int it[2] = {__ldg(my_q + 2 * st), ntl > 1 ? __ldg(my_q + 2 * st + 1) : 0};
+                for (int t = 0; t < ntl; ++t)
+                    if (it[t] < 0 || it[t] >= g.nt) { report(status, kStatusBadIndex); it[t] = 0; }
+                if (st >= 1 && !mbar_wait(empty, (st - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(full, ntl * (C::CUBE_BYTES + 256));
+                load_pair<D>(ring, map, full, g, it, ntl, head, b);
+                for (int t = 0; t < ntl; ++t)
+                    bulk_load(side + 64 * t, side_src + (qrow0 + it[t]) * 64, 256, full);
+                ++issued;
+            }
+            if (*abort_flag) {
+                if (is_q) wait_noabort(&bars->a_full, 0);
+                if (issued > 0) wait_noabort(full, (issued - 1) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            const uint32_t q_addr = smem_u32(sQ), g_addr = smem_u32(sG);
+            const uint32_t tS = tbase + C::S_COL, tP = tbase + C::S_COL + (16u << 16);
+            const uint32_t tdV = tbase + C::ACC_COL, tdK = tbase + C::ACC_COL + (16u << 16);
+            const uint32_t id_acc = idesc_bf16_f32(64, D, false, true);
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
+            for (int st = 0; ok && st < n_steps; ++st) {
+                const int nqs = min(2, nq - 2 * st) * 64;
+                if (!mbar_wait(&bars->x_full, st & 1, abort_flag) || !mbar_wait(&bars->y_full, st & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t id_s = idesc_bf16_f32(64, nqs, false, false);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // S^T = K Q^T, dP^T = V dO^T
+                    const uint32_t ao = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32;
+                    mma_bf16_ss(tS, smem_desc_sw128(k_addr + ao, 16, 1024), smem_desc_sw128(q_addr + bo, 16, 1024), id_s, kk > 0);
+                    mma_bf16_ss(tP, smem_desc_sw128(v_addr + ao, 16, 1024), smem_desc_sw128(g_addr + bo, 16, 1024), id_s, kk > 0);
+                }
+                mma_commit(&bars->s_full);
+                if (!mbar_wait(&bars->ds_full, st & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kk = 0; kk < nqs / 16; ++kk) {      // dV += P^T dO, dK += dS^T Q
+                    mma_bf16_ts(tdV, tS + kk * 8, smem_desc_sw128(g_addr + kk * 2048, C::CHUNK_STRIDE, 1024), id_acc, (st > 0 || kk > 0));
+                    mma_bf16_ts(tdK, tP + kk * 8, smem_desc_sw128(q_addr + kk * 2048, C::CHUNK_STRIDE, 1024), id_acc, (st > 0 || kk > 0));
+                }
+                mma_commit(&bars->x_empty);
+                mma_commit(&bars->y_empty);
+            }
+            if (!ok) fail();
+            mma_commit(&bars->mma_done);
+            wait_noabort(&bars->mma_done, 0);
+        }
+    } else {
+        // softmax warps: P^T = exp2(s * scale_log2 - lse[q]), dS^T = P^T (dP^T - D[q])
+        const int r = 16 * warp + (lane & 15), hf = lane >> 4;   // key row, query cube of the pair
+        const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
+        const uint32_t tS = lane_base + C::S_COL, tP = lane_base + C::S_COL + (16u << 16);
+        bool ok = true;
+        for (int st = 0; st < n_steps; ++st) {
+            const int ntl = min(2, nq - 2 * st);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, st & 1, abort_flag))) { ok = false; break; }
+            // lse and D of this pair landed with the Q / dO pairs
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, st & 1, abort_flag) &&
+                                             mbar_wait(&bars->y_full, st & 1, abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            float s[64], dp[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 16) {
+                tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
+                tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
+            }
+            tmem_wait_ld();
+            const bool have = hf < ntl;                   // odd tail: the second query cube is absent
+            const float* Ls = sL + 64 * hf;
+            const float* Ds = sD + 64 * hf;
+            uint32_t pk[32], dk32[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float p0 = have ? ex2(fmaf(s[2 * e], scale_log2, -Ls[2 * e])) : 0.f;
+                const float p1 = have ? ex2(fmaf(s[2 * e + 1], scale_log2, -Ls[2 * e + 1])) : 0.f;
+                pk[e] = pack_bf16x2(p0, p1);
+                dk32[e] = pack_bf16x2(p0 * (dp[2 * e] - Ds[2 * e]), p1 * (dp[2 * e + 1] - Ds[2 * e + 1]));
+            }
+            tmem_st_16x32bx2_x32(tS, pk);
+            tmem_st_16x32bx2_x32(tP, dk32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_full);
+        }
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag))) ok = false;
+        if (!ok) fail();
+        if (ok) {
+            tc_fence_after();
+            const TileCoord kc = tile_coord(g, j);
+            const int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
+            const bool valid = dt < kc.vt && dh < kc.vh && dw < kc.vw;
+            const long long n = ((long long)(kc.t0 + dt) * g.H + (kc.h0 + dh)) * g.W + (kc.w0 + dw);
+            const long long base = (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
+            if (n_steps > 0) {
+                store_half_row<D>(lane_base + C::ACC_COL, 1.f, dv + base, valid);
+                store_half_row<D>(lane_base + C::ACC_COL + (16u << 16), scale_log2 * 0.6931471805599453f, dk + base, valid);
+            } else {                                      // no query cube kept this key cube
+                store_zero_half_row(D / 2, dv + base, valid);
+                store_zero_half_row(D / 2, dk + base, valid);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+size_t bwd_scratch_bytes(const Grid& g, int topk) {
+    const size_t rows = (size_t)g.B * g.heads * g.nt;
+    const size_t delta = rows * 64 * sizeof(float);
+    const size_t offs = (size_t)g.B * g.heads * (g.nt + 1) * sizeof(int32_t);
+    const size_t ents = rows * (size_t)topk * sizeof(int32_t);
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return up(delta) + up(offs) + up(ents);
+}
+
+template <int D>
+static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
+    using C = BwdCfg<D>;
+    const Grid& g = a.g;
+    static int configured_device = -1;
+    constexpr int DQ_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 256;
+    constexpr int DKDV_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 1024 + 256;
+    static_assert(sizeof(BwdBars) <= 256, "barrier block");
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_device != dev) {
+        e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DKDV_SMEM);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    const long long rows = (long long)g.B * g.heads * g.nt;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    uint8_t* scratch = static_cast<uint8_t*>(a.scratch);
+    float* delta = reinterpret_cast<float*>(scratch);
+    int32_t* off = reinterpret_cast<int32_t*>(scratch + up(rows * 64 * sizeof(float)));
+    int32_t* ents = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(off) +
+                                               up((size_t)g.B * g.heads * (g.nt + 1) * sizeof(int32_t)));
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    const int ragged = (g.T % g.tt) || (g.H % g.th) || (g.W % g.tw);
+
+    delta_kernel<<<(unsigned)((rows * 64 + 7) / 8), 256, 0, stream>>>(
+        a.out32, static_cast<const __nv_bfloat16*>(a.dout), g, delta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long keys = (long long)g.B * g.heads * g.nt;
+    csr_kernel<<<(unsigned)((keys + 255) / 256), 256, 0, stream>>>(a.block_idx, g, a.topk, 0, off, ents);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    csr_scan_kernel<<<(unsigned)(g.B * g.heads), 1024, 0, stream>>>(g, off);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    csr_kernel<<<(unsigned)((keys + 255) / 256), 256, 0, stream>>>(a.block_idx, g, a.topk, 1, off, ents);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dq_kernel<D><<<(unsigned)rows, 224, DQ_SMEM, stream>>>(
+        *a.mq, *a.mk, *a.mv, *a.mg, g, a.block_idx, a.topk, scale_log2, ragged, a.lse, delta,
+        static_cast<__nv_bfloat16*>(a.dq), a.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dkdv_kernel<D><<<(unsigned)rows, 224, DKDV_SMEM, stream>>>(
+        *a.mq, *a.mk, *a.mv, *a.mg, g, a.topk, scale_log2, off, ents, a.lse, delta,
+        static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fine_bwd(const BwdArgs& a, cudaStream_t stream) {
+    return a.g.d == 128 ? launch_bwd_impl<128>(a, stream) : launch_bwd_impl<64>(a, stream);
+}
+
+}  // namespace vsa

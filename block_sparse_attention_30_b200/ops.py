@@ -96,6 +96,28 @@ def vsa_sparse_attn_fwd(q, k, v, block_idx, out, T, H, W, topk, workspace, lin_S
         workspace.numel(), _stream(stream)))
 
 
+def vsa_sparse_attn_fwd_train(q, k, v, block_idx, out, out_f32, lse, T, H, W, topk, workspace,
+                              tile=(4, 4, 4), stream=None):
+    """Sparse-branch forward that also writes, for the backward pass, an fp32
+    copy of the output and lse[B][heads][nt][64] (fp32)."""
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_sparse_attn_fwd_train", _lib.lib().vsa_sparse_attn_fwd_train(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), block_idx.data_ptr(), out.data_ptr(),
+        out_f32.data_ptr(), lse.data_ptr(), *_shape(B, heads, d, T, H, W, tile), topk,
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def vsa_sparse_attn_bwd(q, k, v, out_f32, dout, block_idx, lse, dq, dk, dv, T, H, W, topk, workspace,
+                        tile=(4, 4, 4), stream=None):
+    """Gradients dq, dk, dv (bf16, written in place) of the fine pass."""
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_sparse_attn_bwd", _lib.lib().vsa_sparse_attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out_f32.data_ptr(), dout.data_ptr(),
+        block_idx.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        *_shape(B, heads, d, T, H, W, tile), topk, workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
+
+
 def vsa_device_status(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = VSA_OK)."""
     return _lib.lib().vsa_device_status(workspace.data_ptr(), _stream(stream))

@@ -80,7 +80,8 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
  * holds either the selection's fp64 cube means of q and k
  * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the
  * linear branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is
- * larger.  Returns 0 for invalid shapes.  The
+ * larger (the backward pass's row terms and block-index transpose fit it
+ * too).  Returns 0 for invalid shapes.  The
  * same workspace may be passed to every call of one forward pass; calls that
  * share a workspace must be ordered on one stream. */
 size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W,
@@ -142,6 +143,38 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
                                const int32_t* block_idx, const float* lin_S,
                                const float* lin_z, vsa_bf16* out, int B, int heads,
                                int head_dim, int T, int H, int W, int tt, int th, int tw,
+                               int topk, void* workspace, size_t workspace_bytes,
+                               vsa_stream_t stream);
+
+/* Training forward: vsa_sparse_attn_fwd for the sparse branch alone that
+ * also writes, for the backward pass, out_f32 (the same output in fp32,
+ * [B][N][heads][d], padded slots not written) and lse[B][heads][nt][64]
+ * (fp32, one value per cube slot): log2 of the softmax normaliser of the
+ * row's scaled scores, i.e. m + log2(sum_m 2^(s_m*log2(e)/sqrt(d) - m));
+ * +inf for padded slots.  Needs vsa_workspace_bytes() of workspace (status
+ * word only). */
+vsa_status vsa_sparse_attn_fwd_train(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                                     const int32_t* block_idx, vsa_bf16* out, float* out_f32,
+                                     float* lse, int B, int heads, int head_dim, int T, int H, int W,
+                                     int tt, int th, int tw, int topk, void* workspace,
+                                     size_t workspace_bytes, vsa_stream_t stream);
+
+/* Backward of the fine pass (the sparse branch is trainable: "FastVideo
+ * 稀疏蒸馏技术深度解析", section "2. 视频稀疏注意力VSA"; TurboDiffusion article,
+ * section "稀疏、蒸馏与全链路量化"), with block_idx held fixed: given q, k, v
+ * and the output gradient `dout` (bf16 [B][N][heads][d]) and out_f32 and lse
+ * from vsa_sparse_attn_fwd_train, writes bf16 dq, dk, dv (same layout,
+ * fully overwritten; keys no query cube kept get 0):
+ *     dv = P^T dout, dS = P o (dout v^T - rowsum(dout o out_f32)),
+ *     dq = dS k / sqrt(d), dk = dS^T q / sqrt(d),
+ * P recomputed from lse, products on the tensor cores with fp32
+ * accumulation.  Uses the workspace scratch (vsa_workspace_bytes()) for the
+ * row terms and the transpose of block_idx, so it overwrites an earlier
+ * selection's scratch on the same workspace (not block_idx). */
+vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                               const float* out_f32, const vsa_bf16* dout, const int32_t* block_idx,
+                               const float* lse, vsa_bf16* dq, vsa_bf16* dk, vsa_bf16* dv, int B,
+                               int heads, int head_dim, int T, int H, int W, int tt, int th, int tw,
                                int topk, void* workspace, size_t workspace_bytes,
                                vsa_stream_t stream);
 

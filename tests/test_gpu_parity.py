@@ -376,3 +376,85 @@ def test_sparse97_linear_workload_sampled(ops):
         ref.append(part[r][slots[i] >= 0] + lin)
         got.append(out[b, torch.as_tensor(toks), head].float().cpu().double().numpy())
     check_close(np.concatenate(got), np.concatenate(ref))
+
+
+# ------------------------------------------------------------- backward pass
+# bf16 P and dS feed the tensor cores (relative rounding 2^-9 each) with fp32
+# accumulation, D = rowsum(dO o O) uses the fp32 forward output, and the
+# gradients are rounded to bf16 (2^-9): a few 1e-3 of the gradient scale
+# (measured 0.2-0.6 %).  Bound: relative Frobenius error <= 1e-2 and max-abs
+# error <= 2e-2 x the largest reference magnitude, per gradient.
+GRAD_REL_FRO, GRAD_MAX_REL = 1e-2, 2e-2
+
+
+def check_grad(got, ref, name):
+    ref = np.asarray(ref)
+    scale = max(np.abs(ref).max(), 1e-6)
+    err = np.abs(got - ref).max()
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    print(f"{name}: max-abs {err:.3e} (scale {scale:.3e}, {err / scale:.3%}), rel-Frobenius {rel:.3%}")
+    assert err <= GRAD_MAX_REL * scale and rel <= GRAD_REL_FRO, (name, err, scale, rel)
+
+
+def run_fwd_bwd(ops, w, qd, kd, vd, idx, ws, dout, tile=None):
+    tile = w.tile if tile is None else tile
+    B, N, heads, d = qd.shape
+    nt = ops.vsa_num_tiles(w.T, w.H, w.W, tile)
+    out = torch.empty_like(qd)
+    out32 = torch.empty(qd.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, heads, nt, 64), dtype=torch.float32, device="cuda")
+    ops.vsa_sparse_attn_fwd_train(qd, kd, vd, idx, out, out32, lse, w.T, w.H, w.W, idx.shape[-1], ws, tile)
+    assert torch.equal(out32.to(torch.bfloat16), out), "the fp32 copy rounds to the bf16 output"
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    ops.vsa_sparse_attn_bwd(qd, kd, vd, out32, dout.cuda(), idx, lse, dq, dk, dv, w.T, w.H, w.W,
+                            idx.shape[-1], ws, tile)
+    assert ops.vsa_device_status(ws) == 0
+    return out, lse, dq, dk, dv
+
+
+def make_dout(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (0.5 * torch.randn(shape, generator=g)).to(torch.bfloat16)
+
+
+BWD_CASES = [
+    (4, 8, 8, 2, 128, 2, (4, 4, 4)),        # 4 cubes, even k
+    (5, 6, 7, 2, 128, 3, (4, 4, 4)),        # ragged on every axis, odd k
+    (9, 13, 10, 3, 64, 5, (4, 4, 4)),       # ragged, d = 64
+    (8, 16, 16, 2, 128, 1, (4, 4, 4)),      # k = 1
+    (8, 16, 16, 2, 128, 32, (4, 4, 4)),     # k = nt (dense)
+    (6, 10, 9, 2, 128, 9, (4, 4, 4)),       # ragged, several pairs + odd tail
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_backward_small_grids(ops, case):
+    T, H, W, heads, d, topk, tile = case
+    c = Small(T, H, W, heads, d, topk, tile, seed=hash(case) % 1000 + 1, amplitude=0.7)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    dout = make_dout(c.q.shape, seed=3)
+    out, lse, dq, dk, dv = run_fwd_bwd(ops, c, qd, kd, vd, idx, ws, dout)
+    # the training forward gives the same bf16 output as the plain one
+    out_plain = run_fine(ops, c, qd, kd, vd, idx, ws)
+    assert torch.equal(out, out_plain)
+    idx_np = idx.cpu().numpy()
+    rq, rk, rv = O.fine_bwd(c.q, c.k, c.v, dout, idx_np, 1, heads, d, T, H, W, tile)
+    for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        assert not torch.isnan(got).any(), name + " must be fully written"
+        check_grad(to_f64(got), ref, name)
+
+
+def test_backward_headline_two_heads(ops):
+    """Full-size 14B-480P backward, checked on every token of two heads."""
+    w, q, k, v, qd, kd, vd = inputs("wan14b_480p")
+    idx, ws = run_select(ops, w, qd, kd)
+    dout = make_dout(q.shape, seed=9)
+    out, lse, dq, dk, dv = run_fwd_bwd(ops, w, qd, kd, vd, idx, ws, dout)
+    hs = slice(0, 2)
+    sub = lambda x: x[:, :, hs].contiguous()
+    rq, rk, rv = O.fine_bwd(sub(q), sub(k), sub(v), sub(dout), idx[:, hs].cpu().numpy(), 1, 2,
+                            w.head_dim, w.T, w.H, w.W, w.tile)
+    for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        assert not torch.isnan(got).any(), name + " must be fully written"
+        check_grad(to_f64(got[:, :, hs]), ref, name)
