@@ -11,16 +11,18 @@
 // Kernels:
 //   delta_kernel   D per cube slot, fp32 (0 for padded slots).
 //   csr_*          the transpose of the block index: for every key cube the
-//                  ascending list of query cubes that kept it (deterministic).
-//   dq_kernel      one CTA per query cube: per kept key-cube pair, S = Q K^T
+//                  ascending list of query cubes that kept it (deterministic;
+//                  one warp per key cube).
+//   dq_body        one CTA per query cube: per kept key-cube pair, S = Q K^T
 //                  (TMEM lanes 0-15) and dP = dO V^T (lanes 16-31 of the same
 //                  columns) on the tensor cores, dS written as bf16 over S by
 //                  the softmax warps, then dQ += dS K (A = dS from TMEM).
-//   dkdv_kernel    one CTA per key cube: per pair of query cubes that kept it,
+//   dkdv_body      one CTA per key cube: per pair of query cubes that kept it,
 //                  S^T = K Q^T and dP^T = V dO^T, P^T and dS^T written as bf16
 //                  over them, then dV += P^T dO (lanes 0-15) and
 //                  dK += dS^T Q (lanes 16-31) accumulate in TMEM.
-// One K/Q tile serves as the K-major operand of one product and the MN-major
+// Both run in one launch (bwd_kernel: even CTAs dQ, odd CTAs dK/dV).  One
+// K/Q tile serves as the K-major operand of one product and the MN-major
 // operand of the other, as V does in the forward.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -37,7 +39,8 @@ using namespace sm100;
 // One warp per cube slot: D = sum_c dO[n][c] O[n][c] over the slot's token row,
 // with the forward's fp32 output (its bf16 rounding, 2^-9 relative, would
 // otherwise enter dQ as -dD sum_m P_m k_m / sqrt(d), which does not shrink
-// with dQ when the kept keys share a large common component).
+// with dQ when the kept keys share a large common component).  Each lane
+// reads 4 features at a time (16 bytes of O, 8 bytes of dO).
 __global__ void __launch_bounds__(256)
 delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout, const Grid g,
              float* __restrict__ delta) {
@@ -55,10 +58,13 @@ delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout
     if (dt < c.vt && dh < c.vh && dw < c.vw) {
         const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
         const long long base = (((long long)b * g.N + n) * g.heads + head) * g.d;
-        for (int e = lane * 2; e < g.d; e += 64) {
-            const float2 x = *reinterpret_cast<const float2*>(o + base + e);
-            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + base + e));
-            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+        for (int e = lane * 4; e < g.d; e += 128) {
+            const float4 x = *reinterpret_cast<const float4*>(o + base + e);
+            const uint2 yr = *reinterpret_cast<const uint2*>(dout + base + e);
+            acc = fmaf(x.x, __uint_as_float(yr.x << 16), acc);
+            acc = fmaf(x.y, __uint_as_float(yr.x & 0xffff0000u), acc);
+            acc = fmaf(x.z, __uint_as_float(yr.y << 16), acc);
+            acc = fmaf(x.w, __uint_as_float(yr.y & 0xffff0000u), acc);
         }
     }
 #pragma unroll
@@ -67,8 +73,10 @@ delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout
 }
 
 // ---------------------------------------------------------------- transpose
-// One thread per (b*heads, key cube j): count (pass 0) or list (pass 1) the
-// query cubes i whose ascending block-index row contains j, in increasing i.
+// One warp per (b*heads, key cube j): count (pass 0) or list (pass 1) the
+// query cubes i whose ascending block-index row contains j.  The lanes test
+// 32 consecutive i at a time; a ballot keeps the list in increasing i, so the
+// result is deterministic.
 __device__ __forceinline__ bool row_has(const int32_t* row, int k, int j) {
     int lo = 0, hi = k - 1;
     while (lo <= hi) {
@@ -83,23 +91,25 @@ __device__ __forceinline__ bool row_has(const int32_t* row, int k, int j) {
 __global__ void __launch_bounds__(256)
 csr_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, const int pass,
            int32_t* __restrict__ off, int32_t* __restrict__ entries) {
-    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
     const long long bhs = (long long)g.B * g.heads;
-    if (t >= bhs * g.nt) return;
-    const long long bh = t / g.nt;
-    const int j = (int)(t % g.nt);
+    if (wid >= bhs * g.nt) return;                    // whole warp
+    const long long bh = wid / g.nt;
+    const int j = (int)(wid % g.nt);
     const int32_t* rows = idx + bh * g.nt * k;
     int32_t* o = off + bh * (g.nt + 1);
-    if (pass == 0) {
-        int cnt = 0;
-        for (int i = 0; i < g.nt; ++i) cnt += row_has(rows + (long long)i * k, k, j);
-        o[j + 1] = cnt;                                   // counts; scanned by csr_scan_kernel
-    } else {
-        int32_t* e = entries + bh * g.nt * k + o[j];
-        int c = 0;
-        for (int i = 0; i < g.nt; ++i)
-            if (row_has(rows + (long long)i * k, k, j)) e[c++] = i;
+    int32_t* e = entries + bh * g.nt * k;
+    int base = pass == 0 ? 0 : o[j];
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i0 = 0; i0 < g.nt; i0 += 32) {
+        const int i = i0 + lane;
+        const bool has = i < g.nt && row_has(rows + (long long)i * k, k, j);
+        const unsigned ball = __ballot_sync(0xffffffffu, has);
+        if (pass == 1 && has) e[base + __popc(ball & lt)] = i;
+        base += __popc(ball);
     }
+    if (pass == 0 && lane == 0) o[j + 1] = base;      // counts; scanned by csr_scan_kernel
 }
 
 // One CTA per b*heads: off[0] = 0, off[j+1] = sum of the counts up to j.
@@ -217,18 +227,14 @@ __device__ __forceinline__ void store_zero_half_row(int half, __nv_bfloat16* dst
 // 64-key halves over lanes t and t+16), warp 4 Q + dO + K pairs, warp 5 MMA,
 // warp 6 V pairs.
 template <int D>
-__global__ void __launch_bounds__(224, 2)
-dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-          const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg, const Grid g,
-          const int32_t* __restrict__ block_idx, const int topk, const float scale_log2, const int ragged,
-          const float* __restrict__ lse, const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq,
-          int* status) {
+__device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                        const CUtensorMap& mg, const Grid& g,
+                                        const int32_t* __restrict__ block_idx, const int topk,
+                                        const float scale_log2, const int ragged,
+                                        const float* __restrict__ lse, const float* __restrict__ delta,
+                                        __nv_bfloat16* __restrict__ dq, int* status, uint8_t* smem,
+                                        const long long row_id) {
     using C = BwdCfg<D>;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    if (smem_u32(smem) & 1023) {
-        if (threadIdx.x == 0) report(status, kStatusMisaligned);
-        return;
-    }
     uint8_t* sQ = smem;
     uint8_t* sG = sQ + C::CUBE_BYTES;
     uint8_t* sK = sG + C::CUBE_BYTES;
@@ -236,7 +242,6 @@ dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     BwdBars* bars = reinterpret_cast<BwdBars*>(sV + C::PAIR_BYTES);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long row_id = blockIdx.x;
     const int i = (int)(row_id % g.nt);
     const int bh = (int)(row_id / g.nt);
     const int head = bh % g.heads, b = bh / g.heads;
@@ -381,19 +386,14 @@ dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
 // t+16 hold query cube 0 and 1 of the pair), warp 4 K + V cubes and the Q
 // pairs (+ their lse), warp 5 MMA, warp 6 the dO pairs (+ their D).
 template <int D>
-__global__ void __launch_bounds__(224, 2)
-dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-            const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg, const Grid g,
-            const int topk, const float scale_log2, const int32_t* __restrict__ off,
-            const int32_t* __restrict__ entries, const float* __restrict__ lse,
-            const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-            int* status) {
+__device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                          const CUtensorMap& mg, const Grid& g, const int topk,
+                                          const float scale_log2, const int32_t* __restrict__ off,
+                                          const int32_t* __restrict__ entries, const float* __restrict__ lse,
+                                          const float* __restrict__ delta, __nv_bfloat16* __restrict__ dk,
+                                          __nv_bfloat16* __restrict__ dv, int* status, uint8_t* smem,
+                                          const long long row_id) {
     using C = BwdCfg<D>;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    if (smem_u32(smem) & 1023) {
-        if (threadIdx.x == 0) report(status, kStatusMisaligned);
-        return;
-    }
     uint8_t* sK = smem;
     uint8_t* sV = sK + C::CUBE_BYTES;
     uint8_t* sQ = sV + C::CUBE_BYTES;         // pair of query cubes
@@ -403,8 +403,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     BwdBars* bars = reinterpret_cast<BwdBars*>(sD + 128);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long row_id = blockIdx.x;          // (b*heads + head)*nt + j
-    const int j = (int)(row_id % g.nt);
+    const int j = (int)(row_id % g.nt);           // row_id = (b*heads + head)*nt + j
     const int bh = (int)(row_id / g.nt);
     const int head = bh % g.heads, b = bh / g.heads;
     const int32_t* o = off + (long long)bh * (g.nt + 1);
@@ -507,25 +506,39 @@ dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, st & 1, abort_flag) &&
                                              mbar_wait(&bars->y_full, st & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
-            float s[64], dp[64];
-#pragma unroll
-            for (int c = 0; c < 64; c += 16) {
-                tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
-                tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
-            }
-            tmem_wait_ld();
             const bool have = hf < ntl;                   // odd tail: the second query cube is absent
             const float* Ls = sL + 64 * hf;
             const float* Ds = sD + 64 * hf;
-            uint32_t pk[32], dk32[32];
+            // P^T first: every S^T value of the warp is read before any P^T
+            // word overwrites it; P^T (bf16) stays in registers for dS^T
+            uint32_t pk[32];
+            {
+                float s[64];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float p0 = have ? ex2(fmaf(s[2 * e], scale_log2, -Ls[2 * e])) : 0.f;
-                const float p1 = have ? ex2(fmaf(s[2 * e + 1], scale_log2, -Ls[2 * e + 1])) : 0.f;
-                pk[e] = pack_bf16x2(p0, p1);
-                dk32[e] = pack_bf16x2(p0 * (dp[2 * e] - Ds[2 * e]), p1 * (dp[2 * e + 1] - Ds[2 * e + 1]));
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = have ? ex2(fmaf(s[2 * e], scale_log2, -Ls[2 * e])) : 0.f;
+                    const float p1 = have ? ex2(fmaf(s[2 * e + 1], scale_log2, -Ls[2 * e + 1])) : 0.f;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
             }
             tmem_st_16x32bx2_x32(tS, pk);
+            uint32_t dk32[32];
+            {
+                float dp[64];
+#pragma unroll
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = __uint_as_float(pk[e] << 16), p1 = __uint_as_float(pk[e] & 0xffff0000u);
+                    dk32[e] = pack_bf16x2(p0 * (dp[2 * e] - Ds[2 * e]), p1 * (dp[2 * e + 1] - Ds[2 * e + 1]));
+                }
+            }
             tmem_st_16x32bx2_x32(tP, dk32);
             tmem_wait_st();
             tc_fence_before();
@@ -555,6 +568,29 @@ dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUte
     if (warp == 5) tmem_dealloc(tbase, C::TMEM_COLS);
 }
 
+// dQ (even CTAs) and dK/dV (odd CTAs) in one launch: the two independent
+// halves of the backward share the SMs, and the long tail of the key cubes
+// that many query cubes kept overlaps dQ work.
+template <int D>
+__global__ void __launch_bounds__(224, 2)
+bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+           const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg, const Grid g,
+           const int32_t* __restrict__ block_idx, const int topk, const float scale_log2, const int ragged,
+           const int32_t* __restrict__ off, const int32_t* __restrict__ entries,
+           const float* __restrict__ lse, const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq,
+           __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int* status) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
+        if (threadIdx.x == 0) report(status, kStatusMisaligned);
+        return;
+    }
+    const long long row = blockIdx.x >> 1;
+    if (blockIdx.x & 1)
+        dkdv_body<D>(mq, mk, mv, mg, g, topk, scale_log2, off, entries, lse, delta, dk, dv, status, smem, row);
+    else
+        dq_body<D>(mq, mk, mv, mg, g, block_idx, topk, scale_log2, ragged, lse, delta, dq, status, smem, row);
+}
+
 // ------------------------------------------------------------------ host side
 
 size_t bwd_scratch_bytes(const Grid& g, int topk) {
@@ -573,14 +609,13 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     static int configured_device = -1;
     constexpr int DQ_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 256;
     constexpr int DKDV_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 1024 + 256;
+    constexpr int SMEM = DQ_SMEM > DKDV_SMEM ? DQ_SMEM : DKDV_SMEM;
     static_assert(sizeof(BwdBars) <= 256, "barrier block");
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DKDV_SMEM);
+        e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
@@ -597,20 +632,17 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     delta_kernel<<<(unsigned)((rows * 64 + 7) / 8), 256, 0, stream>>>(
         a.out32, static_cast<const __nv_bfloat16*>(a.dout), g, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const long long keys = (long long)g.B * g.heads * g.nt;
-    csr_kernel<<<(unsigned)((keys + 255) / 256), 256, 0, stream>>>(a.block_idx, g, a.topk, 0, off, ents);
+    const long long keys = (long long)g.B * g.heads * g.nt;     // one warp each
+    csr_kernel<<<(unsigned)((keys + 7) / 8), 256, 0, stream>>>(a.block_idx, g, a.topk, 0, off, ents);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     csr_scan_kernel<<<(unsigned)(g.B * g.heads), 1024, 0, stream>>>(g, off);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    csr_kernel<<<(unsigned)((keys + 255) / 256), 256, 0, stream>>>(a.block_idx, g, a.topk, 1, off, ents);
+    csr_kernel<<<(unsigned)((keys + 7) / 8), 256, 0, stream>>>(a.block_idx, g, a.topk, 1, off, ents);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dq_kernel<D><<<(unsigned)rows, 224, DQ_SMEM, stream>>>(
-        *a.mq, *a.mk, *a.mv, *a.mg, g, a.block_idx, a.topk, scale_log2, ragged, a.lse, delta,
-        static_cast<__nv_bfloat16*>(a.dq), a.status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dkdv_kernel<D><<<(unsigned)rows, 224, DKDV_SMEM, stream>>>(
-        *a.mq, *a.mk, *a.mv, *a.mg, g, a.topk, scale_log2, off, ents, a.lse, delta,
-        static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv), a.status);
+    bwd_kernel<D><<<(unsigned)(2 * rows), 224, SMEM, stream>>>(
+        *a.mq, *a.mk, *a.mv, *a.mg, g, a.block_idx, a.topk, scale_log2, ragged, off, ents, a.lse, delta,
+        static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk), static_cast<__nv_bfloat16*>(a.dv),
+        a.status);
     return cudaGetLastError();
 }
 
