@@ -40,36 +40,49 @@ using namespace sm100;
 // with the forward's fp32 output (its bf16 rounding, 2^-9 relative, would
 // otherwise enter dQ as -dD sum_m P_m k_m / sqrt(d), which does not shrink
 // with dQ when the kept keys share a large common component).  Each lane
-// reads 4 features at a time (16 bytes of O, 8 bytes of dO).
+// reads 4 features at a time (16 bytes of O, 8 bytes of dO), 8 slots per warp.
 __global__ void __launch_bounds__(256)
 delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout, const Grid g,
              float* __restrict__ delta) {
-    const long long slot = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    // one warp per 8 consecutive slots of one cube (8 token rows in flight)
+    const long long grp = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const long long rows = (long long)g.B * g.heads * g.nt;
-    if (slot >= rows * 64) return;
-    const long long row = slot / 64;
-    const int s = (int)(slot % 64);
+    if (grp >= rows * 8) return;
+    const long long row = grp / 8;
+    const int s0 = (int)(grp % 8) * 8;
     const int i = (int)(row % g.nt), bh = (int)(row / g.nt);
     const int head = bh % g.heads, b = bh / g.heads;
     const TileCoord c = tile_coord(g, i);
-    const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
-    float acc = 0.f;
-    if (dt < c.vt && dh < c.vh && dw < c.vw) {
-        const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
-        const long long base = (((long long)b * g.N + n) * g.heads + head) * g.d;
-        for (int e = lane * 4; e < g.d; e += 128) {
-            const float4 x = *reinterpret_cast<const float4*>(o + base + e);
-            const uint2 yr = *reinterpret_cast<const uint2*>(dout + base + e);
-            acc = fmaf(x.x, __uint_as_float(yr.x << 16), acc);
-            acc = fmaf(x.y, __uint_as_float(yr.x & 0xffff0000u), acc);
-            acc = fmaf(x.z, __uint_as_float(yr.y << 16), acc);
-            acc = fmaf(x.w, __uint_as_float(yr.y & 0xffff0000u), acc);
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
+        acc[u] = 0.f;
+        if (dt < c.vt && dh < c.vh && dw < c.vw) {
+            const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
+            const long long base = (((long long)b * g.N + n) * g.heads + head) * g.d;
+            for (int e = lane * 4; e < g.d; e += 128) {
+                const float4 x = *reinterpret_cast<const float4*>(o + base + e);
+                const uint2 yr = *reinterpret_cast<const uint2*>(dout + base + e);
+                acc[u] = fmaf(x.x, __uint_as_float(yr.x << 16), acc[u]);
+                acc[u] = fmaf(x.y, __uint_as_float(yr.x & 0xffff0000u), acc[u]);
+                acc[u] = fmaf(x.z, __uint_as_float(yr.y << 16), acc[u]);
+                acc[u] = fmaf(x.w, __uint_as_float(yr.y & 0xffff0000u), acc[u]);
+            }
         }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) delta[slot] = acc;
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+    if (lane < 8) {
+        float v = acc[0];
+#pragma unroll
+        for (int u = 1; u < 8; ++u) v = lane == u ? acc[u] : v;
+        delta[row * 64 + s0 + lane] = v;
+    }
 }
 
 // ---------------------------------------------------------------- transpose
@@ -629,7 +642,7 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (g.T % g.tt) || (g.H % g.th) || (g.W % g.tw);
 
-    delta_kernel<<<(unsigned)((rows * 64 + 7) / 8), 256, 0, stream>>>(
+    delta_kernel<<<(unsigned)rows, 256, 0, stream>>>(                 // 8 warps x 8 slots per cube
         a.out32, static_cast<const __nv_bfloat16*>(a.dout), g, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long keys = (long long)g.B * g.heads * g.nt;     // one warp each
