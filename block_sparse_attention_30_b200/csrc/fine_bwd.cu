@@ -13,14 +13,17 @@
 //   csr_*          the transpose of the block index: for every key cube the
 //                  ascending list of query cubes that kept it (deterministic;
 //                  one warp per key cube).
-//   dq_body        one CTA per query cube: per kept key-cube pair, S = Q K^T
+//   dq_body        one CTA per query cube: per kept key cube, S = Q K^T
 //                  (TMEM lanes 0-15) and dP = dO V^T (lanes 16-31 of the same
 //                  columns) on the tensor cores, dS written as bf16 over S by
 //                  the softmax warps, then dQ += dS K (A = dS from TMEM).
-//   dkdv_body      one CTA per key cube: per pair of query cubes that kept it,
+//   dkdv_body      one CTA per key cube: per query cube that kept it,
 //                  S^T = K Q^T and dP^T = V dO^T, P^T and dS^T written as bf16
 //                  over them, then dV += P^T dO (lanes 0-15) and
 //                  dK += dS^T Q (lanes 16-31) accumulate in TMEM.
+// Both walk single cubes: two ring slots for the streamed cubes and two S
+// buffers (the two 64-column halves of the S region) let the loads and the
+// softmax of one step overlap the tensor-core work of the next.
 // Both run in one launch (bwd_kernel: even CTAs dQ, odd CTAs dK/dV).  One
 // K/Q tile serves as the K-major operand of one product and the MN-major
 // operand of the other, as V does in the forward.  Every wait is bounded.
@@ -164,38 +167,28 @@ csr_scan_kernel(const Grid g, int32_t* __restrict__ off) {
 }
 
 // ---------------------------------------------------------- shared layout
+// Both bodies walk single cubes (64 keys or 64 queries per step) so that the
+// streamed cubes get two ring slots and S two TMEM buffers within the
+// budget of two CTAs per SM; step t uses ring slot t % 2 and S buffer t % 2.
 template <int D>
 struct BwdCfg {
     static constexpr int NCH = D / 64;
-    static constexpr int CUBE_BYTES = 64 * D * 2;        // one cube of one tensor (bf16)
-    static constexpr int PAIR_BYTES = 2 * CUBE_BYTES;
-    static constexpr int CHUNK_STRIDE = 128 * 128;       // bytes between d chunks of a pair
+    static constexpr int CUBE_BYTES = 64 * D * 2;        // one cube of one tensor (bf16), chunks 8 KB apart
     static constexpr int TMEM_COLS = 256;
     static constexpr int ACC_COL = 0;                    // dQ | dV (lanes 0-15), dK (lanes 16-31)
-    static constexpr int S_COL = 128;                    // S / P (lanes 0-15), dP / dS (lanes 16-31)
+    static constexpr int S_COL = 128;                    // S buffer b at S_COL + 64 b: S / P (lanes 0-15),
+                                                         // dP / dS (lanes 16-31)
+    static constexpr int SMEM = 6 * CUBE_BYTES + 1024 + 256;  // own 2 cubes + 2 x 2 slots, lse/D, barriers
 };
 
 struct BwdBars {
-    uint64_t a_full;                 // the CTA's own cube(s): Q + dO, or K + V
-    uint64_t x_full, x_empty;        // pair ring 1 (K pairs / Q pairs)
-    uint64_t y_full, y_empty;        // pair ring 2 (V pairs / dO pairs)
-    uint64_t s_full, ds_full, mma_done;
+    uint64_t a_full;                 // the CTA's own cubes: Q + dO, or K + V
+    uint64_t x_full[2], x_empty[2];  // ring 1 (K cubes / Q cubes + lse)
+    uint64_t y_full[2], y_empty[2];  // ring 2 (V cubes / dO cubes + D)
+    uint64_t s_full[2], ds_full[2], mma_done;
     uint32_t tmem_base;
     int abort;
 };
-
-// Loads one key/query cube pair (cubes jt[0..ntl)) of the tensor behind `map`
-// into a pair buffer: chunk c of cube t at c * CHUNK_STRIDE + t * 8192.
-template <int D>
-__device__ __forceinline__ void load_pair(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const Grid& g,
-                                          const int* jt, int ntl, int head, int b) {
-    using C = BwdCfg<D>;
-    for (int t = 0; t < ntl; ++t) {
-        const TileCoord kc = tile_coord(g, jt[t]);
-        for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_5d(dst + ch * C::CHUNK_STRIDE + t * 8192, map, bar, head * D + 64 * ch, kc.w0, kc.h0, kc.t0, b);
-    }
-}
 
 template <int D>
 __device__ __forceinline__ void load_cube(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const Grid& g,
@@ -235,10 +228,34 @@ __device__ __forceinline__ void store_zero_half_row(int half, __nv_bfloat16* dst
     for (int c = 0; c < half; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);
 }
 
+// One 64 x 64 product pair into S buffer `sb`: S (lanes 0-15) = A1 B1^T and
+// dP (lanes 16-31) = A2 B2^T, all operands cubes in smem (K-major), K = D.
+template <int D>
+__device__ __forceinline__ void issue_s_dp(uint32_t sb, uint32_t a1, uint32_t b1, uint32_t a2, uint32_t b2) {
+    const uint32_t id = idesc_bf16_f32(64, 64, false, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t o = (kk >> 2) * 8192 + (kk & 3) * 32;
+        mma_bf16_ss(sb, smem_desc_sw128(a1 + o, 16, 1024), smem_desc_sw128(b1 + o, 16, 1024), id, kk > 0);
+        mma_bf16_ss(sb + (16u << 16), smem_desc_sw128(a2 + o, 16, 1024), smem_desc_sw128(b2 + o, 16, 1024), id,
+                    kk > 0);
+    }
+}
+
+// acc += T (TMEM, 64 x 64 bf16 at `t`) x cube (smem, 64 rows x D, as the
+// MN-major B operand), 4 MMAs of K = 16.
+template <int D>
+__device__ __forceinline__ void issue_acc(uint32_t acc, uint32_t t, uint32_t cube, bool accumulate) {
+    const uint32_t id = idesc_bf16_f32(64, D, false, true);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ts(acc, t + kk * 8, smem_desc_sw128(cube + kk * 2048, 8192, 1024), id, accumulate || kk > 0);
+}
+
 // -------------------------------------------------------------------- dQ
-// 224 threads: warps 0-3 softmax (rows 16w..16w+15, each row split in two
-// 64-key halves over lanes t and t+16), warp 4 Q + dO + K pairs, warp 5 MMA,
-// warp 6 V pairs.
+// 224 threads: warps 0-3 softmax (rows 16w..16w+15 of the query cube, each
+// row split over lanes t and t+16: keys 0-31 and 32-63 of the step's cube),
+// warp 4 Q + dO + K cubes, warp 5 MMA, warp 6 V cubes.
 template <int D>
 __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                         const CUtensorMap& mg, const Grid& g,
@@ -250,23 +267,25 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
     using C = BwdCfg<D>;
     uint8_t* sQ = smem;
     uint8_t* sG = sQ + C::CUBE_BYTES;
-    uint8_t* sK = sG + C::CUBE_BYTES;
-    uint8_t* sV = sK + C::PAIR_BYTES;
-    BwdBars* bars = reinterpret_cast<BwdBars*>(sV + C::PAIR_BYTES);
+    uint8_t* sK = sG + C::CUBE_BYTES;                 // 2 slots
+    uint8_t* sV = sK + 2 * C::CUBE_BYTES;             // 2 slots
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + 6 * C::CUBE_BYTES + 1024);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i = (int)(row_id % g.nt);
     const int bh = (int)(row_id / g.nt);
     const int head = bh % g.heads, b = bh / g.heads;
     const int32_t* my_idx = block_idx + row_id * topk;
-    const int n_pairs = (topk + 1) >> 1;
 
     if (tid == 0) {
         bars->abort = 0;
         mbar_init(&bars->a_full, 1);
-        mbar_init(&bars->x_full, 1); mbar_init(&bars->x_empty, 1);
-        mbar_init(&bars->y_full, 1); mbar_init(&bars->y_empty, 1);
-        mbar_init(&bars->s_full, 1); mbar_init(&bars->ds_full, 128); mbar_init(&bars->mma_done, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->x_full[x], 1); mbar_init(&bars->x_empty[x], 1);
+            mbar_init(&bars->y_full[x], 1); mbar_init(&bars->y_empty[x], 1);
+            mbar_init(&bars->s_full[x], 1); mbar_init(&bars->ds_full[x], 128);
+        }
+        mbar_init(&bars->mma_done, 1);
         fence_barrier_init();
     }
     if (warp == 5) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
@@ -279,8 +298,8 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
     if (warp == 4 || warp == 6) {
         if (lane == 0) {
             const bool is_k = warp == 4;
-            uint64_t* full = is_k ? &bars->x_full : &bars->y_full;
-            uint64_t* empty = is_k ? &bars->x_empty : &bars->y_empty;
+            uint64_t* full = is_k ? bars->x_full : bars->y_full;
+            uint64_t* empty = is_k ? bars->x_empty : bars->y_empty;
             uint8_t* ring = is_k ? sK : sV;
             const CUtensorMap* map = is_k ? &mk : &mv;
             if (is_k) {
@@ -289,49 +308,45 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
                 load_cube<D>(sG, &mg, &bars->a_full, g, i, head, b);
             }
             int issued = 0;
-            for (int p = 0; p < n_pairs; ++p) {
-                const int ntl = min(2, topk - 2 * p);
-                int jt[2] = {__ldg(my_idx + 2 * p), ntl > 1 ? __ldg(my_idx + 2 * p + 1) : 0};
-                for (int t = 0; t < ntl; ++t)
-                    if (jt[t] < 0 || jt[t] >= g.nt) { if (is_k) report(status, kStatusBadIndex); jt[t] = 0; }
-                if (p >= 1 && !mbar_wait(empty, (p - 1) & 1, abort_flag)) { fail(); break; }
-                mbar_arrive_expect_tx(full, ntl * C::CUBE_BYTES);
-                load_pair<D>(ring, map, full, g, jt, ntl, head, b);
+            for (int t = 0; t < topk; ++t) {
+                int j = __ldg(my_idx + t);
+                if (j < 0 || j >= g.nt) { if (is_k) report(status, kStatusBadIndex); j = 0; }
+                const int x = t & 1;
+                if (t >= 2 && !mbar_wait(&empty[x], ((t >> 1) - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&full[x], C::CUBE_BYTES);
+                load_cube<D>(ring + x * C::CUBE_BYTES, map, &full[x], g, j, head, b);
                 ++issued;
             }
             if (*abort_flag) {
                 if (is_k) wait_noabort(&bars->a_full, 0);
-                if (issued > 0) wait_noabort(full, (issued - 1) & 1);
+                for (int n = issued > 2 ? issued - 2 : 0; n < issued; ++n) wait_noabort(&full[n & 1], (n >> 1) & 1);
             }
         }
     } else if (warp == 5) {
         if (lane == 0) {
             const uint32_t q_addr = smem_u32(sQ), g_addr = smem_u32(sG);
-            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            const uint32_t tS = tbase + C::S_COL, tP = tbase + C::S_COL + (16u << 16), tAcc = tbase + C::ACC_COL;
-            const uint32_t id_acc = idesc_bf16_f32(64, D, false, true);
-            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
-            for (int p = 0; ok && p < n_pairs; ++p) {
-                const int nkeys = min(2, topk - 2 * p) * 64;
-                if (!mbar_wait(&bars->x_full, p & 1, abort_flag) || !mbar_wait(&bars->y_full, p & 1, abort_flag)) { ok = false; break; }
+            const uint32_t tAcc = tbase + C::ACC_COL;
+            auto sbuf = [&](int x) { return tbase + C::S_COL + 64 * x; };
+            auto issue_s = [&](int t) -> bool {
+                const int x = t & 1;
+                if (!mbar_wait(&bars->x_full[x], (t >> 1) & 1, abort_flag) ||
+                    !mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {        // S = Q K^T and dP = dO V^T (K-major)
-                    const uint32_t ao = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32;
-                    mma_bf16_ss(tS, smem_desc_sw128(q_addr + ao, 16, 1024), smem_desc_sw128(k_addr + bo, 16, 1024), id_s, kk > 0);
-                    mma_bf16_ss(tP, smem_desc_sw128(g_addr + ao, 16, 1024), smem_desc_sw128(v_addr + bo, 16, 1024), id_s, kk > 0);
-                }
-                mma_commit(&bars->s_full);
-                mma_commit(&bars->y_empty);                  // V read by dP only
-                if (!mbar_wait(&bars->ds_full, p & 1, abort_flag)) { ok = false; break; }
+                issue_s_dp<D>(sbuf(x), q_addr, smem_u32(sK + x * C::CUBE_BYTES), g_addr,
+                              smem_u32(sV + x * C::CUBE_BYTES));
+                mma_commit(&bars->s_full[x]);
+                mma_commit(&bars->y_empty[x]);             // V cube read by dP only
+                return true;
+            };
+            // S of step t+2 is issued right after dQ of step t (the last reader of its buffer)
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag) && issue_s(0) && (topk < 2 || issue_s(1));
+            for (int t = 0; ok && t < topk; ++t) {
+                const int x = t & 1;
+                if (!mbar_wait(&bars->ds_full[x], (t >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int kk = 0; kk < nkeys / 16; ++kk) {    // dQ += dS K (K as MN-major B)
-                    const uint64_t bd = smem_desc_sw128(k_addr + kk * 2048, C::CHUNK_STRIDE, 1024);
-                    mma_bf16_ts(tAcc, tS + kk * 8, bd, id_acc, (p > 0 || kk > 0));
-                }
-                mma_commit(&bars->x_empty);
+                issue_acc<D>(tAcc, sbuf(x), smem_u32(sK + x * C::CUBE_BYTES), t > 0);   // dQ += dS K
+                mma_commit(&bars->x_empty[x]);
+                if (t + 2 < topk && !issue_s(t + 2)) { ok = false; break; }
             }
             if (!ok) fail();
             mma_commit(&bars->mma_done);
@@ -341,39 +356,38 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
         // softmax warps: P = exp2(s * scale_log2 - lse), dS = P (dP - D)
         const int r = 16 * warp + (lane & 15), hf = lane >> 4;
         const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
-        const uint32_t tS = lane_base + C::S_COL, tP = lane_base + C::S_COL + (16u << 16);
         const float l2 = __ldg(lse + row_id * 64 + r);
         const float dl = __ldg(delta + row_id * 64 + r);
         bool ok = true;
-        for (int p = 0; p < n_pairs; ++p) {
-            const int ntl = min(2, topk - 2 * p);
-            uint64_t vmask = hf < ntl ? ~0ull : 0ull;
-            if (ragged && hf < ntl) {
-                int j = __ldg(my_idx + 2 * p + hf);
+        for (int t = 0; t < topk; ++t) {
+            const int x = t & 1;
+            uint32_t vmask = 0xffffffffu;                 // keys 32 hf .. 32 hf + 31 of the cube
+            if (ragged) {
+                int j = __ldg(my_idx + t);
                 if (j < 0 || j >= g.nt) j = 0;
-                vmask = valid_slot_mask(g, tile_coord(g, j));
+                vmask = (uint32_t)(valid_slot_mask(g, tile_coord(g, j)) >> (32 * hf));
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, p & 1, abort_flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x], (t >> 1) & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
-            float s[64], dp[64];
-#pragma unroll
-            for (int c = 0; c < 64; c += 16) {
-                tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
-                tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
-            }
+            const uint32_t tS = lane_base + C::S_COL + 64 * x, tP = tS + (16u << 16);
+            float s[32], dp[32];
+            tmem_ld_16x32bx2_x16<32>(tS, *reinterpret_cast<float(*)[16]>(&s[0]));
+            tmem_ld_16x32bx2_x16<32>(tS + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+            tmem_ld_16x32bx2_x16<32>(tP, *reinterpret_cast<float(*)[16]>(&dp[0]));
+            tmem_ld_16x32bx2_x16<32>(tP + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
             tmem_wait_ld();
-            uint32_t pk[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const bool v0 = (vmask >> (2 * e)) & 1ull, v1 = (vmask >> (2 * e + 1)) & 1ull;
+            for (int e = 0; e < 16; ++e) {
+                const bool v0 = (vmask >> (2 * e)) & 1u, v1 = (vmask >> (2 * e + 1)) & 1u;
                 const float p0 = v0 ? ex2(fmaf(s[2 * e], scale_log2, -l2)) : 0.f;
                 const float p1 = v1 ? ex2(fmaf(s[2 * e + 1], scale_log2, -l2)) : 0.f;
                 pk[e] = pack_bf16x2(p0 * (dp[2 * e] - dl), p1 * (dp[2 * e + 1] - dl));
             }
-            tmem_st_16x32bx2_x32(tS, pk);
+            tmem_st_16x32bx2_x16u<16>(tS, pk);            // dS over S: keys 32 hf.. -> columns 16 hf..
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->ds_full);
+            mbar_arrive(&bars->ds_full[x]);
         }
         if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag))) ok = false;
         if (!ok) fail();
@@ -396,8 +410,8 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
 
 // ------------------------------------------------------------------ dK, dV
 // One CTA per key cube: warps 0-3 softmax (key rows 16w..16w+15; lanes t and
-// t+16 hold query cube 0 and 1 of the pair), warp 4 K + V cubes and the Q
-// pairs (+ their lse), warp 5 MMA, warp 6 the dO pairs (+ their D).
+// t+16 hold queries 0-31 and 32-63 of the step's query cube), warp 4 K + V
+// cubes and the Q cubes (+ their lse), warp 5 MMA, warp 6 the dO cubes (+ D).
 template <int D>
 __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                           const CUtensorMap& mg, const Grid& g, const int topk,
@@ -409,11 +423,11 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
     using C = BwdCfg<D>;
     uint8_t* sK = smem;
     uint8_t* sV = sK + C::CUBE_BYTES;
-    uint8_t* sQ = sV + C::CUBE_BYTES;         // pair of query cubes
-    uint8_t* sG = sQ + C::PAIR_BYTES;         // pair of dO cubes
-    float* sL = reinterpret_cast<float*>(sG + C::PAIR_BYTES);   // lse of the pair's 128 query slots
-    float* sD = sL + 128;                                         // D of the pair's 128 query slots
-    BwdBars* bars = reinterpret_cast<BwdBars*>(sD + 128);
+    uint8_t* sQ = sV + C::CUBE_BYTES;                 // 2 slots
+    uint8_t* sG = sQ + 2 * C::CUBE_BYTES;             // 2 slots
+    float* sL = reinterpret_cast<float*>(smem + 6 * C::CUBE_BYTES);   // lse of the slots' query cubes [2][64]
+    float* sD = sL + 128;                                              // D of the slots' query cubes [2][64]
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + 6 * C::CUBE_BYTES + 1024);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = (int)(row_id % g.nt);           // row_id = (b*heads + head)*nt + j
@@ -422,15 +436,17 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
     const int32_t* o = off + (long long)bh * (g.nt + 1);
     const int e0 = __ldg(o + j), nq = __ldg(o + j + 1) - e0;
     const int32_t* my_q = entries + (long long)bh * g.nt * topk + e0;    // ascending query cubes
-    const int n_steps = (nq + 1) >> 1;
     const long long qrow0 = (long long)bh * g.nt;                          // row id of query cube 0
 
     if (tid == 0) {
         bars->abort = 0;
         mbar_init(&bars->a_full, 1);
-        mbar_init(&bars->x_full, 1); mbar_init(&bars->x_empty, 1);
-        mbar_init(&bars->y_full, 1); mbar_init(&bars->y_empty, 1);
-        mbar_init(&bars->s_full, 1); mbar_init(&bars->ds_full, 128); mbar_init(&bars->mma_done, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->x_full[x], 1); mbar_init(&bars->x_empty[x], 1);
+            mbar_init(&bars->y_full[x], 1); mbar_init(&bars->y_empty[x], 1);
+            mbar_init(&bars->s_full[x], 1); mbar_init(&bars->ds_full[x], 128);
+        }
+        mbar_init(&bars->mma_done, 1);
         fence_barrier_init();
     }
     if (warp == 5) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
@@ -443,8 +459,8 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
     if (warp == 4 || warp == 6) {
         if (lane == 0) {
             const bool is_q = warp == 4;
-            uint64_t* full = is_q ? &bars->x_full : &bars->y_full;
-            uint64_t* empty = is_q ? &bars->x_empty : &bars->y_empty;
+            uint64_t* full = is_q ? bars->x_full : bars->y_full;
+            uint64_t* empty = is_q ? bars->x_empty : bars->y_empty;
             uint8_t* ring = is_q ? sQ : sG;
             float* side = is_q ? sL : sD;
             const float* side_src = is_q ? lse : delta;
@@ -455,52 +471,47 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
                 load_cube<D>(sV, &mv, &bars->a_full, g, j, head, b);
             }
             int issued = 0;
-            for (int st = 0; st < n_steps; ++st) {
-                const int ntl = min(2, nq - 2 * st);
-                int it[2] = {__ldg(my_q + 2 * st), ntl > 1 ? __ldg(my_q + 2 * st + 1) : 0};
-                for (int t = 0; t < ntl; ++t)
-                    if (it[t] < 0 || it[t] >= g.nt) { report(status, kStatusBadIndex); it[t] = 0; }
-                if (st >= 1 && !mbar_wait(empty, (st - 1) & 1, abort_flag)) { fail(); break; }
-                mbar_arrive_expect_tx(full, ntl * (C::CUBE_BYTES + 256));
-                load_pair<D>(ring, map, full, g, it, ntl, head, b);
-                for (int t = 0; t < ntl; ++t)
-                    bulk_load(side + 64 * t, side_src + (qrow0 + it[t]) * 64, 256, full);
+            for (int t = 0; t < nq; ++t) {
+                int it = __ldg(my_q + t);
+                if (it < 0 || it >= g.nt) { report(status, kStatusBadIndex); it = 0; }
+                const int x = t & 1;
+                if (t >= 2 && !mbar_wait(&empty[x], ((t >> 1) - 1) & 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&full[x], C::CUBE_BYTES + 256);
+                load_cube<D>(ring + x * C::CUBE_BYTES, map, &full[x], g, it, head, b);
+                bulk_load(side + 64 * x, side_src + (qrow0 + it) * 64, 256, &full[x]);
                 ++issued;
             }
             if (*abort_flag) {
                 if (is_q) wait_noabort(&bars->a_full, 0);
-                if (issued > 0) wait_noabort(full, (issued - 1) & 1);
+                for (int n = issued > 2 ? issued - 2 : 0; n < issued; ++n) wait_noabort(&full[n & 1], (n >> 1) & 1);
             }
         }
     } else if (warp == 5) {
         if (lane == 0) {
             const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            const uint32_t q_addr = smem_u32(sQ), g_addr = smem_u32(sG);
-            const uint32_t tS = tbase + C::S_COL, tP = tbase + C::S_COL + (16u << 16);
             const uint32_t tdV = tbase + C::ACC_COL, tdK = tbase + C::ACC_COL + (16u << 16);
-            const uint32_t id_acc = idesc_bf16_f32(64, D, false, true);
-            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
-            for (int st = 0; ok && st < n_steps; ++st) {
-                const int nqs = min(2, nq - 2 * st) * 64;
-                if (!mbar_wait(&bars->x_full, st & 1, abort_flag) || !mbar_wait(&bars->y_full, st & 1, abort_flag)) { ok = false; break; }
+            auto sbuf = [&](int x) { return tbase + C::S_COL + 64 * x; };
+            auto issue_s = [&](int t) -> bool {
+                const int x = t & 1;
+                if (!mbar_wait(&bars->x_full[x], (t >> 1) & 1, abort_flag) ||
+                    !mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t id_s = idesc_bf16_f32(64, nqs, false, false);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {        // S^T = K Q^T, dP^T = V dO^T
-                    const uint32_t ao = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32;
-                    mma_bf16_ss(tS, smem_desc_sw128(k_addr + ao, 16, 1024), smem_desc_sw128(q_addr + bo, 16, 1024), id_s, kk > 0);
-                    mma_bf16_ss(tP, smem_desc_sw128(v_addr + ao, 16, 1024), smem_desc_sw128(g_addr + bo, 16, 1024), id_s, kk > 0);
-                }
-                mma_commit(&bars->s_full);
-                if (!mbar_wait(&bars->ds_full, st & 1, abort_flag)) { ok = false; break; }
+                // S^T = K Q^T (lanes 0-15), dP^T = V dO^T (lanes 16-31)
+                issue_s_dp<D>(sbuf(x), k_addr, smem_u32(sQ + x * C::CUBE_BYTES), v_addr,
+                              smem_u32(sG + x * C::CUBE_BYTES));
+                mma_commit(&bars->s_full[x]);
+                return true;
+            };
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag) && (nq < 1 || issue_s(0)) && (nq < 2 || issue_s(1));
+            for (int t = 0; ok && t < nq; ++t) {
+                const int x = t & 1;
+                if (!mbar_wait(&bars->ds_full[x], (t >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int kk = 0; kk < nqs / 16; ++kk) {      // dV += P^T dO, dK += dS^T Q
-                    mma_bf16_ts(tdV, tS + kk * 8, smem_desc_sw128(g_addr + kk * 2048, C::CHUNK_STRIDE, 1024), id_acc, (st > 0 || kk > 0));
-                    mma_bf16_ts(tdK, tP + kk * 8, smem_desc_sw128(q_addr + kk * 2048, C::CHUNK_STRIDE, 1024), id_acc, (st > 0 || kk > 0));
-                }
-                mma_commit(&bars->x_empty);
-                mma_commit(&bars->y_empty);
+                issue_acc<D>(tdV, sbuf(x), smem_u32(sG + x * C::CUBE_BYTES), t > 0);                   // dV += P^T dO
+                issue_acc<D>(tdK, sbuf(x) + (16u << 16), smem_u32(sQ + x * C::CUBE_BYTES), t > 0);     // dK += dS^T Q
+                mma_commit(&bars->x_empty[x]);
+                mma_commit(&bars->y_empty[x]);
+                if (t + 2 < nq && !issue_s(t + 2)) { ok = false; break; }
             }
             if (!ok) fail();
             mma_commit(&bars->mma_done);
@@ -508,54 +519,38 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
         }
     } else {
         // softmax warps: P^T = exp2(s * scale_log2 - lse[q]), dS^T = P^T (dP^T - D[q])
-        const int r = 16 * warp + (lane & 15), hf = lane >> 4;   // key row, query cube of the pair
+        const int r = 16 * warp + (lane & 15), hf = lane >> 4;   // key row, query half of the cube
         const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
-        const uint32_t tS = lane_base + C::S_COL, tP = lane_base + C::S_COL + (16u << 16);
         bool ok = true;
-        for (int st = 0; st < n_steps; ++st) {
-            const int ntl = min(2, nq - 2 * st);
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, st & 1, abort_flag))) { ok = false; break; }
-            // lse and D of this pair landed with the Q / dO pairs
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full, st & 1, abort_flag) &&
-                                             mbar_wait(&bars->y_full, st & 1, abort_flag))) { ok = false; break; }
+        for (int t = 0; t < nq; ++t) {
+            const int x = t & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x], (t >> 1) & 1, abort_flag))) { ok = false; break; }
+            // lse and D of this query cube landed with its Q / dO cubes
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_full[x], (t >> 1) & 1, abort_flag) &&
+                                             mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
-            const bool have = hf < ntl;                   // odd tail: the second query cube is absent
-            const float* Ls = sL + 64 * hf;
-            const float* Ds = sD + 64 * hf;
-            // P^T first: every S^T value of the warp is read before any P^T
-            // word overwrites it; P^T (bf16) stays in registers for dS^T
-            uint32_t pk[32];
-            {
-                float s[64];
+            const uint32_t tS = lane_base + C::S_COL + 64 * x, tP = tS + (16u << 16);
+            const float* Ls = sL + 64 * x + 32 * hf;
+            const float* Ds = sD + 64 * x + 32 * hf;
+            float s[32], dp[32];
+            tmem_ld_16x32bx2_x16<32>(tS, *reinterpret_cast<float(*)[16]>(&s[0]));
+            tmem_ld_16x32bx2_x16<32>(tS + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+            tmem_ld_16x32bx2_x16<32>(tP, *reinterpret_cast<float(*)[16]>(&dp[0]));
+            tmem_ld_16x32bx2_x16<32>(tP + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+            tmem_wait_ld();
+            uint32_t pk[16], dk16[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 16)
-                    tmem_ld_16x32bx2_x16<64>(tS + c, *reinterpret_cast<float(*)[16]>(&s[c]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = have ? ex2(fmaf(s[2 * e], scale_log2, -Ls[2 * e])) : 0.f;
-                    const float p1 = have ? ex2(fmaf(s[2 * e + 1], scale_log2, -Ls[2 * e + 1])) : 0.f;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
+            for (int e = 0; e < 16; ++e) {
+                const float p0 = ex2(fmaf(s[2 * e], scale_log2, -Ls[2 * e]));
+                const float p1 = ex2(fmaf(s[2 * e + 1], scale_log2, -Ls[2 * e + 1]));
+                pk[e] = pack_bf16x2(p0, p1);
+                dk16[e] = pack_bf16x2(p0 * (dp[2 * e] - Ds[2 * e]), p1 * (dp[2 * e + 1] - Ds[2 * e + 1]));
             }
-            tmem_st_16x32bx2_x32(tS, pk);
-            uint32_t dk32[32];
-            {
-                float dp[64];
-#pragma unroll
-                for (int c = 0; c < 64; c += 16)
-                    tmem_ld_16x32bx2_x16<64>(tP + c, *reinterpret_cast<float(*)[16]>(&dp[c]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = __uint_as_float(pk[e] << 16), p1 = __uint_as_float(pk[e] & 0xffff0000u);
-                    dk32[e] = pack_bf16x2(p0 * (dp[2 * e] - Ds[2 * e]), p1 * (dp[2 * e + 1] - Ds[2 * e + 1]));
-                }
-            }
-            tmem_st_16x32bx2_x32(tP, dk32);
+            tmem_st_16x32bx2_x16u<16>(tS, pk);            // queries 32 hf.. -> columns 16 hf..
+            tmem_st_16x32bx2_x16u<16>(tP, dk16);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->ds_full);
+            mbar_arrive(&bars->ds_full[x]);
         }
         if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort_flag))) ok = false;
         if (!ok) fail();
@@ -566,7 +561,7 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
             const bool valid = dt < kc.vt && dh < kc.vh && dw < kc.vw;
             const long long n = ((long long)(kc.t0 + dt) * g.H + (kc.h0 + dh)) * g.W + (kc.w0 + dw);
             const long long base = (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
-            if (n_steps > 0) {
+            if (nq > 0) {
                 store_half_row<D>(lane_base + C::ACC_COL, 1.f, dv + base, valid);
                 store_half_row<D>(lane_base + C::ACC_COL + (16u << 16), scale_log2 * 0.6931471805599453f, dk + base, valid);
             } else {                                      // no query cube kept this key cube
@@ -620,9 +615,7 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     using C = BwdCfg<D>;
     const Grid& g = a.g;
     static int configured_device = -1;
-    constexpr int DQ_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 256;
-    constexpr int DKDV_SMEM = 2 * C::CUBE_BYTES + 2 * C::PAIR_BYTES + 1024 + 256;
-    constexpr int SMEM = DQ_SMEM > DKDV_SMEM ? DQ_SMEM : DKDV_SMEM;
+    constexpr int SMEM = C::SMEM;
     static_assert(sizeof(BwdBars) <= 256, "barrier block");
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

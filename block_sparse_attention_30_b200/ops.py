@@ -161,3 +161,58 @@ class BlockSparseVideoAttention:
 
     def status(self, stream=None) -> int:
         return vsa_device_status(self.workspace, stream)
+
+
+class HostPipeline:
+    """Forward passes over a stream of host batches (pinned q, k, v in, output
+    back to pinned host memory), with the copies overlapping the kernels.
+
+    Two device buffer sets and three CUDA streams: while the kernels of step i
+    run, the inputs of step i+1 travel host -> device and the output of step
+    i-1 device -> host (the two copy directions use separate DMA engines).
+    Events order each buffer set's reuse: inputs are overwritten only after
+    the kernels that read them, outputs only after their copy back.
+    """
+
+    def __init__(self, attn, shape, dtype=torch.bfloat16, device="cuda"):
+        self.attn = attn
+        dev = torch.device(device)
+        self.bufs = [tuple(torch.empty(shape, dtype=dtype, device=dev) for _ in range(4))
+                     for _ in range(2)]                       # q, k, v, out per set
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_comp = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+
+    def run(self, items):
+        """items: iterable of (q_h, k_h, v_h, out_h) pinned host tensors of the
+        pipeline's shape.  Enqueues everything; call synchronize() (or wait on
+        the returned event) before reading the host outputs."""
+        for i, (qh, kh, vh, oh) in enumerate(items):
+            x = i % 2
+            q, k, v, o = self.bufs[x]
+            with torch.cuda.stream(self.s_in):
+                if self.used[x]:
+                    self.s_in.wait_event(self.ev_comp[x])     # kernels of step i-2 read q, k, v
+                q.copy_(qh, non_blocking=True)
+                k.copy_(kh, non_blocking=True)
+                v.copy_(vh, non_blocking=True)
+                self.ev_in[x].record(self.s_in)
+            self.s_comp.wait_event(self.ev_in[x])
+            if self.used[x]:
+                self.s_comp.wait_event(self.ev_out[x])        # output of step i-2 copied back
+            self.attn(q, k, v, out=o, stream=self.s_comp)
+            self.ev_comp[x].record(self.s_comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_comp[x])
+                oh.copy_(o, non_blocking=True)
+                self.ev_out[x].record(self.s_out)
+            self.used[x] = True
+        done = torch.cuda.Event(enable_timing=True)
+        done.record(self.s_out)
+        return done
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_comp, self.s_out):
+            s.synchronize()

@@ -458,3 +458,21 @@ def test_backward_headline_two_heads(ops):
     for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
         assert not torch.isnan(got).any(), name + " must be fully written"
         check_grad(to_f64(got[:, :, hs]), ref, name)
+
+
+def test_host_pipeline_matches_direct_calls(ops):
+    """ops.HostPipeline (copies overlapped with the kernels across steps)
+    returns, for every step, exactly what a direct call on the device gives."""
+    T, H, W, heads, d, topk = 6, 10, 9, 2, 128, 5
+    attn = ops.BlockSparseVideoAttention(1, heads, d, T, H, W, topk)
+    batches = [Small(T, H, W, heads, d, topk, seed=s) for s in (21, 22, 23)]
+    pinned = [tuple(x.pin_memory() for x in (c.q, c.k, c.v)) for c in batches]
+    outs = [torch.empty(c.q.shape, dtype=torch.bfloat16).pin_memory() for c in batches]
+    pipe = ops.HostPipeline(attn, batches[0].q.shape)
+    pipe.run([(*p, o) for p, o in zip(pinned, outs)])
+    pipe.synchronize()
+    assert attn.status() == 0
+    for c, o in zip(batches, outs):
+        ref = attn(c.q.cuda(), c.k.cuda(), c.v.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(o, ref.cpu())
