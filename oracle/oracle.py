@@ -194,6 +194,17 @@ def linear_apply(q, S, z, B, heads, d, N, precision="f64") -> np.ndarray:
     return out
 
 
+def linear_bwd(q, k, v, dout, B, heads, d, N, precision="f64"):
+    """Gradients (dq, dk, dv) of the linear branch phi(q)S / (phi(q).z) for
+    the output gradient dout (bf16), each [B][N][heads][d]."""
+    qb, kb, vb, gb = bits(q), bits(k), bits(v), bits(dout)
+    R = _real(precision)
+    dq, dk, dv = (np.empty((B, N, heads, d), R) for _ in range(3))
+    lib(precision).oracle_linear_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _c_int(B), _c_int(heads),
+                                     _c_int(d), _c_i64(N), _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
 def dense(q, k, v, B, heads, d, N, precision="f64") -> np.ndarray:
     qb, kb, vb = bits(q), bits(k), bits(v)
     out = np.empty((B, N, heads, d), _real(precision))

@@ -542,6 +542,89 @@ void oracle_linear_apply(const uint16_t *q, const REAL *S, const REAL *z, int B,
 /* ------------------------------------------------------------ dense (pin)
  * Plain dense softmax attention over all N tokens of the grid; with k equal
  * to the tile count the block-sparse fine pass must reduce to this. */
+/* ---------------------------------------------------- linear branch, backward
+ * Gradients of the linear branch (SLA: the sparse and the linear branch are
+ * trained together, TurboDiffusion article, section "稀疏、蒸馏与全链路量化").
+ * With phi = elu + 1, per (b, head): S = sum_m phi(k_m)^T v_m, z = sum_m
+ * phi(k_m), and for every token lin_n = num_n / den_n with num_n = phi(q_n) S,
+ * den_n = phi(q_n) . z.  Given dlin_n (the output gradient), by the chain rule:
+ *     dnum_n = dlin_n / den_n,   dden_n = -(dlin_n . lin_n) / den_n
+ *     dphi(q_n) = S dnum_n + dden_n z             dq_n = dphi(q_n) o phi'(q_n)
+ *     dS = sum_n phi(q_n)^T dnum_n,  dz = sum_n dden_n phi(q_n)
+ *     dphi(k_m) = dS v_m + dz,  dv_m = dS^T phi(k_m)
+ *     dk_m = dphi(k_m) o phi'(k_m)                 phi'(x) = 1 (x > 0), e^x
+ * dout is bf16 bits; dq, dk, dv are REAL [B][N][heads][d], overwritten. */
+static REAL dphi(REAL x) { return x > 0 ? 1 : ORACLE_EXP(x); }
+
+void oracle_linear_bwd(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
+                       const uint16_t *dout, int B, int heads, int d, int64_t N,
+                       REAL *dq, REAL *dk, REAL *dv)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int hd = 0; hd < heads; ++hd) {
+            REAL *S = (REAL *)calloc((size_t)d * d, sizeof(REAL));
+            REAL *z = (REAL *)calloc((size_t)d, sizeof(REAL));
+            REAL *dS = (REAL *)calloc((size_t)d * d, sizeof(REAL));
+            REAL *dz = (REAL *)calloc((size_t)d, sizeof(REAL));
+            REAL *pq = (REAL *)malloc(sizeof(REAL) * d);
+            REAL *num = (REAL *)malloc(sizeof(REAL) * d);
+            REAL *dnum = (REAL *)malloc(sizeof(REAL) * d);
+            /* forward state */
+            for (int64_t m = 0; m < N; ++m) {
+                const uint16_t *kr = row_ptr(kk, N, heads, d, b, m, hd);
+                const uint16_t *vr = row_ptr(v, N, heads, d, b, m, hd);
+                for (int a = 0; a < d; ++a) {
+                    REAL pk = phi(bf16_to_real(kr[a]));
+                    z[a] += pk;
+                    for (int c = 0; c < d; ++c) S[a * d + c] += pk * bf16_to_real(vr[c]);
+                }
+            }
+            /* query side: dq and the sums dS, dz */
+            for (int64_t n = 0; n < N; ++n) {
+                const uint16_t *qr = row_ptr(q, N, heads, d, b, n, hd);
+                const uint16_t *gr = row_ptr(dout, N, heads, d, b, n, hd);
+                REAL den = 0;
+                for (int a = 0; a < d; ++a) { pq[a] = phi(bf16_to_real(qr[a])); den += pq[a] * z[a]; }
+                for (int c = 0; c < d; ++c) {
+                    REAL acc = 0;
+                    for (int a = 0; a < d; ++a) acc += pq[a] * S[a * d + c];
+                    num[c] = acc;
+                }
+                REAL gl = 0;
+                for (int c = 0; c < d; ++c) gl += bf16_to_real(gr[c]) * num[c] / den;
+                REAL dden = -gl / den;
+                for (int c = 0; c < d; ++c) dnum[c] = bf16_to_real(gr[c]) / den;
+                REAL *dqr = dq + (((int64_t)b * N + n) * heads + hd) * d;
+                for (int a = 0; a < d; ++a) {
+                    REAL acc = dden * z[a];
+                    for (int c = 0; c < d; ++c) acc += S[a * d + c] * dnum[c];
+                    dqr[a] = acc * dphi(bf16_to_real(qr[a]));
+                    dz[a] += dden * pq[a];
+                    for (int c = 0; c < d; ++c) dS[a * d + c] += pq[a] * dnum[c];
+                }
+            }
+            /* key side: dk, dv */
+            for (int64_t m = 0; m < N; ++m) {
+                const uint16_t *kr = row_ptr(kk, N, heads, d, b, m, hd);
+                const uint16_t *vr = row_ptr(v, N, heads, d, b, m, hd);
+                REAL *dkr = dk + (((int64_t)b * N + m) * heads + hd) * d;
+                REAL *dvr = dv + (((int64_t)b * N + m) * heads + hd) * d;
+                for (int a = 0; a < d; ++a) {
+                    REAL acc = dz[a];
+                    for (int c = 0; c < d; ++c) acc += dS[a * d + c] * bf16_to_real(vr[c]);
+                    dkr[a] = acc * dphi(bf16_to_real(kr[a]));
+                }
+                for (int c = 0; c < d; ++c) {
+                    REAL acc = 0;
+                    for (int a = 0; a < d; ++a) acc += dS[a * d + c] * phi(bf16_to_real(kr[a]));
+                    dvr[c] = acc;
+                }
+            }
+            free(S); free(z); free(dS); free(dz); free(pq); free(num); free(dnum);
+        }
+}
+
 void oracle_dense(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
                   int B, int heads, int d, int64_t N, REAL *out)
 {

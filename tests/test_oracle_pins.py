@@ -360,3 +360,45 @@ def test_fine_bwd_dv_is_weights_times_dout(oracle_mod):
     never = P.sum(0) == 0
     assert never.any(), "case should leave some key tiles unselected"
     assert np.all(dk[0, never] == 0) and np.all(dv[0, never] == 0)
+
+
+# ---------------------------------------------------- linear branch backward
+
+def _torch_linear(q, k, v):
+    """phi(q) S / (phi(q) . z) in torch fp64, phi = elu + 1 (autograd-able)."""
+    pq, pk = torch.nn.functional.elu(q) + 1, torch.nn.functional.elu(k) + 1
+    S = torch.einsum("bnhd,bnhe->bhde", pk, v)
+    z = pk.sum(1)                                              # [B, heads, d]
+    num = torch.einsum("bnhd,bhde->bnhe", pq, S)
+    den = torch.einsum("bnhd,bhd->bnh", pq, z)
+    return num / den[..., None]
+
+
+@pytest.mark.parametrize("case", [(1, 2, 8, 40), (2, 1, 16, 24)])
+def test_linear_bwd_matches_autograd(oracle_mod, case):
+    """P10: the linear-branch backward equals torch autograd (fp64) of the
+    branch written with torch's own elu -- an independent differentiation."""
+    B, heads, d, N = case
+    g = torch.Generator().manual_seed(sum(case))
+    q, k, v = ((0.8 * torch.randn((B, N, heads, d), generator=g)).to(torch.bfloat16) for _ in range(3))
+    dout = _dout(q.shape, seed=17)
+    dq, dk, dv = oracle_mod.linear_bwd(q, k, v, dout, B, heads, d, N)
+    tq, tk, tv = (x.to(torch.float64).requires_grad_() for x in (q, k, v))
+    _torch_linear(tq, tk, tv).backward(dout.to(torch.float64))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_linear_bwd_constant_keys_closed_form(oracle_mod):
+    """P10: with every key equal, lin_n = mean of v for any q (phi(q) cancels),
+    so dq = 0 and dv_m = (sum_n dO_n) / N exactly."""
+    B, heads, d, N = 1, 1, 8, 20
+    g = torch.Generator().manual_seed(3)
+    q, v = ((0.8 * torch.randn((B, N, heads, d), generator=g)).to(torch.bfloat16) for _ in range(2))
+    k = (0.8 * torch.randn((1, 1, 1, d), generator=g)).to(torch.bfloat16).expand(B, N, heads, d).contiguous()
+    dout = _dout(q.shape, seed=4)
+    dq, dk, dv = oracle_mod.linear_bwd(q, k, v, dout, B, heads, d, N)
+    np.testing.assert_allclose(dq, 0, atol=1e-12)
+    ref = dout.to(torch.float64).sum(1, keepdim=True).numpy() / N
+    np.testing.assert_allclose(dv, np.broadcast_to(ref, dv.shape), rtol=0, atol=1e-12)
