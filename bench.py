@@ -371,6 +371,12 @@ def run_kernels(args):
             q, k, v, out32, g_out, attn.block_idx, lse, dq, dk, dv, w.T, w.H, w.W, w.topk,
             attn.workspace, w.tile),
          "tensor", 2.5 * w.fine_flops()),
+        # linear branch backward: reads q, k, v, dout and writes dq, dk, dv
+        # (the d x d states are a few MB); its products are ~10 d^2 FLOPs per
+        # token, far below the tensor-core ridge, so HBM bounds it
+        ("linear_branch_bwd (a6 backward)", lambda: ops.vsa_linear_branch_bwd(
+            q, k, v, g_out, attn.lin_S, attn.lin_z, dq, dk, dv, w.T, w.H, w.W, attn.workspace),
+         "hbm", 7 * elem),
     ]
     for name, fn, bound, units in rows:
         ms = timed(fn)

@@ -105,8 +105,10 @@ size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W, 
     size_t scratch = vsa::select_scratch_bytes(g);
     const size_t image = lin_image_bytes(g);
     const size_t bwd = vsa::bwd_scratch_bytes(g, topk);
+    const size_t lin_bwd = (size_t)vsa::linear_bwd_scratch_bytes(g);
     if (image > scratch) scratch = image;
     if (bwd > scratch) scratch = bwd;
+    if (lin_bwd > scratch) scratch = lin_bwd;
     return kStatusBytes + scratch;
 }
 
@@ -281,6 +283,27 @@ vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     a.scratch = static_cast<uint8_t*>(workspace) + kStatusBytes;
     a.status = static_cast<int*>(workspace);
     return from_cuda(vsa::launch_fine_bwd(a, (cudaStream_t)stream));
+}
+
+vsa_status vsa_linear_branch_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                                 const vsa_bf16* dout, const float* lin_S, const float* lin_z,
+                                 vsa_bf16* dq, vsa_bf16* dk, vsa_bf16* dv, int accumulate, int B,
+                                 int heads, int head_dim, int T, int H, int W, void* workspace,
+                                 size_t workspace_bytes, vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, 4, 4, 4);
+    if (s != VSA_OK) return s;
+    for (const void* p : {(const void*)q, (const void*)k, (const void*)v, (const void*)dout,
+                          (const void*)lin_S, (const void*)lin_z, (const void*)dq, (const void*)dk,
+                          (const void*)dv})
+        if (!aligned16(p)) return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, 4, 4, 4);
+    if (workspace_bytes < kStatusBytes + (size_t)vsa::linear_bwd_scratch_bytes(g)) return VSA_ERR_WORKSPACE;
+    auto fn = encode_fn();
+    if (!fn) return VSA_ERR_CUDA;
+    return from_cuda(vsa::launch_linear_bwd(g, q, k, v, dout, lin_S, lin_z, dq, dk, dv, accumulate,
+                                            static_cast<uint8_t*>(workspace) + kStatusBytes,
+                                            static_cast<int*>(workspace), (cudaStream_t)stream, fn));
 }
 
 vsa_status vsa_device_status(void* workspace, vsa_stream_t stream) {

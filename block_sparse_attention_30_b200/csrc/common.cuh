@@ -101,6 +101,13 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
     return d;
 }
 
+// Fire-and-forget vector add of four floats into global memory (16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
 // 2^x on the MUFU unit (hardware approximation, ~2 ulp).
 __device__ __forceinline__ float ex2(float x) {
     float y;

@@ -58,13 +58,6 @@ struct LinBars {
 static_assert(sizeof(LinBars<64>) <= LinCfg<64>::BAR_BYTES, "barrier block");
 static_assert(sizeof(LinBars<128>) <= LinCfg<128>::BAR_BYTES, "barrier block");
 
-// Fire-and-forget vector add of four floats into global memory (16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
-
 // Where 64-token step gs of the flattened (b*heads, step) space lives.
 struct LinStep {
     int bh, st;       // (b, head) pair and 64-token step within it
@@ -278,8 +271,8 @@ linear_state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constan
 // 3-D view (heads*d, N, B) of a [B][N][heads][d] bf16 tensor; box = 64
 // features x 64 tokens of one batch, 128-byte swizzle; tokens past N are
 // zero-filled.
-static bool encode_token_map(CUtensorMap* m, const void* base, const Grid& g,
-                             PFN_cuTensorMapEncodeTiled_v12000 fn) {
+bool encode_token_map(CUtensorMap* m, const void* base, const Grid& g,
+                      PFN_cuTensorMapEncodeTiled_v12000 fn) {
     const cuuint64_t row = (cuuint64_t)g.heads * g.d;
     cuuint64_t dims[3] = {row, (cuuint64_t)g.N, (cuuint64_t)g.B};
     cuuint64_t strides[2] = {row * 2, row * 2 * (cuuint64_t)g.N};

@@ -118,6 +118,18 @@ def vsa_sparse_attn_bwd(q, k, v, out_f32, dout, block_idx, lse, dq, dk, dv, T, H
         _stream(stream)))
 
 
+def vsa_linear_branch_bwd(q, k, v, dout, lin_S, lin_z, dq, dk, dv, T, H, W, workspace,
+                          accumulate=False, stream=None):
+    """Gradients dq, dk, dv (bf16, in place) of the linear branch
+    phi(q)S/(phi(q).z); with accumulate=True they are added to the values
+    already in dq, dk, dv."""
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_linear_branch_bwd", _lib.lib().vsa_linear_branch_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), lin_S.data_ptr(),
+        lin_z.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), int(bool(accumulate)), B,
+        heads, d, T, H, W, workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
 def vsa_device_status(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = VSA_OK)."""
     return _lib.lib().vsa_device_status(workspace.data_ptr(), _stream(stream))

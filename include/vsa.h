@@ -80,8 +80,9 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
  * holds either the selection's fp64 cube means of q and k
  * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the
  * linear branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is
- * larger (the backward pass's row terms and block-index transpose fit it
- * too).  Returns 0 for invalid shapes.  The
+ * larger (the backward passes' scratch fits it too: the sparse branch's row
+ * terms and block-index transpose, the linear branch's two operand images
+ * and fp32 gradient sums).  Returns 0 for invalid shapes.  The
  * same workspace may be passed to every call of one forward pass; calls that
  * share a workspace must be ordered on one stream. */
 size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W,
@@ -177,6 +178,30 @@ vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
                                int heads, int head_dim, int T, int H, int W, int tt, int th, int tw,
                                int topk, void* workspace, size_t workspace_bytes,
                                vsa_stream_t stream);
+
+/* Backward of the linear branch (SparkDiffusion RoLA, paragraph 3;
+ * TurboDiffusion SLA, "稀疏、蒸馏与全链路量化": the linear branch is trained
+ * with the sparse one).  For lin_n = phi(q_n) S / (phi(q_n).z), phi = elu + 1,
+ * with lin_S and lin_z from vsa_linear_branch_fwd over the same k and v, and
+ * the output gradient dout (bf16 [B][N][heads][d]), writes the bf16
+ * gradients of the branch to dq, dk, dv (same layout):
+ *     u_n = S dout_n, e_n = -phi(q_n).u_n / (phi(q_n).z)^2,
+ *     dq_n = (u_n / (phi(q_n).z) + e_n z) o phi'(q_n),
+ *     dS = sum_n phi(q_n)^T dout_n / (phi(q_n).z),  dz = sum_n e_n phi(q_n),
+ *     dk_m = (dS v_m + dz) o phi'(k_m),  dv_m = phi(k_m) dS,
+ * products on the tensor cores with bf16 hi + lo operands (fp32-level) and
+ * fp32 accumulation, dS and dz summed with fp32 atomics (run-to-run
+ * differences at the fp32 rounding level).  accumulate == 0 overwrites dq,
+ * dk, dv; accumulate != 0 adds the branch's gradients to the bf16 values
+ * already there (e.g. from vsa_sparse_attn_bwd), rounding the sum once.
+ * Uses B*heads*3*(4*d*d + 4*d) bytes (each third rounded up to 256) of the
+ * workspace scratch, within vsa_workspace_bytes(); returns VSA_ERR_WORKSPACE
+ * when the workspace is smaller. */
+vsa_status vsa_linear_branch_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                                 const vsa_bf16* dout, const float* lin_S, const float* lin_z,
+                                 vsa_bf16* dq, vsa_bf16* dk, vsa_bf16* dv, int accumulate, int B,
+                                 int heads, int head_dim, int T, int H, int W, void* workspace,
+                                 size_t workspace_bytes, vsa_stream_t stream);
 
 /* Self-test of the device failure path (no counterpart on the pages): a
  * one-warp kernel waits on a barrier nobody arrives at, gives up after

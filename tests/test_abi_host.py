@@ -31,6 +31,7 @@ def declared_functions():
 def test_header_declares_expected_entry_points():
     names = declared_functions()
     for n in ["vsa_select_blocks", "vsa_sparse_attn_fwd", "vsa_linear_branch_fwd",
+              "vsa_sparse_attn_fwd_train", "vsa_sparse_attn_bwd", "vsa_linear_branch_bwd",
               "vsa_gather_tiles", "vsa_scatter_tiles", "vsa_workspace_bytes",
               "vsa_device_status", "vsa_status_string"]:
         assert n in names
@@ -60,9 +61,12 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 0) == 0         # topk < 1
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 456) == 0       # topk > nt
-    # tiny grids: the linear branch's operand image (4*d*d + 4*d bytes per
-    # (b, head)) is larger than the selection scratch and sets the size
-    assert L.vsa_workspace_bytes(1, 2, 128, 4, 8, 8, 4, 4, 4, 2) == 256 + 2 * (4 * 128 * 128 + 4 * 128)
+    # tiny grids: the linear branch's backward scratch (two operand images of
+    # 4*d*d + 4*d bytes per (b, head) and the fp32 (dS, dz) sums, the same
+    # size, each third rounded up to 256 bytes) is larger than the selection
+    # scratch and sets the size
+    third = -(-2 * (4 * 128 * 128 + 4 * 128) // 256) * 256
+    assert L.vsa_workspace_bytes(1, 2, 128, 4, 8, 8, 4, 4, 4, 2) == 256 + 3 * third
 
 
 SHAPE = [1, 2, 128, 4, 8, 8, 4, 4, 4]       # nt = 4
@@ -107,6 +111,15 @@ def test_other_entry_points_validate(L):
     assert L.vsa_linear_branch_fwd(FAKE, FAKE, None, FAKE, 1, 2, 128, 4, 8, 8, FAKE, 1024, None) == INVALID
     assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 32, 4, 8, 8, FAKE, 1024, None) == UNSUPPORTED
     assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, 1, 2, 128, 4, 8, 8, None, 1024, None) == WORKSPACE
+    lb = L.vsa_linear_branch_bwd
+    third = -(-2 * (4 * 128 * 128 + 4 * 128) // 256) * 256
+    ok_ws = 256 + 3 * third
+    assert lb(*[FAKE] * 9, 0, 1, 2, 128, 4, 8, 8, FAKE, ok_ws - 16, None) == WORKSPACE
+    assert lb(*[FAKE] * 9, 0, 1, 2, 128, 4, 8, 8, None, ok_ws, None) == WORKSPACE
+    assert lb(FAKE, FAKE, FAKE, None, *[FAKE] * 5, 0, 1, 2, 128, 4, 8, 8, FAKE, ok_ws, None) == INVALID
+    assert lb(*[FAKE] * 8, FAKE + 8, 0, 1, 2, 128, 4, 8, 8, FAKE, ok_ws, None) == INVALID   # misaligned dv
+    assert lb(*[FAKE] * 9, 0, 1, 2, 96, 4, 8, 8, FAKE, ok_ws, None) == UNSUPPORTED
+    assert lb(*[FAKE] * 9, 0, 0, 2, 128, 4, 8, 8, FAKE, ok_ws, None) == INVALID
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID

@@ -476,3 +476,88 @@ def test_host_pipeline_matches_direct_calls(ops):
         ref = attn(c.q.cuda(), c.k.cuda(), c.v.cuda())
         torch.cuda.synchronize()
         assert torch.equal(o, ref.cpu())
+
+
+# ------------------------------------------------ linear branch, backward
+# dout is exact in bf16 and meets S as bf16 hi + lo; phi(q)/den, phi(k) and dS
+# also enter the tensor cores as hi + lo, and the per-token terms are fp32, so
+# the products are good to ~2^-16 relative and the error is set by the final
+# bf16 rounding of the gradients (2^-9 relative per element) and by dz, dS
+# summed in fp32.  Bound: relative Frobenius error <= 4e-3 and max-abs error
+# <= 1e-2 x the largest reference magnitude, per gradient.
+LIN_GRAD_REL_FRO, LIN_GRAD_MAX_REL = 4e-3, 1e-2
+
+
+def check_lin_grad(got, ref, name):
+    ref = np.asarray(ref)
+    scale = max(np.abs(ref).max(), 1e-6)
+    err = np.abs(got - ref).max()
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    print(f"{name}: max-abs {err:.3e} (scale {scale:.3e}, {err / scale:.3%}), rel-Frobenius {rel:.3%}")
+    assert err <= LIN_GRAD_MAX_REL * scale and rel <= LIN_GRAD_REL_FRO, (name, err, scale, rel)
+
+
+def run_linear_bwd(ops, q, k, v, dout, T, H, W, prefill=None):
+    B, N, heads, d = q.shape
+    qd, kd, vd, gd = (x.cuda() for x in (q, k, v, dout))
+    S = torch.empty((B, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((B, heads, d), dtype=torch.float32, device="cuda")
+    ws = ops.new_workspace(B, heads, d, T, H, W, 1)
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
+    if prefill is None:
+        dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    else:
+        dq, dk, dv = (x.cuda().clone() for x in prefill)
+    ops.vsa_linear_branch_bwd(qd, kd, vd, gd, S, z, dq, dk, dv, T, H, W, ws,
+                              accumulate=prefill is not None)
+    assert ops.vsa_device_status(ws) == 0
+    return dq, dk, dv
+
+
+LIN_BWD_CASES = [
+    # B, heads, d, T, H, W
+    (1, 2, 128, 4, 8, 8),        # N = 256: two whole 128-token steps per head
+    (1, 3, 128, 5, 6, 7),        # N = 210: ragged last step
+    (2, 2, 64, 9, 13, 10),       # d = 64, B = 2, ragged
+    (1, 8, 128, 20, 16, 16),     # 40 steps per head: 3-step CTA slices cross (b, head)
+]
+
+
+@pytest.mark.parametrize("case", LIN_BWD_CASES)
+def test_linear_backward_small(ops, case):
+    B, heads, d, T, H, W = case
+    q, k, v = synth.make_qkv(B, heads, d, T, H, W, amplitude=0.7, seed=sum(case))
+    dout = make_dout(q.shape, seed=5)
+    dq, dk, dv = run_linear_bwd(ops, q, k, v, dout, T, H, W)
+    refs = O.linear_bwd(q, k, v, dout, B, heads, d, T * H * W)
+    for got, ref, name in zip((dq, dk, dv), refs, ("dq", "dk", "dv")):
+        assert not torch.isnan(got).any(), name + " must be fully written"
+        check_lin_grad(to_f64(got), ref, name)
+
+
+def test_linear_backward_accumulates(ops):
+    """accumulate: the branch's gradients are added to what dq, dk, dv hold
+    (the sparse branch's gradients in a training step), one rounding."""
+    B, heads, d, T, H, W = 1, 2, 128, 5, 6, 7
+    q, k, v = synth.make_qkv(B, heads, d, T, H, W, amplitude=0.7, seed=77)
+    dout = make_dout(q.shape, seed=6)
+    prefill = [make_dout(q.shape, seed=s) for s in (10, 11, 12)]
+    dq, dk, dv = run_linear_bwd(ops, q, k, v, dout, T, H, W, prefill=prefill)
+    refs = O.linear_bwd(q, k, v, dout, B, heads, d, T * H * W)
+    for got, ref, pre, name in zip((dq, dk, dv), refs, prefill, ("dq", "dk", "dv")):
+        check_lin_grad(to_f64(got), ref + pre.double().numpy(), name)
+
+
+def test_linear_backward_workload_two_heads(ops):
+    """Full-size 97 %-sparse workload with the linear branch: the backward
+    over all 12 heads, every token of two heads checked."""
+    w, q, k, v, qd, kd, vd = inputs("sparse97_linear_480p")
+    dout = make_dout(q.shape, seed=13)
+    dq, dk, dv = run_linear_bwd(ops, q, k, v, dout, w.T, w.H, w.W)
+    for x, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        assert torch.isfinite(x).all(), name
+    hs = slice(0, 2)
+    sub = lambda x: x[:, :, hs].contiguous()
+    refs = O.linear_bwd(sub(q), sub(k), sub(v), sub(dout), w.B, 2, w.head_dim, w.N)
+    for got, ref, name in zip((dq, dk, dv), refs, ("dq", "dk", "dv")):
+        check_lin_grad(to_f64(got[:, :, hs]), ref, name)
