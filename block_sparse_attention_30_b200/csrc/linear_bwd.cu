@@ -15,7 +15,8 @@
 // kept from the forward pass: S and z are its only state.
 //
 // Two kernels, each one CTA per SM over 128-token steps of the flattened
-// (b*heads, step) space, warps 0-3 one thread per token, warp 4 TMA + MMA:
+// (b*heads, step) space, warps 0-7 two threads per token (one per half of the
+// features), warp 8 TMA + MMA:
 //  * query side: U = G S^T on the tensor cores (G = dout is exact in bf16, S
 //    enters as bf16 hi + lo, so u is good to ~2^-17), the per-token terms on
 //    the CUDA cores, then dS += (phi(Q)/den)^T G (phi/den as hi + lo) into a
@@ -47,7 +48,9 @@ struct LbCfg {
     static constexpr int IMG_OFF = 5 * TILE;
     static constexpr int BAR_OFF = IMG_OFF + IMG;
     static constexpr int SMEM_BYTES = BAR_OFF + 256;
-    static constexpr int THREADS = 160;
+    static constexpr int EPI = 256;                      // epilogue threads: 2 per token
+    static constexpr int MMA_WARP = EPI / 32;            // TMA + MMA warp
+    static constexpr int THREADS = EPI + 32;
     static constexpr int ACC2 = 128;                     // TMEM column of the second accumulator
     static constexpr int TMEM_COLS = 256;
 };
@@ -58,8 +61,9 @@ struct LbBars {
     uint64_t done[2];     // (query side) MMAs reading buffer b finished
     uint64_t img_full;    // operand image landed (once per segment)
     uint64_t acc_full;    // the step's accumulator(s) written
-    uint64_t ready;       // epilogue warps finished a step (128 arrivals)
-    uint64_t kready;      // (key side) phi(K) hi/lo written (128 arrivals)
+    uint64_t ready;       // epilogue warps finished a step (all epilogue threads)
+    uint64_t kready;      // (key side) phi(K) hi/lo written (all epilogue threads)
+    uint64_t pair[4];     // (query side) both warps of a token group finished pass 1
     uint64_t seg_done;    // (query side) dS accumulation of a segment finished
     uint64_t mma_idle;    // every MMA of the CTA finished
     uint32_t tmem_base;
@@ -162,13 +166,14 @@ __device__ __forceinline__ LbBars* lb_setup(uint8_t* smem, int warp) {
         }
         mbar_init(&bars->img_full, 1);
         mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->ready, 128);
-        mbar_init(&bars->kready, 128);
+        mbar_init(&bars->ready, C::EPI);
+        mbar_init(&bars->kready, C::EPI);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 64);
         mbar_init(&bars->seg_done, 1);
         mbar_init(&bars->mma_idle, 1);
         fence_barrier_init();
     }
-    if (warp == 4) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+    if (warp == C::MMA_WARP) { tmem_alloc(&bars->tmem_base, C::TMEM_COLS); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -223,7 +228,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
     const int n_steps = (int)max(0ll, min((long long)steps_per_cta, total_steps - gs0));
     auto fail = [&]() { *abort_flag = 1; report(status, kStatusTimeout); };
 
-    if (warp == 4) {
+    if (warp == C::MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             // ------------------------------------------------ loads + MMAs
             const uint32_t id_u = idesc_bf16_f32(128, D, false, false);   // U = G S^T
@@ -297,13 +302,18 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
             wait_noabort(&bars->mma_idle, 0);
         }
     } else {
-        // ------------------------------------------- one thread per token
-        const int r = tid;                                   // row of the step tile
-        const uint32_t lanes = (uint32_t)(32 * warp) << 16;  // this warp's TMEM lanes
+        // ------------------------------------------ two threads per token
+        // warps w and w + 4 share TMEM sub-partition w % 4 (tokens 32 (w % 4)
+        // + lane) and split the features in halves; both form the per-token
+        // dot products over all features, which costs less than exchanging them
+        constexpr int HC = D / 32;                           // 16-feature chunks per half
+        const int sp = warp & 3, hf = warp >> 2;
+        const int r = 32 * sp + lane;                        // row of the step tile
+        const uint32_t lanes = (uint32_t)(32 * sp) << 16;    // this warp's TMEM lanes
         const float* zs = reinterpret_cast<const float*>(smem + C::IMG_OFF + 4 * D * D);
-        float dzacc[D / 16];
+        float dzacc[HC];
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) dzacc[c] = 0.f;
+        for (int c = 0; c < HC; ++c) dzacc[c] = 0.f;
         bool ok = true;
         int seg = -1;
         for (int t = 0; t < n_steps; ++t) {
@@ -340,13 +350,17 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                     gu = fmaf(p, u[e], gu);
                 }
             }
+            // pass 2 overwrites this half of the Q tile, which the other warp's
+            // pass 1 reads: both finish pass 1 first
+            mbar_arrive(&bars->pair[sp]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->pair[sp], t & 1, abort_flag))) { ok = false; break; }
             const float rden = valid ? 1.f / den : 0.f;
             const float ecoef = -gu * rden * rden;
 
-            // pass 2: dq, (phi/den) hi/lo for the dS product, dz
+            // pass 2 (this warp's half): dq, (phi/den) hi/lo for the dS product, dz
             __nv_bfloat16* dqrow = dq + (((long long)bb * g.N + n) * g.heads + head) * D;
 #pragma unroll 1
-            for (int c16 = 0; c16 < D / 16; ++c16) {
+            for (int c16 = hf * HC; c16 < (hf + 1) * HC; ++c16) {
                 float u[16];
                 tmem_ld_32x32b_x16(tbase + lanes + 16 * c16, u);
                 float qf[16];
@@ -375,7 +389,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                     store8(dqrow + 16 * c16, dqv, accumulate != 0);
                     store8(dqrow + 16 * c16 + 8, dqv + 8, accumulate != 0);
                 }
-                dzacc[c16] += warp_reduce_scatter16(zc, lane);
+                dzacc[c16 - hf * HC] += warp_reduce_scatter16(zc, lane);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -385,19 +399,20 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                 // dz of the segment: lane 2j holds feature 16 c + j of each chunk c
                 if ((lane & 1) == 0) {
 #pragma unroll
-                    for (int c = 0; c < D / 16; ++c) atomicAdd(dz + (long long)x.bh * D + 16 * c + (lane >> 1), dzacc[c]);
+                    for (int c = 0; c < HC; ++c)
+                        atomicAdd(dz + (long long)x.bh * D + 16 * (hf * HC + c) + (lane >> 1), dzacc[c]);
                 }
 #pragma unroll
-                for (int c = 0; c < D / 16; ++c) dzacc[c] = 0.f;
+                for (int c = 0; c < HC; ++c) dzacc[c] = 0.f;
                 // dS of the segment: M = 128 puts feature a in lane a; M = 64
                 // puts it in lane (a % 16) + 32 (a / 16)
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars->seg_done, seg & 1, abort_flag))) { ok = false; break; }
                 tc_fence_after();
-                const int a = D == 128 ? 32 * warp + lane : 16 * warp + lane;
+                const int a = D == 128 ? 32 * sp + lane : 16 * sp + lane;
                 const bool mine = D == 128 || lane < 16;
                 float* Sb = dS + ((long long)x.bh * D + a) * D;
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 16) {
+                for (int c0 = hf * D / 2; c0 < (hf + 1) * D / 2; c0 += 16) {
                     float vals[16];
                     tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + c0, vals);
                     tmem_wait_ld();
@@ -414,7 +429,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) tmem_dealloc(tbase, C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tmem_dealloc(tbase, C::TMEM_COLS);
 }
 
 // --------------------------------------------------------------- key side
@@ -440,7 +455,7 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
     const int n_steps = (int)max(0ll, min((long long)steps_per_cta, total_steps - gs0));
     auto fail = [&]() { *abort_flag = 1; report(status, kStatusTimeout); };
 
-    if (warp == 4) {
+    if (warp == C::MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             const uint32_t id_u = idesc_bf16_f32(128, D, false, false);   // U' = V dS^T
             const uint32_t id_v = idesc_bf16_f32(128, D, false, true);    // dV = phi(K) dS
@@ -497,8 +512,11 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             wait_noabort(&bars->mma_idle, 0);
         }
     } else {
-        const int r = tid;
-        const uint32_t lanes = (uint32_t)(32 * warp) << 16;
+        // warps w and w + 4: tokens 32 (w % 4) + lane, feature halves
+        constexpr int HC = D / 32;
+        const int sp = warp & 3, hf = warp >> 2;
+        const int r = 32 * sp + lane;
+        const uint32_t lanes = (uint32_t)(32 * sp) << 16;
         const float* dzs = reinterpret_cast<const float*>(smem + C::IMG_OFF + 4 * D * D);
         bool ok = true;
         int seg = -1;
@@ -513,7 +531,7 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->full[b], (t >> 1) & 1, abort_flag))) { ok = false; break; }
             // phi(K) hi in place, lo beside it; zero past the end of the grid
 #pragma unroll 1
-            for (int u = 0; u < D / 8; ++u) {
+            for (int u = hf * D / 16; u < (hf + 1) * D / 16; ++u) {
                 const uint32_t o = unit_off<D>(u >> 3, u & 7, r);
                 float f[8];
                 unpack8(*reinterpret_cast<const uint4*>(kt + o), f);
@@ -535,7 +553,7 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             __nv_bfloat16* dkrow = dk + (((long long)bb * g.N + n) * g.heads + head) * D;
             __nv_bfloat16* dvrow = dv + (((long long)bb * g.N + n) * g.heads + head) * D;
 #pragma unroll 1
-            for (int c16 = 0; c16 < D / 16; ++c16) {
+            for (int c16 = hf * HC; c16 < (hf + 1) * HC; ++c16) {
                 float u[16], w[16];
                 tmem_ld_32x32b_x16(tbase + lanes + 16 * c16, u);
                 tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + 16 * c16, w);
@@ -567,7 +585,7 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) tmem_dealloc(tbase, C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tmem_dealloc(tbase, C::TMEM_COLS);
 }
 
 long long linear_bwd_scratch_bytes(const Grid& g) {
