@@ -15,8 +15,8 @@
 // kept from the forward pass: S and z are its only state.
 //
 // Two kernels, each one CTA per SM over 128-token steps of the flattened
-// (b*heads, step) space, warps 0-7 two threads per token (one per half of the
-// features), warp 8 TMA + MMA:
+// (b*heads, step) space, with G epilogue threads per token (each owning D/G
+// features; G = 2 on the query side, 4 on the key side) and one TMA + MMA warp:
 //  * query side: U = G S^T on the tensor cores (G = dout is exact in bf16, S
 //    enters as bf16 hi + lo, so u is good to ~2^-17), the per-token terms on
 //    the CUDA cores, then dS += (phi(Q)/den)^T G (phi/den as hi + lo) into a
@@ -38,23 +38,31 @@
 namespace vsa {
 using namespace sm100;
 
-template <int D>
+// G epilogue threads per token, each owning D/G consecutive features.
+template <int D, int G>
 struct LbCfg {
     static constexpr int ROWS = 128;                     // tokens per step
     static constexpr int CHUNK = ROWS * 128;             // one 64-feature chunk of a step tile
     static constexpr int TILE = (D / 64) * CHUNK;        // one tensor's step tile
-    static constexpr int IMG = (int)((linear_image_bytes(D) + 1023) / 1024 * 1024);
-    static constexpr int LO_OFF = 4 * TILE;              // [X0 | Y0 | X1 | Y1 | LO | IMG | bars]
+    static constexpr int IMG = (int)linear_image_bytes(D);  // S hi, S lo (1024-aligned), z
+    static constexpr int LO_OFF = 4 * TILE;              // [X0 | Y0 | X1 | Y1 | LO | IMG | bars | xch]
     static constexpr int IMG_OFF = 5 * TILE;
     static constexpr int BAR_OFF = IMG_OFF + IMG;
-    static constexpr int SMEM_BYTES = BAR_OFF + 256;
-    static constexpr int EPI = 256;                      // epilogue threads: 2 per token
+    static constexpr int XCH_OFF = BAR_OFF + 256;        // per-token partial sums (query side)
+    static constexpr int XCH_BYTES = G * 2 * ROWS * 4;
+    static constexpr int EPI = ROWS * G;                 // epilogue threads
     static constexpr int MMA_WARP = EPI / 32;            // TMA + MMA warp
     static constexpr int THREADS = EPI + 32;
+    static constexpr int FC = D / G;                     // features per epilogue thread
+    static constexpr int NC = FC / 16;                   // 16-feature chunks per epilogue thread
     static constexpr int ACC2 = 128;                     // TMEM column of the second accumulator
     static constexpr int TMEM_COLS = 256;
 };
-static_assert(LbCfg<128>::SMEM_BYTES <= 232448, "shared memory");
+// query side: 2 threads per token and the exchange area; key side: 4, none
+constexpr int kQueryG = 2, kKeyG = 4;
+static_assert(LbCfg<128, kQueryG>::XCH_OFF + LbCfg<128, kQueryG>::XCH_BYTES <= 232448, "shared memory");
+static_assert(LbCfg<128, kKeyG>::XCH_OFF <= 232448, "shared memory");
+static_assert(LbCfg<64, kKeyG>::NC >= 1, "at least one chunk per thread");
 
 struct LbBars {
     uint64_t full[2];     // X and Y tiles of buffer b landed
@@ -63,7 +71,7 @@ struct LbBars {
     uint64_t acc_full;    // the step's accumulator(s) written
     uint64_t ready;       // epilogue warps finished a step (all epilogue threads)
     uint64_t kready;      // (key side) phi(K) hi/lo written (all epilogue threads)
-    uint64_t pair[4];     // (query side) both warps of a token group finished pass 1
+    uint64_t pair[4];     // (query side) all warps of a token group finished pass 1
     uint64_t seg_done;    // (query side) dS accumulation of a segment finished
     uint64_t mma_idle;    // every MMA of the CTA finished
     uint32_t tmem_base;
@@ -146,17 +154,25 @@ __device__ __forceinline__ float warp_reduce_scatter16(float (&v)[16], int lane)
     return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
+// Ties 16 values to this point of the program: placed right after
+// tcgen05.wait::ld, it keeps the compiler from touching registers that an
+// asynchronous TMEM load is still writing before the wait.
+__device__ __forceinline__ void reg_fence16(float (&v)[16]) {
+    asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                      "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                      "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+
 // Byte offset of 16-byte unit u (8 features) of 64-feature chunk ch of token
 // row r in a step tile (TMA 128-byte swizzle).
-template <int D>
 __device__ __forceinline__ uint32_t unit_off(int ch, int u, int r) {
-    return ch * LbCfg<D>::CHUNK + r * 128 + ((u ^ (r & 7)) << 4);
+    return ch * (128 * 128) + r * 128 + ((u ^ (r & 7)) << 4);
 }
 
 // Shared setup: barriers and TMEM.
-template <int D>
+template <int D, int G>
 __device__ __forceinline__ LbBars* lb_setup(uint8_t* smem, int warp) {
-    using C = LbCfg<D>;
+    using C = LbCfg<D, G>;
     LbBars* bars = reinterpret_cast<LbBars*>(smem + C::BAR_OFF);
     if (threadIdx.x == 0) {
         bars->abort = 0;
@@ -168,7 +184,7 @@ __device__ __forceinline__ LbBars* lb_setup(uint8_t* smem, int warp) {
         mbar_init(&bars->acc_full, 1);
         mbar_init(&bars->ready, C::EPI);
         mbar_init(&bars->kready, C::EPI);
-        for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 64);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 32 * G);
         mbar_init(&bars->seg_done, 1);
         mbar_init(&bars->mma_idle, 1);
         fence_barrier_init();
@@ -181,11 +197,11 @@ __device__ __forceinline__ LbBars* lb_setup(uint8_t* smem, int warp) {
 }
 
 // Loads of one step (two tensors, 128 tokens, all features) into buffer b.
-template <int D>
+template <int D, int G>
 __device__ __forceinline__ void lb_load_step(uint8_t* smem, LbBars* bars, const CUtensorMap* mx,
                                              const CUtensorMap* my, const Grid& g, const LbStep& x,
                                              int b) {
-    using C = LbCfg<D>;
+    using C = LbCfg<D, G>;
     const int bb = x.bh / g.heads, head = x.bh % g.heads;
     uint8_t* xb = smem + (2 * b) * C::TILE;
     uint8_t* yb = smem + (2 * b + 1) * C::TILE;
@@ -198,30 +214,30 @@ __device__ __forceinline__ void lb_load_step(uint8_t* smem, LbBars* bars, const 
         }
 }
 
-template <int D>
+template <int D, int G>
 __device__ __forceinline__ void lb_load_image(uint8_t* smem, LbBars* bars, const uint8_t* image, int bh) {
     mbar_arrive_expect_tx(&bars->img_full, (uint32_t)linear_image_bytes(D));
-    bulk_load(smem + LbCfg<D>::IMG_OFF, image + (long long)bh * linear_image_bytes(D),
+    bulk_load(smem + LbCfg<D, G>::IMG_OFF, image + (long long)bh * linear_image_bytes(D),
               (uint32_t)linear_image_bytes(D), &bars->img_full);
 }
 
 // ------------------------------------------------------------- query side
 // X = Q (overwritten in place by (phi(q)/den) hi), Y = G = dout.
 template <int D>
-__global__ void __launch_bounds__(LbCfg<D>::THREADS, 1)
+__global__ void __launch_bounds__(LbCfg<D, kQueryG>::THREADS, 1)
 linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mg,
                         const Grid g, const int steps_per_head, const long long total_steps,
                         const int steps_per_cta, const uint8_t* __restrict__ image,
                         __nv_bfloat16* __restrict__ dq, const int accumulate, float* __restrict__ dS,
                         float* __restrict__ dz, int* status) {
-    using C = LbCfg<D>;
+    using C = LbCfg<D, kQueryG>;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {
         if (threadIdx.x == 0) report(status, kStatusMisaligned);
         return;
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    LbBars* bars = lb_setup<D>(smem, warp);
+    LbBars* bars = lb_setup<D, kQueryG>(smem, warp);
     volatile int* abort_flag = &bars->abort;
     const uint32_t tbase = bars->tmem_base;
     const long long gs0 = (long long)blockIdx.x * steps_per_cta;
@@ -262,9 +278,9 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
             };
             bool ok = true;
             int issued = 0, seg = 0;
-            lb_load_image<D>(smem, bars, image, lb_step(gs0, 0, n_steps, steps_per_head).bh);
+            lb_load_image<D, kQueryG>(smem, bars, image, lb_step(gs0, 0, n_steps, steps_per_head).bh);
             for (int t = 0; t < min(2, n_steps); ++t) {
-                lb_load_step<D>(smem, bars, &mq, &mg, g, lb_step(gs0, t, n_steps, steps_per_head), t);
+                lb_load_step<D, kQueryG>(smem, bars, &mq, &mg, g, lb_step(gs0, t, n_steps, steps_per_head), t);
                 ++issued;
             }
             if (!mbar_wait_spin(&bars->img_full, 0, abort_flag) || !mbar_wait_spin(&bars->full[0], 0, abort_flag)) ok = false;
@@ -280,7 +296,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                     if (x1.first) {
                         // U(t) was read (ready), so the old image is free
                         ++seg;
-                        lb_load_image<D>(smem, bars, image, x1.bh);
+                        lb_load_image<D, kQueryG>(smem, bars, image, x1.bh);
                         if (!mbar_wait_spin(&bars->img_full, seg & 1, abort_flag)) { ok = false; break; }
                     }
                     if (!mbar_wait_spin(&bars->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -289,7 +305,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                 }
                 if (t + 2 < n_steps) {
                     if (!mbar_wait_spin(&bars->done[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-                    lb_load_step<D>(smem, bars, &mq, &mg, g, lb_step(gs0, t + 2, n_steps, steps_per_head), t & 1);
+                    lb_load_step<D, kQueryG>(smem, bars, &mq, &mg, g, lb_step(gs0, t + 2, n_steps, steps_per_head), t & 1);
                     ++issued;
                 }
             }
@@ -302,18 +318,21 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
             wait_noabort(&bars->mma_idle, 0);
         }
     } else {
-        // ------------------------------------------ two threads per token
-        // warps w and w + 4 share TMEM sub-partition w % 4 (tokens 32 (w % 4)
-        // + lane) and split the features in halves; both form the per-token
-        // dot products over all features, which costs less than exchanging them
-        constexpr int HC = D / 32;                           // 16-feature chunks per half
-        const int sp = warp & 3, hf = warp >> 2;
+        // ------------------------------------------ G threads per token
+        // warps w, w + 4, ... share TMEM sub-partition w % 4 (tokens 32 (w % 4)
+        // + lane) and split the features: warp w owns the NC 16-feature chunks
+        // from (w / 4) NC.  The per-token dot products are summed from the parts
+        // through shared memory.
+        constexpr int NC = C::NC;
+        const int sp = warp & 3, part = warp >> 2;
         const int r = 32 * sp + lane;                        // row of the step tile
         const uint32_t lanes = (uint32_t)(32 * sp) << 16;    // this warp's TMEM lanes
+        const int c_lo = part * NC;
         const float* zs = reinterpret_cast<const float*>(smem + C::IMG_OFF + 4 * D * D);
-        float dzacc[HC];
+        float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);   // [G][den, gu][128 rows]
+        float dzacc[NC];
 #pragma unroll
-        for (int c = 0; c < HC; ++c) dzacc[c] = 0.f;
+        for (int c = 0; c < NC; ++c) dzacc[c] = 0.f;
         bool ok = true;
         int seg = -1;
         for (int t = 0; t < n_steps; ++t) {
@@ -332,64 +351,86 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
             uint8_t* qt = smem + (2 * b) * C::TILE;
             uint8_t* lot = smem + C::LO_OFF;
 
-            // pass 1: den = phi(q).z, gu = phi(q).u
+            // pass 1 (own features): partial den = phi(q).z and gu = phi(q).u;
+            // the TMEM read of chunk i + 1 overlaps the arithmetic of chunk i
             float den = 0.f, gu = 0.f;
-#pragma unroll 1
-            for (int c16 = 0; c16 < D / 16; ++c16) {
-                float u[16];
-                tmem_ld_32x32b_x16(tbase + lanes + 16 * c16, u);
-                float qf[16];
-                const int ch = c16 >> 2, u0 = 2 * (c16 & 3);
-                unpack8(*reinterpret_cast<const uint4*>(qt + unit_off<D>(ch, u0, r)), qf);
-                unpack8(*reinterpret_cast<const uint4*>(qt + unit_off<D>(ch, u0 + 1, r)), qf + 8);
+            {
+                float ub[2][16];
+                tmem_ld_32x32b_x16(tbase + lanes + 16 * c_lo, ub[0]);
                 tmem_wait_ld();
+                reg_fence16(ub[0]);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p = phi_elu1(qf[e]);
-                    den = fmaf(p, zs[16 * c16 + e], den);
-                    gu = fmaf(p, u[e], gu);
+                for (int i = 0; i < NC; ++i) {
+                    const int c16 = c_lo + i;
+                    if (i + 1 < NC) tmem_ld_32x32b_x16(tbase + lanes + 16 * (c16 + 1), ub[(i + 1) & 1]);
+                    float qf[16];
+                    const int ch = c16 >> 2, u0 = 2 * (c16 & 3);
+                    unpack8(*reinterpret_cast<const uint4*>(qt + unit_off(ch, u0, r)), qf);
+                    unpack8(*reinterpret_cast<const uint4*>(qt + unit_off(ch, u0 + 1, r)), qf + 8);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p = phi_elu1(qf[e]);
+                        den = fmaf(p, zs[16 * c16 + e], den);
+                        gu = fmaf(p, ub[i & 1][e], gu);
+                    }
+                    if (i + 1 < NC) { tmem_wait_ld(); reg_fence16(ub[(i + 1) & 1]); }
                 }
             }
-            // pass 2 overwrites this half of the Q tile, which the other warp's
-            // pass 1 reads: both finish pass 1 first
+            xch[(2 * part) * 128 + r] = den;
+            xch[(2 * part + 1) * 128 + r] = gu;
+            // the parts are shared, and pass 2 overwrites this part of the Q
+            // tile that the other warps' pass 1 reads: all finish pass 1 first
             mbar_arrive(&bars->pair[sp]);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pair[sp], t & 1, abort_flag))) { ok = false; break; }
+            den = 0.f;
+            gu = 0.f;
+#pragma unroll
+            for (int p2 = 0; p2 < kQueryG; ++p2) {     // same order in every warp
+                den += xch[(2 * p2) * 128 + r];
+                gu += xch[(2 * p2 + 1) * 128 + r];
+            }
             const float rden = valid ? 1.f / den : 0.f;
             const float ecoef = -gu * rden * rden;
 
-            // pass 2 (this warp's half): dq, (phi/den) hi/lo for the dS product, dz
+            // pass 2 (own features): dq, (phi/den) hi/lo for the dS product, dz
             __nv_bfloat16* dqrow = dq + (((long long)bb * g.N + n) * g.heads + head) * D;
-#pragma unroll 1
-            for (int c16 = hf * HC; c16 < (hf + 1) * HC; ++c16) {
-                float u[16];
-                tmem_ld_32x32b_x16(tbase + lanes + 16 * c16, u);
-                float qf[16];
-                const int ch = c16 >> 2, u0 = 2 * (c16 & 3);
-                const uint32_t o0 = unit_off<D>(ch, u0, r), o1 = unit_off<D>(ch, u0 + 1, r);
-                unpack8(*reinterpret_cast<const uint4*>(qt + o0), qf);
-                unpack8(*reinterpret_cast<const uint4*>(qt + o1), qf + 8);
+            {
+                float ub[2][16];
+                tmem_ld_32x32b_x16(tbase + lanes + 16 * c_lo, ub[0]);
                 tmem_wait_ld();
-                float dqv[16], w[16], zc[16];
+                reg_fence16(ub[0]);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p = valid ? phi_elu1(qf[e]) : 0.f;
-                    const float dphi = fmaf(u[e], rden, ecoef * zs[16 * c16 + e]);
-                    dqv[e] = dphi * (qf[e] > 0.f ? 1.f : p);
-                    w[e] = p * rden;
-                    zc[e] = ecoef * p;
+                for (int i = 0; i < NC; ++i) {
+                    const int c16 = c_lo + i;
+                    if (i + 1 < NC) tmem_ld_32x32b_x16(tbase + lanes + 16 * (c16 + 1), ub[(i + 1) & 1]);
+                    float qf[16];
+                    const int ch = c16 >> 2, u0 = 2 * (c16 & 3);
+                    const uint32_t o0 = unit_off(ch, u0, r), o1 = unit_off(ch, u0 + 1, r);
+                    unpack8(*reinterpret_cast<const uint4*>(qt + o0), qf);
+                    unpack8(*reinterpret_cast<const uint4*>(qt + o1), qf + 8);
+                    float dqv[16], w[16], zc[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p = valid ? phi_elu1(qf[e]) : 0.f;
+                        const float dphi = fmaf(ub[i & 1][e], rden, ecoef * zs[16 * c16 + e]);
+                        dqv[e] = dphi * (qf[e] > 0.f ? 1.f : p);
+                        w[e] = p * rden;
+                        zc[e] = ecoef * p;
+                    }
+                    uint4 h0, l0, h1, l1;
+                    split8(w, h0, l0);
+                    split8(w + 8, h1, l1);
+                    *reinterpret_cast<uint4*>(qt + o0) = h0;
+                    *reinterpret_cast<uint4*>(qt + o1) = h1;
+                    *reinterpret_cast<uint4*>(lot + o0) = l0;
+                    *reinterpret_cast<uint4*>(lot + o1) = l1;
+                    if (valid) {
+                        store8(dqrow + 16 * c16, dqv, accumulate != 0);
+                        store8(dqrow + 16 * c16 + 8, dqv + 8, accumulate != 0);
+                    }
+                    dzacc[i] += warp_reduce_scatter16(zc, lane);
+                    if (i + 1 < NC) { tmem_wait_ld(); reg_fence16(ub[(i + 1) & 1]); }
                 }
-                uint4 h0, l0, h1, l1;
-                split8(w, h0, l0);
-                split8(w + 8, h1, l1);
-                *reinterpret_cast<uint4*>(qt + o0) = h0;
-                *reinterpret_cast<uint4*>(qt + o1) = h1;
-                *reinterpret_cast<uint4*>(lot + o0) = l0;
-                *reinterpret_cast<uint4*>(lot + o1) = l1;
-                if (valid) {
-                    store8(dqrow + 16 * c16, dqv, accumulate != 0);
-                    store8(dqrow + 16 * c16 + 8, dqv + 8, accumulate != 0);
-                }
-                dzacc[c16 - hf * HC] += warp_reduce_scatter16(zc, lane);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -399,11 +440,11 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                 // dz of the segment: lane 2j holds feature 16 c + j of each chunk c
                 if ((lane & 1) == 0) {
 #pragma unroll
-                    for (int c = 0; c < HC; ++c)
-                        atomicAdd(dz + (long long)x.bh * D + 16 * (hf * HC + c) + (lane >> 1), dzacc[c]);
+                    for (int c = 0; c < NC; ++c)
+                        atomicAdd(dz + (long long)x.bh * D + 16 * (c_lo + c) + (lane >> 1), dzacc[c]);
                 }
 #pragma unroll
-                for (int c = 0; c < HC; ++c) dzacc[c] = 0.f;
+                for (int c = 0; c < NC; ++c) dzacc[c] = 0.f;
                 // dS of the segment: M = 128 puts feature a in lane a; M = 64
                 // puts it in lane (a % 16) + 32 (a / 16)
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars->seg_done, seg & 1, abort_flag))) { ok = false; break; }
@@ -412,7 +453,7 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
                 const bool mine = D == 128 || lane < 16;
                 float* Sb = dS + ((long long)x.bh * D + a) * D;
 #pragma unroll 1
-                for (int c0 = hf * D / 2; c0 < (hf + 1) * D / 2; c0 += 16) {
+                for (int c0 = part * C::FC; c0 < (part + 1) * C::FC; c0 += 16) {
                     float vals[16];
                     tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + c0, vals);
                     tmem_wait_ld();
@@ -435,20 +476,20 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
 // --------------------------------------------------------------- key side
 // X = K (overwritten in place by phi(k) hi), Y = V.
 template <int D>
-__global__ void __launch_bounds__(LbCfg<D>::THREADS, 1)
+__global__ void __launch_bounds__(LbCfg<D, kKeyG>::THREADS, 1)
 linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       const Grid g, const int steps_per_head, const long long total_steps,
                       const int steps_per_cta, const uint8_t* __restrict__ image,
                       __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                       const int accumulate, int* status) {
-    using C = LbCfg<D>;
+    using C = LbCfg<D, kKeyG>;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {
         if (threadIdx.x == 0) report(status, kStatusMisaligned);
         return;
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    LbBars* bars = lb_setup<D>(smem, warp);
+    LbBars* bars = lb_setup<D, kKeyG>(smem, warp);
     volatile int* abort_flag = &bars->abort;
     const uint32_t tbase = bars->tmem_base;
     const long long gs0 = (long long)blockIdx.x * steps_per_cta;
@@ -463,9 +504,9 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             const uint32_t lo = smem_u32(smem + C::LO_OFF);
             bool ok = true;
             int issued = 0, seg = 0;
-            lb_load_image<D>(smem, bars, image, lb_step(gs0, 0, n_steps, steps_per_head).bh);
+            lb_load_image<D, kKeyG>(smem, bars, image, lb_step(gs0, 0, n_steps, steps_per_head).bh);
             for (int t = 0; t < min(2, n_steps); ++t) {
-                lb_load_step<D>(smem, bars, &mk, &mv, g, lb_step(gs0, t, n_steps, steps_per_head), t);
+                lb_load_step<D, kKeyG>(smem, bars, &mk, &mv, g, lb_step(gs0, t, n_steps, steps_per_head), t);
                 ++issued;
             }
             for (int t = 0; t < n_steps; ++t) {
@@ -473,9 +514,9 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
                 if (t > 0) {
                     // epilogue(t-1) is done with TMEM, its K buffer, LO and the image
                     if (!mbar_wait_spin(&bars->ready, (t - 1) & 1, abort_flag)) { ok = false; break; }
-                    if (x.first) { ++seg; lb_load_image<D>(smem, bars, image, x.bh); }
+                    if (x.first) { ++seg; lb_load_image<D, kKeyG>(smem, bars, image, x.bh); }
                     if (t + 1 < n_steps) {
-                        lb_load_step<D>(smem, bars, &mk, &mv, g, lb_step(gs0, t + 1, n_steps, steps_per_head), (t + 1) & 1);
+                        lb_load_step<D, kKeyG>(smem, bars, &mk, &mv, g, lb_step(gs0, t + 1, n_steps, steps_per_head), (t + 1) & 1);
                         ++issued;
                     }
                 }
@@ -512,11 +553,14 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             wait_noabort(&bars->mma_idle, 0);
         }
     } else {
-        // warps w and w + 4: tokens 32 (w % 4) + lane, feature halves
-        constexpr int HC = D / 32;
-        const int sp = warp & 3, hf = warp >> 2;
+        // G threads per token: warps w, w + 4, ... take tokens 32 (w % 4) +
+        // lane and split the features (NU 16-byte units, NC 16-feature chunks
+        // each); no value crosses warps
+        constexpr int NC = C::NC, NU = D / 8 / kKeyG;
+        const int sp = warp & 3, part = warp >> 2;
         const int r = 32 * sp + lane;
         const uint32_t lanes = (uint32_t)(32 * sp) << 16;
+        const int c_lo = part * NC;
         const float* dzs = reinterpret_cast<const float*>(smem + C::IMG_OFF + 4 * D * D);
         bool ok = true;
         int seg = -1;
@@ -530,9 +574,10 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             uint8_t* lot = smem + C::LO_OFF;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->full[b], (t >> 1) & 1, abort_flag))) { ok = false; break; }
             // phi(K) hi in place, lo beside it; zero past the end of the grid
-#pragma unroll 1
-            for (int u = hf * D / 16; u < (hf + 1) * D / 16; ++u) {
-                const uint32_t o = unit_off<D>(u >> 3, u & 7, r);
+#pragma unroll
+            for (int i = 0; i < NU; ++i) {
+                const int u = part * NU + i;
+                const uint32_t o = unit_off(u >> 3, u & 7, r);
                 float f[8];
                 unpack8(*reinterpret_cast<const uint4*>(kt + o), f);
 #pragma unroll
@@ -552,29 +597,42 @@ linear_bwd_key_kernel(const __grid_constant__ CUtensorMap mk, const __grid_const
             tc_fence_after();
             __nv_bfloat16* dkrow = dk + (((long long)bb * g.N + n) * g.heads + head) * D;
             __nv_bfloat16* dvrow = dv + (((long long)bb * g.N + n) * g.heads + head) * D;
-#pragma unroll 1
-            for (int c16 = hf * HC; c16 < (hf + 1) * HC; ++c16) {
-                float u[16], w[16];
-                tmem_ld_32x32b_x16(tbase + lanes + 16 * c16, u);
-                tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + 16 * c16, w);
+            // the TMEM reads of chunk i + 1 overlap the arithmetic of chunk i
+            float ub[2][16], wb[2][16];
+            tmem_ld_32x32b_x16(tbase + lanes + 16 * c_lo, ub[0]);
+            tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + 16 * c_lo, wb[0]);
+            tmem_wait_ld();
+            reg_fence16(ub[0]);
+            reg_fence16(wb[0]);
+#pragma unroll
+            for (int i = 0; i < NC; ++i) {
+                const int c16 = c_lo + i;
+                if (i + 1 < NC) {
+                    tmem_ld_32x32b_x16(tbase + lanes + 16 * (c16 + 1), ub[(i + 1) & 1]);
+                    tmem_ld_32x32b_x16(tbase + lanes + C::ACC2 + 16 * (c16 + 1), wb[(i + 1) & 1]);
+                }
                 const int ch = c16 >> 2, u0 = 2 * (c16 & 3);
                 float ph[16], pl[16];
-                unpack8(*reinterpret_cast<const uint4*>(kt + unit_off<D>(ch, u0, r)), ph);
-                unpack8(*reinterpret_cast<const uint4*>(kt + unit_off<D>(ch, u0 + 1, r)), ph + 8);
-                unpack8(*reinterpret_cast<const uint4*>(lot + unit_off<D>(ch, u0, r)), pl);
-                unpack8(*reinterpret_cast<const uint4*>(lot + unit_off<D>(ch, u0 + 1, r)), pl + 8);
-                tmem_wait_ld();
+                unpack8(*reinterpret_cast<const uint4*>(kt + unit_off(ch, u0, r)), ph);
+                unpack8(*reinterpret_cast<const uint4*>(kt + unit_off(ch, u0 + 1, r)), ph + 8);
+                unpack8(*reinterpret_cast<const uint4*>(lot + unit_off(ch, u0, r)), pl);
+                unpack8(*reinterpret_cast<const uint4*>(lot + unit_off(ch, u0 + 1, r)), pl + 8);
                 float dkv[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     // phi'(k) = 1 for k > 0 (phi > 1) and phi(k) = e^k otherwise
-                    dkv[e] = (u[e] + dzs[16 * c16 + e]) * fminf(ph[e] + pl[e], 1.f);
+                    dkv[e] = (ub[i & 1][e] + dzs[16 * c16 + e]) * fminf(ph[e] + pl[e], 1.f);
                 }
                 if (valid) {
                     store8(dkrow + 16 * c16, dkv, accumulate != 0);
                     store8(dkrow + 16 * c16 + 8, dkv + 8, accumulate != 0);
-                    store8(dvrow + 16 * c16, w, accumulate != 0);
-                    store8(dvrow + 16 * c16 + 8, w + 8, accumulate != 0);
+                    store8(dvrow + 16 * c16, wb[i & 1], accumulate != 0);
+                    store8(dvrow + 16 * c16 + 8, wb[i & 1] + 8, accumulate != 0);
+                }
+                if (i + 1 < NC) {
+                    tmem_wait_ld();
+                    reg_fence16(ub[(i + 1) & 1]);
+                    reg_fence16(wb[(i + 1) & 1]);
                 }
             }
             tc_fence_before();
@@ -599,15 +657,17 @@ static cudaError_t launch_linear_bwd_impl(const Grid& g, const void* q, const vo
                                           void* dk, void* dv, int accumulate, uint8_t* scratch,
                                           int* status, cudaStream_t stream,
                                           PFN_cuTensorMapEncodeTiled_v12000 enc) {
-    using C = LbCfg<D>;
+    using CQ = LbCfg<D, kQueryG>;
+    using CK = LbCfg<D, kKeyG>;
+    constexpr int smem_q = CQ::XCH_OFF + CQ::XCH_BYTES, smem_k = CK::XCH_OFF;
     static int configured_device = -1;
     int dev = 0, sms = 148;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(linear_bwd_query_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        e = cudaFuncSetAttribute(linear_bwd_query_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(linear_bwd_key_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        e = cudaFuncSetAttribute(linear_bwd_key_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
@@ -631,14 +691,14 @@ static cudaError_t launch_linear_bwd_impl(const Grid& g, const void* q, const vo
     const long long total = bh * steps_per_head;
     const long long per = (total + sms - 1) / sms;
     const long long ctas = (total + per - 1) / per;
-    linear_bwd_query_kernel<D><<<(unsigned)ctas, C::THREADS, C::SMEM_BYTES, stream>>>(
+    linear_bwd_query_kernel<D><<<(unsigned)ctas, CQ::THREADS, smem_q, stream>>>(
         mq, mg, g, steps_per_head, total, (int)per, img_s, static_cast<__nv_bfloat16*>(dq), accumulate,
         dS, dz, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = launch_linear_pack(g, dS, dz, img_ds, stream);
     if (e != cudaSuccess) return e;
-    linear_bwd_key_kernel<D><<<(unsigned)ctas, C::THREADS, C::SMEM_BYTES, stream>>>(
+    linear_bwd_key_kernel<D><<<(unsigned)ctas, CK::THREADS, smem_k, stream>>>(
         mk, mv, g, steps_per_head, total, (int)per, img_ds, static_cast<__nv_bfloat16*>(dk),
         static_cast<__nv_bfloat16*>(dv), accumulate, status);
     return cudaGetLastError();

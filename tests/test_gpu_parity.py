@@ -561,3 +561,25 @@ def test_linear_backward_workload_two_heads(ops):
     refs = O.linear_bwd(sub(q), sub(k), sub(v), sub(dout), w.B, 2, w.head_dim, w.N)
     for got, ref, name in zip((dq, dk, dv), refs, ("dq", "dk", "dv")):
         check_lin_grad(to_f64(got[:, :, hs]), ref, name)
+
+
+def test_training_gradients_both_branches_batch_of_two(ops):
+    """B = 2: the gradient of out = sparse + linear, formed as a training step
+    forms it (sparse backward, then the linear backward accumulated into the
+    same buffers), against the sum of the two oracle gradients."""
+    T, H, W, heads, d, topk = 5, 6, 7, 2, 128, 3
+    c = Small(T, H, W, heads, d, topk, seed=61, amplitude=0.7, B=2)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    dout = make_dout(c.q.shape, seed=8)
+    out, lse, dq, dk, dv = run_fwd_bwd(ops, c, qd, kd, vd, idx, ws, dout)
+    S = torch.empty((2, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((2, heads, d), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
+    ops.vsa_linear_branch_bwd(qd, kd, vd, dout.cuda(), S, z, dq, dk, dv, T, H, W, ws, accumulate=True)
+    assert ops.vsa_device_status(ws) == 0
+    idx_np = idx.cpu().numpy()
+    rs = O.fine_bwd(c.q, c.k, c.v, dout, idx_np, 2, heads, d, T, H, W, c.tile)
+    rl = O.linear_bwd(c.q, c.k, c.v, dout, 2, heads, d, T * H * W)
+    for got, a, b, name in zip((dq, dk, dv), rs, rl, ("dq", "dk", "dv")):
+        check_grad(to_f64(got), a + b, name)
