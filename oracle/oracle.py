@@ -163,6 +163,74 @@ def fine_tiles(q, k, v, idx, rows, B, heads, d, T, H, W, tile=(4, 4, 4),
     return out
 
 
+def e4m3_encode(x) -> np.ndarray:
+    """float32 values -> FP8 E4M3 codes (uint8): nearest, ties to even,
+    magnitudes above 448 saturated."""
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().oracle_e4m3_encode(_ptr(x), _c_i64(x.size), _ptr(out))
+    return out
+
+
+def e4m3_decode(codes, precision="f64") -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    out = np.empty(codes.shape, _real(precision))
+    lib(precision).oracle_e4m3_decode(_ptr(codes), _c_i64(codes.size), _ptr(out))
+    return out
+
+
+def quant_e4m3_cubes(x, B, heads, d, T, H, W, tile=(4, 4, 4)):
+    """Per-(b, head, cube) E4M3 quantisation of a bf16 tensor [B, N, heads, d]:
+    (codes uint8 [B, N, heads, d], scales float32 [B, heads, nt])."""
+    xb = bits(x)
+    nt = num_tiles(T, H, W, tile)
+    codes = np.zeros((B, T * H * W, heads, d), np.uint8)
+    scales = np.empty((B, heads, nt), np.float32)
+    lib().oracle_quant_e4m3_cubes(_ptr(xb), _c_int(B), _c_int(heads), _c_int(d),
+                                  *_grid_args(T, H, W, tile), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def dequant_e4m3_cubes(codes, scales, T, H, W, tile=(4, 4, 4)) -> np.ndarray:
+    """codes x their cube's scale, fp64, [B, N, heads, d]."""
+    slots = tile_slots(T, H, W, tile)
+    cube_of = np.empty(T * H * W, np.int64)
+    for j, row in enumerate(slots):
+        cube_of[row[row >= 0]] = j
+    sc = scales.astype(np.float64)[:, :, cube_of]                 # [B, heads, N]
+    return e4m3_decode(codes) * sc.transpose(0, 2, 1)[..., None]
+
+
+def fine_tiles_real(qh, kh, v, idx, rows, B, heads, d, T, H, W, tile=(4, 4, 4)) -> np.ndarray:
+    """fine_tiles with real-valued q, k ([B, N, heads, d] fp64) and bf16 v."""
+    qh = np.ascontiguousarray(qh, np.float64)
+    kh = np.ascontiguousarray(kh, np.float64)
+    vb = bits(v)
+    idx = np.ascontiguousarray(idx, np.int32)
+    rows = np.ascontiguousarray(rows, np.int64)
+    vol = tile[0] * tile[1] * tile[2]
+    out = np.zeros((len(rows), vol, d), np.float64)
+    lib().oracle_fine_tiles_real(_ptr(qh), _ptr(kh), _ptr(vb), _ptr(idx), _c_int(B), _c_int(heads),
+                                 _c_int(d), *_grid_args(T, H, W, tile), _c_int(idx.shape[-1]),
+                                 _ptr(rows), _c_i64(len(rows)), _ptr(out))
+    return out
+
+
+def fine_real(qh, kh, v, idx, B, heads, d, T, H, W, tile=(4, 4, 4)) -> np.ndarray:
+    """Fine pass with real-valued q, k over every query tile, grid order."""
+    nt = num_tiles(T, H, W, tile)
+    rows = np.arange(B * heads * nt, dtype=np.int64)
+    part = fine_tiles_real(qh, kh, v, idx, rows, B, heads, d, T, H, W, tile)
+    slots = tile_slots(T, H, W, tile)
+    out = np.zeros((B, T * H * W, heads, d), np.float64)
+    for r in range(len(rows)):
+        bh, i = divmod(r, nt)
+        b, hd = divmod(bh, heads)
+        ok = slots[i] >= 0
+        out[b, slots[i][ok], hd] = part[r][ok]
+    return out
+
+
 def weights(q, k, idx, b, head, n, B, heads, d, T, H, W, tile=(4, 4, 4)) -> np.ndarray:
     qb, kb = bits(q), bits(k)
     idx = np.ascontiguousarray(idx, np.int32)

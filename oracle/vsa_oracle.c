@@ -358,6 +358,143 @@ void oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
     }
 }
 
+/* ------------------------------------------- low-precision fine pass (NEXT)
+ * The low-precision variant quantises q and k to FP8 E4M3 before Q K^T, one
+ * scale per (b, head, cube) ("sparse is orthogonal to low-bit tensor cores":
+ * TurboDiffusion article, section "稀疏、蒸馏与全链路量化", SageSLA built on
+ * SageAttention's quantised products).  E4M3 as the OCP 8-bit floating-point
+ * format defines it ("fn" flavour, no infinities): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits; normal values 1.m x 2^(e-7) for e = 1..15
+ * except e = 15, m = 7 (NaN), so the largest is 1.75 x 2^8 = 448; subnormals
+ * m x 2^-9 (e = 0).  Rounding: to nearest, ties to even; magnitudes above 448
+ * saturate to 448.  Reading made here: scale = amax / 448 in fp32 over the
+ * cube's valid tokens and all d features (1 for an all-zero cube), code =
+ * E4M3(x / scale) with the division in fp32. */
+uint8_t oracle_e4m3_encode_one(float x)
+{
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a > 448.0) return sign | 0x7E;
+    if (a < 0.015625) {                       /* below 2^-6: quantum 2^-9 */
+        double m = nearbyint(a * 512.0);      /* 8 carries into 2^-6 = code 8 */
+        return sign | (uint8_t)m;
+    }
+    int e2;
+    frexp(a, &e2);                            /* a = f 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;                           /* 2^E <= a < 2^(E+1) */
+    double m = nearbyint(a / ldexp(1.0, E - 3));   /* 8 .. 16 */
+    if (m == 16.0) { m = 8.0; E += 1; }
+    return sign | (uint8_t)(((E + 7) << 3) | ((int)m - 8));
+}
+
+REAL oracle_e4m3_decode_one(uint8_t c)
+{
+    int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    REAL v = e == 0 ? (REAL)ldexp((double)m, -9) : (REAL)ldexp((double)(8 + m), e - 10);
+    return (c & 0x80) ? -v : v;
+}
+
+void oracle_e4m3_encode(const float *x, int64_t n, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode_one(x[i]);
+}
+
+void oracle_e4m3_decode(const uint8_t *codes, int64_t n, REAL *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_decode_one(codes[i]);
+}
+
+/* Per-cube quantisation of x [B][N][heads][d] (bf16 bits): codes in the same
+ * layout (valid tokens only), scales [B][heads][nt]. */
+void oracle_quant_e4m3_cubes(const uint16_t *x, int B, int heads, int d, int T, int H, int W,
+                             int tt, int th, int tw, uint8_t *codes, float *scales)
+{
+    grid_t g = make_grid(T, H, W, tt, th, tw);
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int hd = 0; hd < heads; ++hd)
+            for (int j = 0; j < g.nt; ++j) {
+                float amax = 0.0f;
+                for (int s = 0; s < g.vol; ++s) {
+                    int64_t n = slot_token(&g, j, s);
+                    if (n < 0) continue;
+                    const uint16_t *xr = row_ptr(x, g.N, heads, d, b, n, hd);
+                    for (int c = 0; c < d; ++c) {
+                        float v = fabsf((float)bf16_to_real(xr[c]));
+                        if (v > amax) amax = v;
+                    }
+                }
+                volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+                scales[((int64_t)b * heads + hd) * g.nt + j] = scale;
+                for (int s = 0; s < g.vol; ++s) {
+                    int64_t n = slot_token(&g, j, s);
+                    if (n < 0) continue;
+                    const uint16_t *xr = row_ptr(x, g.N, heads, d, b, n, hd);
+                    uint8_t *cr = codes + (((int64_t)b * g.N + n) * heads + hd) * d;
+                    for (int c = 0; c < d; ++c) {
+                        volatile float y = (float)bf16_to_real(xr[c]) / scale;
+                        cr[c] = oracle_e4m3_encode_one(y);
+                    }
+                }
+            }
+}
+
+/* Fine pass (as oracle_fine_tiles) with real-valued q and k [B][N][heads][d]
+ * (e.g. the dequantised codes times their cube scales) and bf16 v. */
+void oracle_fine_tiles_real(const REAL *q, const REAL *kk, const uint16_t *v,
+                            const int32_t *idx, int B, int heads, int d,
+                            int T, int H, int W, int tt, int th, int tw, int k,
+                            const int64_t *rows, int64_t nrows, REAL *out_rows)
+{
+    grid_t g = make_grid(T, H, W, tt, th, tw);
+    (void)B;
+    REAL inv_sqrt_d = (REAL)1 / ORACLE_SQRT((REAL)d);
+#pragma omp parallel
+    {
+        int64_t *tok = (int64_t *)malloc(sizeof(int64_t) * (size_t)k * g.vol);
+        REAL *sb = (REAL *)malloc(sizeof(REAL) * (size_t)k * g.vol);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t row = rows[r];
+            int i = (int)(row % g.nt);
+            int bh = (int)(row / g.nt);
+            int b = bh / heads, hd = bh % heads;
+            const int32_t *sel = idx + row * k;
+            REAL *out = out_rows + r * g.vol * d;
+            int nk = 0;
+            for (int m = 0; m < k; ++m)
+                for (int s = 0; s < g.vol; ++s) {
+                    int64_t n = slot_token(&g, sel[m], s);
+                    if (n >= 0) tok[nk++] = n;
+                }
+            for (int s = 0; s < g.vol; ++s) {
+                REAL *o = out + (int64_t)s * d;
+                for (int c = 0; c < d; ++c) o[c] = 0;
+                int64_t nq = slot_token(&g, i, s);
+                if (nq < 0) continue;
+                const REAL *qr = q + (((int64_t)b * g.N + nq) * heads + hd) * d;
+                REAL mx = -INFINITY;
+                for (int m = 0; m < nk; ++m) {
+                    const REAL *kr = kk + (((int64_t)b * g.N + tok[m]) * heads + hd) * d;
+                    REAL acc = 0;
+                    for (int c = 0; c < d; ++c) acc += qr[c] * kr[c];
+                    sb[m] = acc * inv_sqrt_d;
+                    if (sb[m] > mx) mx = sb[m];
+                }
+                REAL sum = 0;
+                for (int m = 0; m < nk; ++m) { sb[m] = ORACLE_EXP(sb[m] - mx); sum += sb[m]; }
+                for (int m = 0; m < nk; ++m) {
+                    const uint16_t *vr = row_ptr(v, g.N, heads, d, b, tok[m], hd);
+                    REAL p = sb[m] / sum;
+                    for (int c = 0; c < d; ++c) o[c] += p * bf16_to_real(vr[c]);
+                }
+            }
+        }
+        free(tok); free(sb);
+    }
+}
+
 /* Attention weights of one query (b, head, token n) over ALL N keys in grid
  * order: zero outside the selected tiles.  Used to check that each row sums
  * to one and vanishes off the selection. */

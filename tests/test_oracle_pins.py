@@ -402,3 +402,95 @@ def test_linear_bwd_constant_keys_closed_form(oracle_mod):
     np.testing.assert_allclose(dq, 0, atol=1e-12)
     ref = dout.to(torch.float64).sum(1, keepdim=True).numpy() / N
     np.testing.assert_allclose(dv, np.broadcast_to(ref, dv.shape), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------- low-precision (E4M3) fine pass
+
+def _torch_e4m3(x: np.ndarray) -> np.ndarray:
+    """torch's own float32 -> float8_e4m3fn conversion (in-range values)."""
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.float8_e4m3fn) \
+        .view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_matches_torch_and_the_format(oracle_mod):
+    """P11: every finite code decodes as torch's float8_e4m3fn does, and the
+    format's landmarks hold: 1 = 0x38, 2^-9 = 0x01 (least subnormal), 2^-6 =
+    0x08 (least normal), 448 = 0x7E (largest), 0x7F / 0xFF are NaN."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle_mod.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    finite = ~np.isin(codes, [0x7F, 0xFF])
+    np.testing.assert_array_equal(got[finite], ref[finite])
+    assert np.isnan(got[~finite]).all()
+    assert got[0x38] == 1.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+    assert got[0x7E] == 448.0 and got[0xFE] == -448.0
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates(oracle_mod):
+    """P11: encoding equals torch's conversion on random magnitudes over the
+    whole range and on every exact midpoint between neighbouring codes (ties
+    to even); magnitudes above 448 saturate to the largest finite value."""
+    rng = np.random.default_rng(3)
+    mags = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(448.0), 20000))
+    x = (mags * rng.choice([-1.0, 1.0], mags.size)).astype(np.float32)
+    vals = oracle_mod.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))       # 0 .. 448
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    for arr in (x, mids, -mids):
+        np.testing.assert_array_equal(oracle_mod.e4m3_encode(arr), _torch_e4m3(arr))
+    big = np.array([448.5, 464.0, 480.0, 1e4, -1e6], np.float32)
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(big), [0x7E, 0x7E, 0x7E, 0x7E, 0xFE])
+
+
+@pytest.mark.parametrize("case", [(5, 6, 7, (4, 4, 4), 2, 16), (3, 5, 9, (2, 2, 2), 2, 8)])
+def test_cube_quantisation_matches_torch(oracle_mod, case):
+    """P11: per-cube scale = amax / 448 (fp32) and codes = E4M3(x / scale)
+    equal the same steps done with torch (max, float32 division,
+    float8_e4m3fn); every nonzero cube reaches the largest code."""
+    T, H, W, tile, heads, d = case
+    q, _, _ = _inputs(T, H, W, tile, heads, d, seed=5, amplitude=0.7)
+    codes, scales = oracle_mod.quant_e4m3_cubes(q, 1, heads, d, T, H, W, tile)
+    slots = oracle_mod.tile_slots(T, H, W, tile)
+    qf = q.float()
+    for j, row in enumerate(slots):
+        toks = torch.as_tensor(row[row >= 0])
+        for h in range(heads):
+            blk = qf[0, toks, h]
+            sc = (blk.abs().max() / torch.tensor(448.0)).to(torch.float32)
+            assert scales[0, h, j] == sc.item()
+            ref = _torch_e4m3((blk / sc).numpy())
+            np.testing.assert_array_equal(codes[0, row[row >= 0], h], ref)
+            assert np.abs(oracle_mod.e4m3_decode(codes[0, row[row >= 0], h])).max() == 448.0
+
+
+def test_fine_real_equals_fine_on_exactly_representable_inputs(oracle_mod):
+    """P11: when every q, k value is an E4M3 value times a power of two and
+    each cube holds a +-448 multiple, quantisation is lossless, so the fine
+    pass on the dequantised q, k equals the pinned bf16 fine pass."""
+    T, H, W, tile, heads, d, k = 5, 6, 7, (4, 4, 4), 2, 16, 3
+    rng = np.random.default_rng(11)
+    vals = oracle_mod.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    N = T * H * W
+    slots = oracle_mod.tile_slots(T, H, W, tile)
+
+    def exact_tensor(seed_shift):
+        x = rng.choice(vals, size=(1, N, heads, d)) * rng.choice([-1.0, 1.0], size=(1, N, heads, d))
+        for j, row in enumerate(slots):
+            for h in range(heads):
+                s = 2.0 ** int(rng.integers(-8, -3))
+                x[0, row[row >= 0], h] *= s
+                x[0, row[row >= 0][0], h, 0] = 448.0 * s             # the cube maximum
+        return torch.from_numpy(x).to(torch.bfloat16)
+
+    q, kk = exact_tensor(0), exact_tensor(1)
+    _, _, v = _inputs(T, H, W, tile, heads, d, seed=2)
+    assert torch.equal(q.double().to(torch.bfloat16), q)            # bf16-exact by construction
+    idx = oracle_mod.select(q, kk, 1, heads, d, T, H, W, k, tile)
+    cq, sq = oracle_mod.quant_e4m3_cubes(q, 1, heads, d, T, H, W, tile)
+    ck, sk = oracle_mod.quant_e4m3_cubes(kk, 1, heads, d, T, H, W, tile)
+    qh = oracle_mod.dequant_e4m3_cubes(cq, sq, T, H, W, tile)
+    kh = oracle_mod.dequant_e4m3_cubes(ck, sk, T, H, W, tile)
+    np.testing.assert_array_equal(qh, q.double().numpy())
+    np.testing.assert_array_equal(kh, kk.double().numpy())
+    got = oracle_mod.fine_real(qh, kh, v, idx, 1, heads, d, T, H, W, tile)
+    ref = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
