@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "fine_attn.h"
 #include "linear.h"
+#include "quant.h"
 #include "select.h"
 #include "tiles.h"
 #include "fine_bwd.h"
@@ -68,6 +69,21 @@ bool encode_grid_map(CUtensorMap* m, const void* base, const vsa::Grid& g) {
     cuuint32_t box[5] = {64, (cuuint32_t)g.tw, (cuuint32_t)g.th, (cuuint32_t)g.tt, 1};
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same 5-D view over E4M3 codes (one byte per element): box {128 codes
+// (= 128 bytes, the whole d of a head at d = 128), tw, th, tt, 1}.
+bool encode_grid_map_u8(CUtensorMap* m, const void* base, const vsa::Grid& g) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t row = (cuuint64_t)g.heads * g.d;
+    cuuint64_t dims[5] = {row, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T, (cuuint64_t)g.B};
+    cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
+    cuuint32_t box[5] = {128, (cuuint32_t)g.tw, (cuuint32_t)g.th, (cuuint32_t)g.tt, 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -203,6 +219,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     a.out = out;
     a.out32 = nullptr;
     a.lse = nullptr;
+    a.q_scale = a.k_scale = nullptr;
     a.status = static_cast<int*>(workspace);
     if (lin_S) {
         // the bf16 hi/lo operand image of (S, z) goes into the workspace scratch
@@ -242,6 +259,7 @@ vsa_status vsa_sparse_attn_fwd_train(const vsa_bf16* q, const vsa_bf16* k, const
     a.out = out;
     a.out32 = out_f32;
     a.lse = lse;
+    a.q_scale = a.k_scale = nullptr;
     a.status = static_cast<int*>(workspace);
     return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
 }
@@ -304,6 +322,54 @@ vsa_status vsa_linear_branch_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa
     return from_cuda(vsa::launch_linear_bwd(g, q, k, v, dout, lin_S, lin_z, dq, dk, dv, accumulate,
                                             static_cast<uint8_t*>(workspace) + kStatusBytes,
                                             static_cast<int*>(workspace), (cudaStream_t)stream, fn));
+}
+
+vsa_status vsa_quantize_qk_e4m3(const vsa_bf16* q, const vsa_bf16* k, uint8_t* q8, uint8_t* k8,
+                                float* q_scale, float* k_scale, int B, int heads, int head_dim,
+                                int T, int H, int W, int tt, int th, int tw, vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (s != VSA_OK) return s;
+    for (const void* p : {(const void*)q, (const void*)k, (const void*)q8, (const void*)k8,
+                          (const void*)q_scale, (const void*)k_scale})
+        if (!aligned16(p)) return VSA_ERR_INVALID_ARGUMENT;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
+    return from_cuda(vsa::launch_quant_e4m3(g, q, k, q8, k8, q_scale, k_scale, (cudaStream_t)stream));
+}
+
+vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
+                                    const float* k_scale, const vsa_bf16* v,
+                                    const int32_t* block_idx, vsa_bf16* out, int B, int heads,
+                                    int head_dim, int T, int H, int W, int tt, int th, int tw,
+                                    int topk, void* workspace, size_t workspace_bytes,
+                                    vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (s != VSA_OK) return s;
+    if (head_dim != 128) return VSA_ERR_UNSUPPORTED;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
+    for (const void* p : {(const void*)q8, (const void*)k8, (const void*)q_scale, (const void*)k_scale,
+                          (const void*)v, (const void*)block_idx, (const void*)out})
+        if (!aligned16(p)) return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes) return VSA_ERR_WORKSPACE;
+    CUtensorMap mq, mk, mv;
+    if (!encode_grid_map_u8(&mq, q8, g) || !encode_grid_map_u8(&mk, k8, g) || !encode_grid_map(&mv, v, g))
+        return VSA_ERR_CUDA;
+    vsa::FineArgs a;
+    a.g = g;
+    a.mq = &mq;
+    a.mk = &mk;
+    a.mv = &mv;
+    a.block_idx = block_idx;
+    a.topk = topk;
+    a.lin_image = nullptr;
+    a.out = out;
+    a.out32 = nullptr;
+    a.lse = nullptr;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.status = static_cast<int*>(workspace);
+    return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
 }
 
 vsa_status vsa_device_status(void* workspace, vsa_stream_t stream) {

@@ -44,15 +44,22 @@
 namespace vsa {
 using namespace sm100;
 
-template <int D>
+// Q8: the low-precision variant (q and k as E4M3 codes, one byte each).
+template <int D, bool Q8 = false>
 struct FineCfg {
-    static constexpr int NCH = D / 64;                 // 64-element (128-byte) d chunks
-    static constexpr int Q_BYTES = 64 * D * 2;         // one query cube
-    static constexpr int CUBE_BYTES = 64 * D * 2;      // one key cube (K or V)
-    static constexpr int PAIR_BYTES = 2 * CUBE_BYTES;  // two key cubes
+    static constexpr int QB = Q8 ? 1 : 2;              // bytes per q / k element
+    static constexpr int NCH = D / 64;                 // 128-byte d chunks of V
+    static constexpr int NCH_QK = D * QB / 128;        // 128-byte d chunks of Q and K
+    static constexpr int Q_BYTES = 64 * D * QB;        // one query cube
+    static constexpr int K_CUBE_BYTES = 64 * D * QB;   // one key cube of K
+    static constexpr int V_CUBE_BYTES = 64 * D * 2;    // one key cube of V
+    static constexpr int K_PAIR_BYTES = 2 * K_CUBE_BYTES;
+    static constexpr int V_PAIR_BYTES = 2 * V_CUBE_BYTES;
     static constexpr int CHUNK_STRIDE = 128 * 128;     // bytes between d chunks of a pair
     static constexpr int NK = (D == 128) ? 2 : 3;      // K pair stages
-    static constexpr int NV = (D == 128) ? 1 : 3;      // V pair stages
+    // the smaller K and Q of the low-precision variant leave room for a
+    // second V stage within two CTAs per SM
+    static constexpr int NV = Q8 ? 2 : ((D == 128) ? 1 : 3);   // V pair stages
     static constexpr int TMEM_COLS = 256;
     // A ring slot is free once the MMAs reading it are done.  With two K stages
     // the stage of pair p is the S buffer p & 1, so the K producer can wait on
@@ -66,16 +73,16 @@ struct FineCfg {
     static constexpr int S_COL = 128;                  // fp32 S (128 cols) / bf16 P (64 cols)
     static constexpr int BAR_BYTES = 256;
     static constexpr int Z_BYTES = D * 4;              // linear branch: z (fp32)
-    static constexpr int SMEM_BYTES = Q_BYTES + (NK + NV) * PAIR_BYTES + BAR_BYTES + Z_BYTES;
+    static constexpr int SMEM_BYTES = Q_BYTES + NK * K_PAIR_BYTES + NV * V_PAIR_BYTES + BAR_BYTES + Z_BYTES;
     // the linear branch's S hi + lo image must fit the K ring, phi(Q) lo the V ring
-    static_assert(4 * D * D <= NK * PAIR_BYTES && Q_BYTES <= NV * PAIR_BYTES, "linear operands");
+    static_assert(Q8 || (4 * D * D <= NK * K_PAIR_BYTES && Q_BYTES <= NV * V_PAIR_BYTES), "linear operands");
 };
 
-template <int D>
+template <int D, bool Q8 = false>
 struct FineBars {
     uint64_t q_full;
-    uint64_t k_full[FineCfg<D>::NK], k_empty[FineCfg<D>::NK];
-    uint64_t v_full[FineCfg<D>::NV], v_empty[FineCfg<D>::NV];
+    uint64_t k_full[FineCfg<D, Q8>::NK], k_empty[FineCfg<D, Q8>::NK];
+    uint64_t v_full[FineCfg<D, Q8>::NV], v_empty[FineCfg<D, Q8>::NV];
     uint64_t s_full[2], p_full[2], o_ready[2];   // per S / O buffer (pair parity)
     uint64_t mma_done, lin_full, lin_ready, lin_done;
     uint32_t tmem_base;
@@ -83,16 +90,20 @@ struct FineBars {
 };
 static_assert(sizeof(FineBars<128>) <= FineCfg<128>::BAR_BYTES, "barrier block");
 static_assert(sizeof(FineBars<64>) <= FineCfg<64>::BAR_BYTES, "barrier block");
+static_assert(sizeof(FineBars<128, true>) <= FineCfg<128, true>::BAR_BYTES, "barrier block");
+static_assert(FineCfg<128, true>::SMEM_BYTES <= 232448 / 2 - 1024, "two CTAs per SM");
 
-template <int D, bool LIN>
+template <int D, bool LIN, bool Q8>
 __global__ void __launch_bounds__(224, 2)
 fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                  const __grid_constant__ CUtensorMap mv, const Grid g,
                  const int32_t* __restrict__ block_idx, const int topk, const float scale_log2,
                  const int ragged, const uint8_t* __restrict__ lin_image,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ out32, float* __restrict__ lse,
+                 const float* __restrict__ q_scale, const float* __restrict__ k_scale,
                  int* status) {
-    using C = FineCfg<D>;
+    using C = FineCfg<D, Q8>;
+    static_assert(!(Q8 && LIN), "the low-precision variant has no linear branch");
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
         if (threadIdx.x == 0) report(status, kStatusMisaligned);
@@ -100,8 +111,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     }
     uint8_t* sQ = smem;
     uint8_t* sK = smem + C::Q_BYTES;
-    uint8_t* sV = sK + C::NK * C::PAIR_BYTES;
-    FineBars<D>* bars = reinterpret_cast<FineBars<D>*>(sV + C::NV * C::PAIR_BYTES);
+    uint8_t* sV = sK + C::NK * C::K_PAIR_BYTES;
+    FineBars<D, Q8>* bars = reinterpret_cast<FineBars<D, Q8>*>(sV + C::NV * C::V_PAIR_BYTES);
     volatile int* abort_flag = &bars->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -121,7 +132,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     uint8_t* sPhiLo = sV;
     uint8_t* sSHi = sK;
     uint8_t* sSLo = sK + D * D * 2;
-    float* sZ = reinterpret_cast<float*>(sV + C::NV * C::PAIR_BYTES + C::BAR_BYTES);
+    float* sZ = reinterpret_cast<float*>(sV + C::NV * C::V_PAIR_BYTES + C::BAR_BYTES);
 
     if (tid == 0) {
         bars->abort = 0;
@@ -160,8 +171,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             if (is_k) {
                 const TileCoord qc = tile_coord(g, i);
                 mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-                for (int c = 0; c < C::NCH; ++c)
-                    tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + 64 * c, qc.w0, qc.h0, qc.t0, b);
+                for (int c = 0; c < C::NCH_QK; ++c)
+                    tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + (128 / C::QB) * c, qc.w0, qc.h0, qc.t0, b);
             }
             const int nst = is_k ? C::NK : C::NV;
             uint64_t* full = is_k ? bars->k_full : bars->v_full;
@@ -186,12 +197,16 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     if (!is_k && C::V_ON_O) { bar = &bars->o_ready[(p - 1) & 1]; par = ((p - 1) >> 1) & 1; }
                     if (!mbar_wait(bar, par, abort_flag)) { fail(); break; }
                 }
-                mbar_arrive_expect_tx(&full[st], ntl * C::CUBE_BYTES);
+                // K: NCH_QK chunks of 128 / QB elements; V: NCH chunks of 64
+                const int nch = is_k ? C::NCH_QK : C::NCH;
+                const int cw = is_k ? 128 / C::QB : 64;
+                const int pair_bytes = is_k ? C::K_PAIR_BYTES : C::V_PAIR_BYTES;
+                mbar_arrive_expect_tx(&full[st], ntl * (is_k ? C::K_CUBE_BYTES : C::V_CUBE_BYTES));
                 for (int t = 0; t < ntl; ++t) {
                     const TileCoord kc = tile_coord(g, jt[t]);
-                    for (int c = 0; c < C::NCH; ++c)
-                        tma_load_5d(ring + st * C::PAIR_BYTES + c * C::CHUNK_STRIDE + t * 8192, map,
-                                    &full[st], head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
+                    for (int c = 0; c < nch; ++c)
+                        tma_load_5d(ring + st * pair_bytes + c * C::CHUNK_STRIDE + t * 8192, map,
+                                    &full[st], head * D + cw * c, kc.w0, kc.h0, kc.t0, b);
                 }
                 ++issued;
             }
@@ -237,12 +252,23 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 const int sk = p % C::NK;
                 if (!mbar_wait(&bars->k_full[sk], (p / C::NK) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
+                if constexpr (Q8) {
+                    // E4M3 codes: K = 32 per MMA, one 128-byte row per token
+                    const uint32_t id_s = idesc_e4m3_f32(64, nkeys, false, false);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(k_addr + sk * C::PAIR_BYTES + (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32, 16, 1024);
-                    mma_bf16_ss(tS(p & 1), a, bd, id_s, kk > 0);
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t a = smem_desc_sw128(q_addr + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(k_addr + sk * C::K_PAIR_BYTES + kk * 32, 16, 1024);
+                        mma_e4m3_ss(tS(p & 1), a, bd, id_s, kk > 0);
+                    }
+                } else {
+                    const uint32_t id_s = idesc_bf16_f32(64, nkeys, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(k_addr + sk * C::K_PAIR_BYTES + (kk >> 2) * C::CHUNK_STRIDE + (kk & 3) * 32, 16, 1024);
+                        mma_bf16_ss(tS(p & 1), a, bd, id_s, kk > 0);
+                    }
                 }
                 mma_commit(&bars->s_full[p & 1]);
                 if (!C::K_ON_S) mma_commit(&bars->k_empty[sk]);
@@ -257,7 +283,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 if (!mbar_wait(&bars->v_full[sv], (p / C::NV) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int kk = 0; kk < nkeys / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(v_addr + sv * C::PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
+                    const uint64_t bd = smem_desc_sw128(v_addr + sv * C::V_PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
                     mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
                 }
                 mma_commit(&bars->o_ready[x]);
@@ -300,13 +326,18 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         auto tO = [&](int x) { return lane_base + C::O_COL + ((uint32_t)x << 20); };
         SoftmaxState sm{-INFINITY, 0.f};
         bool ok = true;
+        // low-precision variant: raw scores are in units of the query cube's
+        // scale times the key cube's scale
+        const float sq_row = Q8 ? __ldg(q_scale + row_id) : 1.f;
         for (int p = 0; p < n_pairs; ++p) {
             const int ntl = min(2, topk - 2 * p);
             uint64_t vmask = hf < ntl ? ~0ull : 0ull;   // odd tail: this half has no cube
-            if (ragged && hf < ntl) {                   // edge cubes: mask padded keys
+            float sc = scale_log2;
+            if ((ragged || Q8) && hf < ntl) {
                 int j = __ldg(my_idx + 2 * p + hf);
                 if (j < 0 || j >= g.nt) j = 0;
-                vmask = valid_slot_mask(g, tile_coord(g, j));
+                if (ragged) vmask = valid_slot_mask(g, tile_coord(g, j));   // edge cubes: mask padded keys
+                if (Q8) sc = scale_log2 * sq_row * __ldg(k_scale + (long long)bh * g.nt + j);
             }
             const int x = p & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x], (p >> 1) & 1, abort_flag))) { ok = false; break; }
@@ -320,8 +351,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             uint32_t pk[32];
             bool resc;
             const bool masked = __any_sync(0xffffffffu, vmask != ~0ull);
-            const float alpha = masked ? softmax_step<true>(s, vmask, scale_log2, sm, resc, pk)
-                                       : softmax_step<false>(s, vmask, scale_log2, sm, resc, pk);
+            const float alpha = masked ? softmax_step<true>(s, vmask, sc, sm, resc, pk)
+                                       : softmax_step<false>(s, vmask, sc, sm, resc, pk);
             tmem_st_16x32bx2_x32(tS(x), pk);
             if (p > 0 && __any_sync(0xffffffffu, resc)) {
                 // the two O buffers hold PV up to pair p-1 (the completion of
@@ -453,15 +484,15 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-template <int D, bool LIN>
+template <int D, bool LIN, bool Q8 = false>
 static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
-    using C = FineCfg<D>;
+    using C = FineCfg<D, Q8>;
     static int configured_device = -1;   // per process: attribute set once per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_device != dev) {
-        e = cudaFuncSetAttribute(fine_attn_kernel<D, LIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(fine_attn_kernel<D, LIN, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured_device = dev;
@@ -469,13 +500,15 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     const long long rows = (long long)a.g.B * a.g.heads * a.g.nt;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (a.g.T % a.g.tt) || (a.g.H % a.g.th) || (a.g.W % a.g.tw);
-    fine_attn_kernel<D, LIN><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
+    fine_attn_kernel<D, LIN, Q8><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
         *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged,
-        static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.out32, a.lse, a.status);
+        static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.out32, a.lse,
+        a.q_scale, a.k_scale, a.status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
+    if (a.q_scale) return launch_fine_impl<128, false, true>(a, stream);   // E4M3 q, k (d = 128)
     const bool lin = a.lin_image != nullptr;
     if (a.g.d == 128) return lin ? launch_fine_impl<128, true>(a, stream) : launch_fine_impl<128, false>(a, stream);
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);

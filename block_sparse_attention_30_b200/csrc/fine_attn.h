@@ -21,6 +21,8 @@ struct FineArgs {
     float* out32;                // optional fp32 copy of out (for the backward pass)
     float* lse;                  // optional [B][heads][nt][64]: log2 softmax normaliser
                                  // of the scaled scores per cube slot (+inf if padded)
+    const float* q_scale;        // low-precision variant: E4M3 q, k with one scale
+    const float* k_scale;        // per (b, head, cube) [B][heads][nt]; null for bf16
     int* status;                 // device status word
 };
 

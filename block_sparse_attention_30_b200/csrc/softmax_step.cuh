@@ -27,7 +27,8 @@ struct SoftmaxState {
     float l_run;    // this half's running sum of weights
 };
 
-// s: this thread's 64 raw scores (q.k); vmask: valid keys (bit e = key e),
+// s: this thread's 64 raw scores (q.k); scale_log2: this thread's factor from
+// a raw score to the exp2 domain; vmask: valid keys (bit e = key e),
 // consulted only when `masked`.  Writes the 32 packed bf16x2 weights to pk
 // and returns the factor by which O must be rescaled (1 if unchanged) and
 // whether any rescale happened for this row.
@@ -48,8 +49,11 @@ __device__ __forceinline__ float softmax_step(float (&s)[64], uint64_t vmask, fl
         m2 = max3f(m2, s[e + 4], s[e + 5]);
         m3 = max3f(m3, s[e + 6], s[e + 7]);
     }
-    float mx = fmaxf(max3f(m0, m1, m2), m3);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * scale_log2;
+    // each half scales its own maximum (the two halves may hold key cubes
+    // with different scales); for a common positive scale this equals scaling
+    // the maximum of both, as rounding is monotonic
+    float mx = fmaxf(max3f(m0, m1, m2), m3) * scale_log2;
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     rescaled = mx > st.m_run + 8.f;
     const float m_new = rescaled ? mx : st.m_run;
     const float alpha = rescaled ? ex2(st.m_run - m_new) : 1.f;

@@ -130,6 +130,25 @@ def vsa_linear_branch_bwd(q, k, v, dout, lin_S, lin_z, dq, dk, dv, T, H, W, work
         heads, d, T, H, W, workspace.data_ptr(), workspace.numel(), _stream(stream)))
 
 
+def vsa_quantize_qk_e4m3(q, k, q8, k8, q_scale, k_scale, T, H, W, tile=(4, 4, 4), stream=None):
+    """Per-cube E4M3 codes (uint8, q's layout) and fp32 scales [B, heads, nt]
+    of q and k, written in place."""
+    B, heads, d = _grid_of(q, T, H, W)
+    _lib.check("vsa_quantize_qk_e4m3", _lib.lib().vsa_quantize_qk_e4m3(
+        q.data_ptr(), k.data_ptr(), q8.data_ptr(), k8.data_ptr(), q_scale.data_ptr(),
+        k_scale.data_ptr(), *_shape(B, heads, d, T, H, W, tile), _stream(stream)))
+
+
+def vsa_sparse_attn_fwd_e4m3(q8, k8, q_scale, k_scale, v, block_idx, out, T, H, W, topk, workspace,
+                             tile=(4, 4, 4), stream=None):
+    """Fine pass with Q K^T in E4M3 (codes and scales from vsa_quantize_qk_e4m3)."""
+    B, heads, d = _grid_of(v, T, H, W)
+    _lib.check("vsa_sparse_attn_fwd_e4m3", _lib.lib().vsa_sparse_attn_fwd_e4m3(
+        q8.data_ptr(), k8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(), v.data_ptr(),
+        block_idx.data_ptr(), out.data_ptr(), *_shape(B, heads, d, T, H, W, tile), topk,
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
 def vsa_device_status(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = VSA_OK)."""
     return _lib.lib().vsa_device_status(workspace.data_ptr(), _stream(stream))

@@ -203,6 +203,31 @@ vsa_status vsa_linear_branch_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa
                                  int heads, int head_dim, int T, int H, int W, void* workspace,
                                  size_t workspace_bytes, vsa_stream_t stream);
 
+/* Low-precision fine pass (sparse attention is orthogonal to low-bit tensor
+ * cores: TurboDiffusion article, section "稀疏、蒸馏与全链路量化", SageSLA).
+ * Step 1, vsa_quantize_qk_e4m3: per (b, head, cube) scale = amax / 448 (fp32,
+ * over the cube's valid tokens and all d features; 1 for an all-zero cube)
+ * and codes = FP8 E4M3 of x / scale (fp32 division, nearest-even, saturating
+ * at 448), for q and k.  q8, k8: [B][N][heads][d] codes, one byte each (only
+ * valid tokens are written); q_scale, k_scale: fp32 [B][heads][nt].  All
+ * device pointers 16-byte aligned; no workspace. */
+vsa_status vsa_quantize_qk_e4m3(const vsa_bf16* q, const vsa_bf16* k, uint8_t* q8, uint8_t* k8,
+                                float* q_scale, float* k_scale, int B, int heads, int head_dim,
+                                int T, int H, int W, int tt, int th, int tw, vsa_stream_t stream);
+
+/* Step 2, vsa_sparse_attn_fwd_e4m3: the fine pass of vsa_sparse_attn_fwd with
+ * Q K^T on the tensor cores in E4M3 (fp32 accumulation), scores rescaled by
+ * q_scale[query cube] * k_scale[key cube], softmax and P V as in the bf16
+ * pass (bf16 P and v), output bf16 in grid order.  head_dim 128 only
+ * (VSA_ERR_UNSUPPORTED otherwise); no linear branch.  Needs
+ * vsa_workspace_bytes() of workspace (status word only). */
+vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
+                                    const float* k_scale, const vsa_bf16* v,
+                                    const int32_t* block_idx, vsa_bf16* out, int B, int heads,
+                                    int head_dim, int T, int H, int W, int tt, int th, int tw,
+                                    int topk, void* workspace, size_t workspace_bytes,
+                                    vsa_stream_t stream);
+
 /* Self-test of the device failure path (no counterpart on the pages): a
  * one-warp kernel waits on a barrier nobody arrives at, gives up after
  * `limit_cycles` SM clock cycles exactly as the library's kernels do, and

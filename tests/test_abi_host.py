@@ -120,6 +120,14 @@ def test_other_entry_points_validate(L):
     assert lb(*[FAKE] * 8, FAKE + 8, 0, 1, 2, 128, 4, 8, 8, FAKE, ok_ws, None) == INVALID   # misaligned dv
     assert lb(*[FAKE] * 9, 0, 1, 2, 96, 4, 8, 8, FAKE, ok_ws, None) == UNSUPPORTED
     assert lb(*[FAKE] * 9, 0, 0, 2, 128, 4, 8, 8, FAKE, ok_ws, None) == INVALID
+    qz = L.vsa_quantize_qk_e4m3
+    assert qz(*[FAKE] * 6, 1, 2, 96, 4, 8, 8, 4, 4, 4, None) == UNSUPPORTED
+    assert qz(FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, 1, 2, 128, 4, 8, 8, 4, 4, 4, None) == INVALID
+    fe = L.vsa_sparse_attn_fwd_e4m3
+    assert fe(*[FAKE] * 7, 1, 2, 64, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == UNSUPPORTED   # d = 64
+    assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 5, FAKE, 1024, None) == INVALID     # topk > nt
+    assert fe(*[FAKE] * 6, FAKE + 2, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == INVALID
+    assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 8, None) == WORKSPACE
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID
