@@ -6,15 +6,16 @@
 // cores (SageSLA, built on SageAttention's quantised attention products).
 // Reading: one fp32 scale per (b, head, cube) = amax / 448 over the cube's
 // valid tokens and all d features (1 for an all-zero cube), codes =
-// E4M3(x / scale) rounded to nearest-even with saturation at 448 (the largest
-// finite E4M3 value), the division in IEEE fp32.  Codes keep the
-// [B][N][heads][d] layout (one byte per element) so the fine kernel's 5-D
-// TMA boxes cut cubes out of them exactly as out of the bf16 tensors.
+// E4M3(x * inv) with inv = 1 / scale, both rounded to nearest fp32, the
+// conversion rounded to nearest-even with saturation at 448 (the largest
+// finite E4M3 value).  Codes keep the [B][N][heads][d] layout (one byte per
+// element) so the fine kernel's 5-D TMA boxes cut cubes out of them exactly
+// as out of the bf16 tensors.
 //
-// One CTA per (cube, batch, group of 4 heads, q|k), 256 threads: each thread
-// holds its 16-byte vectors of the cube's tokens in registers, so the data is
-// read once; the cube maximum of each head is reduced over the threads that
-// share the head (shuffles, then shared memory across token groups).
+// One warp per (q|k, b, cube, head); consecutive warps take consecutive heads
+// of a cube, so a CTA reads contiguous spans of each token row.  The warp
+// streams the cube twice: once for the maximum (a warp reduction), once to
+// convert; the second pass is served by L2.
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -22,15 +23,6 @@
 #include "quant.h"
 
 namespace vsa {
-
-template <int D>
-struct QuantCfg {
-    static constexpr int HG = 4;                       // heads per CTA
-    static constexpr int VPT = D / 8;                  // 16-byte vectors per (token, head)
-    static constexpr int VPR = HG * VPT;               // vectors per token row of the group
-    static constexpr int TG = 256 / VPR;               // token groups
-    static constexpr int TPT = 64 / TG;                // tokens per thread
-};
 
 // 8 floats -> 8 E4M3 codes (nearest-even, saturating), packed little-endian.
 __device__ __forceinline__ uint2 to_e4m3x8(const float (&y)[8]) {
@@ -46,83 +38,87 @@ __device__ __forceinline__ uint2 to_e4m3x8(const float (&y)[8]) {
     return make_uint2(w[0], w[1]);
 }
 
+// Token of cube slot s (the cube's origin c), with a shift-only path for the
+// 4 x 4 x 4 tile.
+__device__ __forceinline__ long long slot_token(const Grid& g, const TileCoord& c, int s, bool t444) {
+    int dt, dh, dw;
+    if (t444) { dt = s >> 4; dh = (s >> 2) & 3; dw = s & 3; }
+    else { dt = s / (g.th * g.tw); dh = (s / g.tw) % g.th; dw = s % g.tw; }
+    return ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256)
 quant_e4m3_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g,
                   uint8_t* __restrict__ q8, uint8_t* __restrict__ k8, float* __restrict__ q_scale,
-                  float* __restrict__ k_scale) {
-    using C = QuantCfg<D>;
-    __shared__ float part[C::TG][C::HG];
-    const int j = blockIdx.x;
-    const int hgroups = (g.heads + C::HG - 1) / C::HG;
-    const int b = blockIdx.y / hgroups, h0 = (blockIdx.y % hgroups) * C::HG;
-    const bool is_k = blockIdx.z != 0;
+                  float* __restrict__ k_scale, const long long n_warps) {
+    constexpr int VPT = D / 8;                         // 16-byte vectors per (token, head)
+    constexpr int TPL = 32 / VPT;                      // tokens per warp-wide load
+    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= n_warps) return;                        // whole warps only
+    const int lane = threadIdx.x & 31;
+    const int head = (int)(wid % g.heads);
+    long long r = wid / g.heads;
+    const int j = (int)(r % g.nt);
+    r /= g.nt;
+    const int b = (int)(r % g.B);
+    const bool is_k = r / g.B != 0;
     const uint16_t* x = is_k ? k : q;
     uint8_t* x8 = is_k ? k8 : q8;
     float* scales = is_k ? k_scale : q_scale;
-    const int tid = threadIdx.x;
-    const int v = tid % C::VPR, tg = tid / C::VPR;     // vector of the row, token group
-    const int hl = v / C::VPT, head = h0 + hl;         // head of this vector
-    const bool head_ok = head < g.heads;
     const TileCoord c = tile_coord(g, j);
     const uint64_t valid = valid_slot_mask(g, c);
+    const bool t444 = g.tt == 4 && g.th == 4 && g.tw == 4;
+    const int vec = lane % VPT, tsub = lane / VPT;
 
-    uint4 raw[C::TPT];
     float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < C::TPT; ++i) {
-        const int s = tg + C::TG * i;                  // cube slot
-        raw[i] = make_uint4(0, 0, 0, 0);
-        if (head_ok && ((valid >> s) & 1ull)) {
-            const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
-            const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
-            raw[i] = __ldg(reinterpret_cast<const uint4*>(x + ((b * g.N + n) * g.heads + head) * D) +
-                           (v % C::VPT));
-        }
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll 4
+    for (int i = 0; i < 64 / TPL; ++i) {
+        const int s = i * TPL + tsub;
+        if (!((valid >> s) & 1ull)) continue;
+        const long long n = slot_token(g, c, s, t444);
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + ((b * g.N + n) * g.heads + head) * D) + vec);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
                                      fabsf(__uint_as_float(w[e] & 0xffff0000u))));
     }
-    // the VPT threads of a (token group, head) are consecutive lanes
 #pragma unroll
-    for (int o = C::VPT / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (v % C::VPT == 0) part[tg][hl] = amax;
-    __syncthreads();
-    float m = 0.f;
-#pragma unroll
-    for (int t = 0; t < C::TG; ++t) m = fmaxf(m, part[t][hl]);
-    const float scale = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-    if (head_ok && tg == 0 && v % C::VPT == 0) scales[((long long)b * g.heads + head) * g.nt + j] = scale;
-#pragma unroll
-    for (int i = 0; i < C::TPT; ++i) {
-        const int s = tg + C::TG * i;
-        if (!head_ok || !((valid >> s) & 1ull)) continue;
-        const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
-        const long long n = ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float inv = __frcp_rn(scale);
+    if (lane == 0) scales[((long long)b * g.heads + head) * g.nt + j] = scale;
+#pragma unroll 4
+    for (int i = 0; i < 64 / TPL; ++i) {
+        const int s = i * TPL + tsub;
+        if (!((valid >> s) & 1ull)) continue;
+        const long long n = slot_token(g, c, s, t444);
+        const long long row = (b * g.N + n) * g.heads + head;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + row * D) + vec);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
         float y[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            y[2 * e] = __fdiv_rn(__uint_as_float(w[e] << 16), scale);
-            y[2 * e + 1] = __fdiv_rn(__uint_as_float(w[e] & 0xffff0000u), scale);
+            y[2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), inv);
+            y[2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xffff0000u), inv);
         }
-        reinterpret_cast<uint2*>(x8 + ((b * g.N + n) * g.heads + head) * D)[v % C::VPT] = to_e4m3x8(y);
+        reinterpret_cast<uint2*>(x8 + row * D)[vec] = to_e4m3x8(y);
     }
 }
 
 cudaError_t launch_quant_e4m3(const Grid& g, const void* q, const void* k, void* q8, void* k8,
                               float* q_scale, float* k_scale, cudaStream_t stream) {
-    const dim3 grid((unsigned)g.nt, (unsigned)(g.B * ((g.heads + 3) / 4)), 2);
+    const long long n_warps = 2ll * g.B * g.nt * g.heads;
+    const unsigned ctas = (unsigned)((n_warps + 7) / 8);
     if (g.d == 128)
-        quant_e4m3_kernel<128><<<grid, 256, 0, stream>>>(
+        quant_e4m3_kernel<128><<<ctas, 256, 0, stream>>>(
             static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), g,
-            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale);
+            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, n_warps);
     else
-        quant_e4m3_kernel<64><<<grid, 256, 0, stream>>>(
+        quant_e4m3_kernel<64><<<ctas, 256, 0, stream>>>(
             static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), g,
-            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale);
+            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, n_warps);
     return cudaGetLastError();
 }
 

@@ -207,8 +207,8 @@ vsa_status vsa_linear_branch_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa
  * cores: TurboDiffusion article, section "稀疏、蒸馏与全链路量化", SageSLA).
  * Step 1, vsa_quantize_qk_e4m3: per (b, head, cube) scale = amax / 448 (fp32,
  * over the cube's valid tokens and all d features; 1 for an all-zero cube)
- * and codes = FP8 E4M3 of x / scale (fp32 division, nearest-even, saturating
- * at 448), for q and k.  q8, k8: [B][N][heads][d] codes, one byte each (only
+ * and codes = FP8 E4M3 of x * (1 / scale) (reciprocal and product rounded to
+ * nearest fp32; conversion nearest-even, saturating at 448), for q and k.  q8, k8: [B][N][heads][d] codes, one byte each (only
  * valid tokens are written); q_scale, k_scale: fp32 [B][heads][nt].  All
  * device pointers 16-byte aligned; no workspace. */
 vsa_status vsa_quantize_qk_e4m3(const vsa_bf16* q, const vsa_bf16* k, uint8_t* q8, uint8_t* k8,

@@ -369,7 +369,8 @@ void oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
  * m x 2^-9 (e = 0).  Rounding: to nearest, ties to even; magnitudes above 448
  * saturate to 448.  Reading made here: scale = amax / 448 in fp32 over the
  * cube's valid tokens and all d features (1 for an all-zero cube), code =
- * E4M3(x / scale) with the division in fp32. */
+ * E4M3(x * inv) with inv = 1 / scale, both rounded to nearest fp32 (the
+ * dequantised value is code * scale). */
 uint8_t oracle_e4m3_encode_one(float x)
 {
     uint8_t sign = signbit(x) ? 0x80 : 0;
@@ -426,6 +427,7 @@ void oracle_quant_e4m3_cubes(const uint16_t *x, int B, int heads, int d, int T, 
                     }
                 }
                 volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+                volatile float inv = 1.0f / scale;
                 scales[((int64_t)b * heads + hd) * g.nt + j] = scale;
                 for (int s = 0; s < g.vol; ++s) {
                     int64_t n = slot_token(&g, j, s);
@@ -433,7 +435,7 @@ void oracle_quant_e4m3_cubes(const uint16_t *x, int B, int heads, int d, int T, 
                     const uint16_t *xr = row_ptr(x, g.N, heads, d, b, n, hd);
                     uint8_t *cr = codes + (((int64_t)b * g.N + n) * heads + hd) * d;
                     for (int c = 0; c < d; ++c) {
-                        volatile float y = (float)bf16_to_real(xr[c]) / scale;
+                        volatile float y = (float)bf16_to_real(xr[c]) * inv;
                         cr[c] = oracle_e4m3_encode_one(y);
                     }
                 }

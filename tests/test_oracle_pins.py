@@ -443,9 +443,9 @@ def test_e4m3_encode_rounds_to_nearest_even_and_saturates(oracle_mod):
 
 @pytest.mark.parametrize("case", [(5, 6, 7, (4, 4, 4), 2, 16), (3, 5, 9, (2, 2, 2), 2, 8)])
 def test_cube_quantisation_matches_torch(oracle_mod, case):
-    """P11: per-cube scale = amax / 448 (fp32) and codes = E4M3(x / scale)
-    equal the same steps done with torch (max, float32 division,
-    float8_e4m3fn); every nonzero cube reaches the largest code."""
+    """P11: per-cube scale = amax / 448 (fp32) and codes = E4M3(x * (1 /
+    scale)) equal the same steps done with torch (max, float32 reciprocal and
+    product, float8_e4m3fn); every nonzero cube reaches the largest code."""
     T, H, W, tile, heads, d = case
     q, _, _ = _inputs(T, H, W, tile, heads, d, seed=5, amplitude=0.7)
     codes, scales = oracle_mod.quant_e4m3_cubes(q, 1, heads, d, T, H, W, tile)
@@ -457,7 +457,8 @@ def test_cube_quantisation_matches_torch(oracle_mod, case):
             blk = qf[0, toks, h]
             sc = (blk.abs().max() / torch.tensor(448.0)).to(torch.float32)
             assert scales[0, h, j] == sc.item()
-            ref = _torch_e4m3((blk / sc).numpy())
+            inv = (torch.tensor(1.0, dtype=torch.float32) / sc).to(torch.float32)
+            ref = _torch_e4m3((blk * inv).numpy())
             np.testing.assert_array_equal(codes[0, row[row >= 0], h], ref)
             assert np.abs(oracle_mod.e4m3_decode(codes[0, row[row >= 0], h])).max() == 448.0
 
