@@ -12,11 +12,10 @@
 // element) so the fine kernel's 5-D TMA boxes cut cubes out of them exactly
 // as out of the bf16 tensors.
 //
-// One CTA per (q|k, b, cube) (and chunk of heads when there are many), each
-// warp a pair of heads (d = 128) or four (d = 64): a warp-wide load is one
-// token's consecutive head rows, so the CTA reads whole token rows.  Each
-// warp streams the cube twice: once for the per-head maximum (lane
-// reductions), once to convert; the second pass is served from L1.
+// Each CTA holds its part of a cube in registers between the maximum and the
+// conversion, so q and k are read from HBM once.  (A version that streamed
+// each cube twice lost the second pass to L2 evictions: with every SM busy
+// the data in flight between the passes exceeds L2.)
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -48,28 +47,38 @@ __device__ __forceinline__ long long slot_token(const Grid& g, const TileCoord& 
     return ((long long)(c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
 }
 
-// One CTA per (q|k, b, cube, chunk of up to 64 heads); warp w of the CTA
-// takes heads 2w and 2w + 1 of the chunk (HPW heads per warp: 32 lanes = HPW
-// heads x VPT 16-byte vectors), so each warp-wide load is HPW consecutive
-// head rows of one token and the CTA reads whole token rows.
+// One CTA per (q|k, b, cube, group of HG heads), 256 threads: thread t holds
+// vector t % 32 of the group's token-row chunk (HG heads x D/8 vectors, 512
+// bytes, contiguous) for 8 of the cube's 64 slots in registers, so the data
+// is read from HBM once and several CTAs fit on an SM.  The cube maximum of a
+// head is reduced over its lanes (shuffles), then over the 8 token groups
+// (shared memory).
 template <int D>
-__global__ void __launch_bounds__(1024)
+struct QuantCfg {
+    static constexpr int VPT = D / 8;                  // 16-byte vectors per (token, head)
+    static constexpr int HG = 32 / VPT;                // heads per CTA (one warp-wide row chunk)
+    static constexpr int TG = 256 / 32;                // token groups (one per warp)
+    static constexpr int TPT = 64 / TG;                // slots per thread
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, 3)
 quant_e4m3_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g,
                   uint8_t* __restrict__ q8, uint8_t* __restrict__ k8, float* __restrict__ q_scale,
-                  float* __restrict__ k_scale, const int head_chunks) {
-    constexpr int VPT = D / 8;                         // 16-byte vectors per (token, head)
-    constexpr int HPW = 32 / VPT;                      // heads per warp
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+                  float* __restrict__ k_scale, const int head_groups) {
+    using C = QuantCfg<D>;
+    __shared__ float part[C::TG][C::HG];
+    const int lane = threadIdx.x & 31, tg = threadIdx.x >> 5;
     long long r = blockIdx.x;
-    const int hc = (int)(r % head_chunks);
-    r /= head_chunks;
+    const int hgi = (int)(r % head_groups);
+    r /= head_groups;
     const int j = (int)(r % g.nt);
     r /= g.nt;
     const int b = (int)(r % g.B);
     const bool is_k = r / g.B != 0;
-    const int head = hc * (32 * HPW) + warp * HPW + lane / VPT;   // 32 warps x HPW heads per chunk
+    const int hl = lane / C::VPT, vec = lane % C::VPT;
+    const int head = hgi * C::HG + hl;
     const bool head_ok = head < g.heads;
-    const int vec = lane % VPT;
     const uint16_t* x = is_k ? k : q;
     uint8_t* x8 = is_k ? k8 : q8;
     float* scales = is_k ? k_scale : q_scale;
@@ -77,13 +86,20 @@ quant_e4m3_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k
     const uint64_t valid = valid_slot_mask(g, c);
     const bool t444 = g.tt == 4 && g.th == 4 && g.tw == 4;
 
+    uint4 raw[C::TPT];
+    int tok[C::TPT];                                   // token of each slot, -1 if not held
     float amax = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < 64; ++s) {
-        if (!head_ok || !((valid >> s) & 1ull)) continue;
-        const long long n = slot_token(g, c, s, t444);
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + ((b * g.N + n) * g.heads + head) * D) + vec);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < C::TPT; ++i) {
+        const int s = tg + C::TG * i;
+        const bool ok = head_ok && ((valid >> s) & 1ull);
+        tok[i] = ok ? (int)slot_token(g, c, s, t444) : -1;
+        raw[i] = ok ? __ldg(reinterpret_cast<const uint4*>(x + ((b * g.N + tok[i]) * g.heads + head) * D) + vec)
+                    : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < C::TPT; ++i) {
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
@@ -91,43 +107,42 @@ quant_e4m3_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k
     }
     // the VPT lanes of a head are consecutive
 #pragma unroll
-    for (int o = VPT / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    for (int o = C::VPT / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (vec == 0) part[tg][hl] = amax;
+    __syncthreads();
+    float m = 0.f;
+#pragma unroll
+    for (int t = 0; t < C::TG; ++t) m = fmaxf(m, part[t][hl]);
+    const float scale = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
     const float inv = __frcp_rn(scale);
-    if (head_ok && vec == 0) scales[((long long)b * g.heads + head) * g.nt + j] = scale;
-#pragma unroll 8
-    for (int s = 0; s < 64; ++s) {
-        if (!head_ok || !((valid >> s) & 1ull)) continue;
-        const long long n = slot_token(g, c, s, t444);
-        const long long row = (b * g.N + n) * g.heads + head;
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + row * D) + vec);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    if (head_ok && tg == 0 && vec == 0) scales[((long long)b * g.heads + head) * g.nt + j] = scale;
+#pragma unroll
+    for (int i = 0; i < C::TPT; ++i) {
+        if (tok[i] < 0) continue;
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
         float y[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             y[2 * e] = __fmul_rn(__uint_as_float(w[e] << 16), inv);
             y[2 * e + 1] = __fmul_rn(__uint_as_float(w[e] & 0xffff0000u), inv);
         }
-        reinterpret_cast<uint2*>(x8 + row * D)[vec] = to_e4m3x8(y);
+        reinterpret_cast<uint2*>(x8 + ((b * g.N + tok[i]) * g.heads + head) * D)[vec] = to_e4m3x8(y);
     }
 }
 
 cudaError_t launch_quant_e4m3(const Grid& g, const void* q, const void* k, void* q8, void* k8,
                               float* q_scale, float* k_scale, cudaStream_t stream) {
-    const int hpw = 32 / (g.d / 8);                            // heads per warp
-    const int per_chunk = 32 * hpw;                            // heads per CTA (at most 32 warps)
-    const int head_chunks = (g.heads + per_chunk - 1) / per_chunk;
-    const int heads_in_cta = g.heads < per_chunk ? g.heads : per_chunk;
-    const int threads = 32 * ((heads_in_cta + hpw - 1) / hpw);
-    const unsigned ctas = (unsigned)(2ll * g.B * g.nt * head_chunks);
+    const int hg = 32 / (g.d / 8);                             // heads per CTA
+    const int head_groups = (g.heads + hg - 1) / hg;
+    const unsigned ctas = (unsigned)(2ll * g.B * g.nt * head_groups);
     if (g.d == 128)
-        quant_e4m3_kernel<128><<<ctas, threads, 0, stream>>>(
+        quant_e4m3_kernel<128><<<ctas, 256, 0, stream>>>(
             static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), g,
-            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, head_chunks);
+            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, head_groups);
     else
-        quant_e4m3_kernel<64><<<ctas, threads, 0, stream>>>(
+        quant_e4m3_kernel<64><<<ctas, 256, 0, stream>>>(
             static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), g,
-            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, head_chunks);
+            static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), q_scale, k_scale, head_groups);
     return cudaGetLastError();
 }
 
