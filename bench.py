@@ -339,20 +339,20 @@ def run_kernels(args):
         return sorted(ts)[len(ts) // 2]
 
     rows = [
-        ("gather_tiles (a1)", lambda: ops.vsa_gather_tiles(q, tiles, w.T, w.H, w.W, w.tile),
+        ("gather_tiles (cube gather)", lambda: ops.vsa_gather_tiles(q, tiles, w.T, w.H, w.W, w.tile),
          "hbm", elem + tile_bytes),
-        ("scatter_tiles (a7)", lambda: ops.vsa_scatter_tiles(tiles, out, w.T, w.H, w.W, w.tile),
+        ("scatter_tiles (cube scatter)", lambda: ops.vsa_scatter_tiles(tiles, out, w.T, w.H, w.W, w.tile),
          "hbm", 2 * elem),
-        ("select_blocks (a2-a4)", lambda: ops.vsa_select_blocks(q, k, w.T, w.H, w.W, w.topk,
+        ("select_blocks (pool, coarse scores, top-k)", lambda: ops.vsa_select_blocks(q, k, w.T, w.H, w.W, w.topk,
                                                                   attn.block_idx, attn.workspace, w.tile),
          "hbm", 2 * elem + w.B * w.heads * nt * w.topk * 4),
-        ("linear_branch_fwd (a6 state)", lambda: ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W,
+        ("linear_branch_fwd (linear state)", lambda: ops.vsa_linear_branch_fwd(k, v, attn.lin_S, attn.lin_z, w.T, w.H, w.W,
                                                                            attn.workspace),
          "hbm", 2 * elem),
-        ("sparse_attn_fwd (a1+a5+a7 fused)", lambda: ops.vsa_sparse_attn_fwd(q, k, v, attn.block_idx, out, w.T, w.H, w.W,
+        ("sparse_attn_fwd (fine pass, gather and scatter fused)", lambda: ops.vsa_sparse_attn_fwd(q, k, v, attn.block_idx, out, w.T, w.H, w.W,
                                                                             w.topk, attn.workspace, tile=w.tile),
          "tensor", w.fine_flops()),
-        ("sparse_attn_fwd + linear apply (a5+a6)", lambda: ops.vsa_sparse_attn_fwd(
+        ("sparse_attn_fwd + linear apply", lambda: ops.vsa_sparse_attn_fwd(
             q, k, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, attn.lin_S, attn.lin_z, w.tile),
          "tensor", w.fine_flops()),
     ]
@@ -374,7 +374,7 @@ def run_kernels(args):
         # linear branch backward: reads q, k, v, dout and writes dq, dk, dv
         # (the d x d states are a few MB); its products are ~10 d^2 FLOPs per
         # token, far below the tensor-core ridge, so HBM bounds it
-        ("linear_branch_bwd (a6 backward)", lambda: ops.vsa_linear_branch_bwd(
+        ("linear_branch_bwd (linear branch backward)", lambda: ops.vsa_linear_branch_bwd(
             q, k, v, g_out, attn.lin_S, attn.lin_z, dq, dk, dv, w.T, w.H, w.W, attn.workspace),
          "hbm", 7 * elem),
     ]

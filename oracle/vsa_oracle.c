@@ -358,7 +358,7 @@ void oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
     }
 }
 
-/* ------------------------------------------- low-precision fine pass (NEXT)
+/* ----------------------------------------------- low-precision fine pass
  * The low-precision variant quantises q and k to FP8 E4M3 before Q K^T, one
  * scale per (b, head, cube) ("sparse is orthogonal to low-bit tensor cores":
  * TurboDiffusion article, section "稀疏、蒸馏与全链路量化", SageSLA built on
