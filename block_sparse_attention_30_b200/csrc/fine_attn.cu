@@ -30,6 +30,12 @@
 // Two CTAs share an SM (256 TMEM columns and ~112 KB of shared memory each),
 // so one CTA's softmax overlaps the other's MMAs.
 //
+// Low-precision variant (Q8, d = 128): q and k arrive as FP8 E4M3 codes with
+// one scale per (b, head, cube) (quant.cu); Q K^T runs as tcgen05
+// kind::f8f6f4 (K = 32 per MMA, one 128-byte row per token), the softmax
+// multiplies each half row by its query and key cube scales, P V stays bf16.
+// The halved Q and K tiles make room for a second V stage.
+//
 // Every wait is bounded; on a timeout the CTA records kStatusTimeout in the
 // status word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
