@@ -689,3 +689,48 @@ def test_e4m3_headline_workload_sampled(ops):
         ref.append(part[r][ok])
         got.append(to_f64(out[0, torch.as_tensor(slots[i][ok]), head]))
     check_close(np.concatenate(got), np.concatenate(ref))
+
+
+# ------------------------------------------------------------ degenerate grids
+
+def test_single_token_grid_closed_forms(ops):
+    """A 1 x 1 x 1 grid: one cube with one valid token.  Softmax over a single
+    key is 1, so out = v exactly; the linear branch reduces to v as well
+    (phi(q) phi(k)^T v / (phi(q) . phi(k))); the sparse gradients are dq = dk
+    = 0 and dv = dO, and the linear ones dq = dk = 0, dv = dO."""
+    T = H = W = 1
+    heads, d, topk = 2, 128, 1
+    c = Small(T, H, W, heads, d, topk, seed=5, amplitude=0.7)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    assert idx.cpu().numpy().ravel().tolist() == [0, 0]
+    out = run_fine(ops, c, qd, kd, vd, idx, ws)
+    assert torch.equal(out, vd)
+    S = torch.empty((1, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((1, heads, d), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
+    out_lin = run_fine(ops, c, qd, kd, vd, idx, ws, lin=(S, z))
+    np.testing.assert_allclose(to_f64(out_lin), 2 * to_f64(vd), rtol=1e-2, atol=0)
+    dout = make_dout(c.q.shape, seed=2)
+    _, _, dq, dk, dv = run_fwd_bwd(ops, c, qd, kd, vd, idx, ws, dout)
+    g = to_f64(dout.cuda())
+    assert np.abs(to_f64(dq)).max() <= 1e-3 * np.abs(g).max()
+    assert np.abs(to_f64(dk)).max() <= 1e-3 * np.abs(g).max()
+    assert torch.equal(dv, dout.cuda())
+    lq, lk, lv = run_linear_bwd(ops, c.q, c.k, c.v, dout, T, H, W)
+    assert np.abs(to_f64(lq)).max() <= 1e-3 * np.abs(g).max()
+    assert np.abs(to_f64(lk)).max() <= 1e-3 * np.abs(g).max()
+    np.testing.assert_allclose(to_f64(lv), g, rtol=1e-2, atol=0)
+
+
+def test_grid_smaller_than_a_cube_is_dense_attention(ops):
+    """A 3 x 2 x 3 grid is one ragged cube of 18 tokens: with k = 1 every query
+    attends every token, i.e. dense attention (torch SDPA, fp64)."""
+    T, H, W, heads, d, topk = 3, 2, 3, 2, 128, 1
+    c = Small(T, H, W, heads, d, topk, seed=8, amplitude=0.7)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    out = run_fine(ops, c, qd, kd, vd, idx, ws)
+    q64, k64, v64 = (x.double().permute(0, 2, 1, 3) for x in (c.q, c.k, c.v))
+    ref = torch.nn.functional.scaled_dot_product_attention(q64, k64, v64).permute(0, 2, 1, 3)
+    check_close(to_f64(out), ref.numpy())
