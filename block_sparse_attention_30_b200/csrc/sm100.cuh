@@ -119,7 +119,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 5-D tiled load (no multicast) of one box into this CTA's shared memory;
+// 5-D tiled load of one box into this CTA's own shared memory;
 // completion is reported on `bar` as transaction bytes.
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, int c3, int c4) {
@@ -131,7 +131,7 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// 3-D tiled load (no multicast) of one box into this CTA's shared memory.
+// 3-D tiled load of one box into this CTA's own shared memory.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
     asm volatile(
@@ -141,7 +141,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// Untiled bulk copy (no multicast) of `bytes` contiguous bytes from global to
+// Untiled bulk copy of `bytes` contiguous bytes from global to
 // this CTA's shared memory; both addresses 16-byte aligned, bytes a multiple
 // of 16.  Completion is reported on `bar` as transaction bytes.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
