@@ -17,9 +17,9 @@
 // Two kernels, each one CTA per SM over 128-token steps of the flattened
 // (b*heads, step) space, with G epilogue threads per token (each owning D/G
 // features; G = 2 on the query side, 4 on the key side) and one TMA + MMA warp:
-//  * query side: U = G S^T on the tensor cores (G = dout is exact in bf16, S
-//    enters as bf16 hi + lo, so u is good to ~2^-17), the per-token terms on
-//    the CUDA cores, then dS += (phi(Q)/den)^T G (phi/den as hi + lo) into a
+//  * query side: U = dO S^T on the tensor cores (dO = dout is exact in bf16,
+//    S enters as bf16 hi + lo, so u is good to ~2^-17), the per-token terms on
+//    the CUDA cores, then dS += (phi(Q)/den)^T dO (phi/den as hi + lo) into a
 //    TMEM accumulator that is added to a global fp32 dS at the end of each
 //    (b, head) segment; dz by warp reductions.
 //  * key side: U' = V dS^T (dS hi + lo) and dV = phi(K) dS (three products:
@@ -222,7 +222,7 @@ __device__ __forceinline__ void lb_load_image(uint8_t* smem, LbBars* bars, const
 }
 
 // ------------------------------------------------------------- query side
-// X = Q (overwritten in place by (phi(q)/den) hi), Y = G = dout.
+// X = Q (overwritten in place by (phi(q)/den) hi), Y = dO (dout).
 template <int D>
 __global__ void __launch_bounds__(LbCfg<D, kQueryG>::THREADS, 1)
 linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mg,
@@ -247,8 +247,8 @@ linear_bwd_query_kernel(const __grid_constant__ CUtensorMap mq, const __grid_con
     if (warp == C::MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             // ------------------------------------------------ loads + MMAs
-            const uint32_t id_u = idesc_bf16_f32(128, D, false, false);   // U = G S^T
-            const uint32_t id_s = idesc_bf16_f32(D, D, true, true);       // dS += W^T G
+            const uint32_t id_u = idesc_bf16_f32(128, D, false, false);   // U = dO S^T
+            const uint32_t id_s = idesc_bf16_f32(D, D, true, true);       // dS += W^T dO
             const uint32_t img = smem_u32(smem + C::IMG_OFF);
             auto mma_u = [&](int t) {
                 const uint32_t ga = smem_u32(smem + (2 * (t & 1) + 1) * C::TILE);
