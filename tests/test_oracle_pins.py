@@ -495,3 +495,38 @@ def test_fine_real_equals_fine_on_exactly_representable_inputs(oracle_mod):
     got = oracle_mod.fine_real(qh, kh, v, idx, 1, heads, d, T, H, W, tile)
     ref = oracle_mod.fine(q, kk, v, idx, 1, heads, d, T, H, W, tile)
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------ property-based pins
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(T=st.integers(1, 9), H=st.integers(1, 9), W=st.integers(1, 9),
+       tile=st.sampled_from([(4, 4, 4), (2, 4, 8), (8, 2, 4), (1, 8, 8), (2, 2, 2)]))
+def test_tile_map_is_a_bijection_for_any_grid(oracle_mod, T, H, W, tile):
+    """P5 (any shape): the tiling map sends every token of the grid to exactly
+    one slot, of the cube the coordinate formula names, and marks exactly the
+    out-of-grid slots as padding."""
+    slots = oracle_mod.tile_slots(T, H, W, tile)
+    cube, nt = twin.cube_of_token(T, H, W, tile)
+    assert slots.shape == (nt, tile[0] * tile[1] * tile[2])
+    valid = slots[slots >= 0]
+    assert np.array_equal(np.sort(valid), np.arange(T * H * W))
+    for j in range(nt):
+        assert np.all(cube[slots[j][slots[j] >= 0]] == j)
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.lists(st.floats(-448.0, 448.0, allow_nan=False, width=32), min_size=1, max_size=64))
+def test_e4m3_rounding_error_and_monotonicity(oracle_mod, xs):
+    """P11 (any value in range): decoding the code of x is within half a step
+    of x (a step is 2^(e-3) for 2^e <= |x| < 2^(e+1), 2^-9 below 2^-6), and
+    encoding preserves order."""
+    x = np.array(xs, np.float32)
+    d = oracle_mod.e4m3_decode(oracle_mod.e4m3_encode(x))
+    a = np.abs(x.astype(np.float64))
+    step = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3))
+    assert np.all(np.abs(d - x) <= step / 2)
+    order = np.argsort(x, kind="stable")
+    assert np.all(np.diff(d[order]) >= 0)
