@@ -530,3 +530,20 @@ def test_e4m3_rounding_error_and_monotonicity(oracle_mod, xs):
     assert np.all(np.abs(d - x) <= step / 2)
     order = np.argsort(x, kind="stable")
     assert np.all(np.diff(d[order]) >= 0)
+
+
+@settings(max_examples=40, deadline=None)
+@given(nt=st.integers(1, 40), k=st.integers(1, 40), levels=st.integers(1, 6), seed=st.integers(0, 2**31 - 1))
+def test_topk_matches_a_sort_with_ties_to_the_lower_id(oracle_mod, nt, k, levels, seed):
+    """P4 (any row, heavy ties): the kept cubes are the first k of the order
+    (score descending, cube id ascending), emitted ascending.  Scores drawn
+    from a few levels force ties."""
+    k = min(k, nt)
+    rng = np.random.default_rng(seed)
+    scores = rng.integers(0, levels, size=(1, 2, nt, nt)).astype(np.float64) / levels
+    got = oracle_mod.topk(scores, k)
+    for h in range(2):
+        for i in range(nt):
+            row = scores[0, h, i]
+            order = np.lexsort((np.arange(nt), -row))
+            assert got[0, h, i].tolist() == sorted(order[:k].tolist())
