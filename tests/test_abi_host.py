@@ -128,6 +128,20 @@ def test_other_entry_points_validate(L):
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 5, FAKE, 1024, None) == INVALID     # topk > nt
     assert fe(*[FAKE] * 6, FAKE + 2, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == INVALID
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 8, None) == WORKSPACE
+    ft = L.vsa_sparse_attn_fwd_train
+    assert ft(*[FAKE] * 7, *SHAPE, 2, None, 1 << 30, None) == WORKSPACE
+    assert ft(*[FAKE] * 5, FAKE + 4, FAKE, *SHAPE, 2, FAKE, 1 << 30, None) == INVALID        # out_f32
+    assert ft(*[FAKE] * 7, *SHAPE, 5, FAKE, 1 << 30, None) == INVALID                        # topk > nt
+    bad = list(SHAPE); bad[2] = 96
+    assert ft(*[FAKE] * 7, *bad, 2, FAKE, 1 << 30, None) == UNSUPPORTED
+    bw = L.vsa_sparse_attn_bwd
+    rows = 1 * 2 * 4                                       # B * heads * nt
+    up = lambda x: -(-x // 256) * 256
+    need = 256 + up(rows * 64 * 4) + up(1 * 2 * (4 + 1) * 4) + up(rows * 2 * 4)
+    assert L.vsa_workspace_bytes(*SHAPE, 2) >= need
+    assert bw(*[FAKE] * 10, *SHAPE, 2, FAKE, need - 16, None) == WORKSPACE
+    assert bw(*[FAKE] * 7, FAKE + 8, FAKE, FAKE, *SHAPE, 2, FAKE, need, None) == INVALID      # dq
+    assert bw(*[FAKE] * 10, *SHAPE, 0, FAKE, need, None) == INVALID                           # topk < 1
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID
