@@ -41,25 +41,31 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-FINE_SOURCES = ["fine_attn.cu", "softmax_step.cuh", "sm100.cuh", "common.cuh"]
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "fine_attn_wan1.3b_480p.md")
+# Sources of the fine kernel the step runs for bf16 d = 128 without the linear
+# branch (the persistent two-cube kernel); a DRAM-traffic figure is reported
+# only while they hash to the value recorded beside it.
+FINE_SOURCES = ["fine_pair.cu", "softmax_step.cuh", "sm100.cuh", "common.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per fine launch from the committed ncu summary, or None when
-    the summary lacks this workload or the kernel sources changed since."""
+def fine_sources_hash():
     import hashlib
-    import re
-    if not os.path.exists(TRAFFIC_PROFILE):
-        return None
-    text = open(TRAFFIC_PROFILE, encoding="utf-8").read()
-    m_hash = re.search(r"^sources_sha256: ([0-9a-f]+)$", text, re.M)
-    m_val = re.search(r"^traffic_bytes_per_launch\[%s\]: (\d+)$" % re.escape(workload), text, re.M)
-    if not m_hash or not m_val:
-        return None
     csrc = os.path.join(ROOT, "block_sparse_attention_30_b200", "csrc")
     h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in FINE_SOURCES))
-    return int(m_val.group(1)) if h.hexdigest()[:16] == m_hash.group(1) else None
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, path=TRAFFIC_FILE):
+    """DRAM bytes (ncu dram__bytes_read.sum + dram__bytes_write.sum) per fine
+    launch from the committed capture data, or None when the data lacks this
+    workload or the kernel sources changed since the capture."""
+    if not os.path.exists(path):
+        return None
+    data = json.load(open(path, encoding="utf-8"))
+    if data.get("sources_sha256") != fine_sources_hash():
+        return None
+    val = data.get("bytes_per_launch", {}).get(workload)
+    return int(val) if val is not None else None
 
 
 def dist_env():
@@ -147,6 +153,13 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def fine_kernel_name(w):
+    """The fine kernel vsa_sparse_attn_fwd launches for this workload."""
+    if w.head_dim == 128 and not w.linear:
+        return "fine_pair_kernel<128>"
+    return "fine_attn_kernel<%d, %s>" % (w.head_dim, "LIN" if w.linear else "-")
 
 
 def gpu_step_fn(w, q, k, v, out, attn, fine_events):
@@ -276,7 +289,7 @@ def run_gpu(args):
                             "pct_of_bf16_sustained": round(100 * fine_tflops / peaks["bf16_tflops_sustained"], 2)},
             "pct_of_bf16_peak": round(100 * (value / world) / peak, 2),
             "roofline": {
-                "bound": "tensor", "kernel": "fine_attn_kernel<%d>" % w.head_dim,
+                "bound": "tensor", "kernel": fine_kernel_name(w),
                 "achieved": round(fine_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(fine_tflops / peak, 4),
                 "peak_source": f"{src} bf16_tflops (burst)",
@@ -299,6 +312,96 @@ def run_gpu(args):
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def run_sharded(args):
+    """Sequence-sharded forward over N GPUs (strong scaling): every rank holds
+    tokens [r*N/P, (r+1)*N/P) of q, k, v of ONE workload; a step is the
+    seq -> heads all-to-all, select + fine on this rank's heads, and the
+    heads -> seq all-to-all (block_sparse_attention_30_b200.sharded)."""
+    import datetime
+    import torch.distributed as dist
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from block_sparse_attention_30_b200 import build, sharded
+    build.build()
+    w = WORKLOADS[args.workload]
+    q_h, k_h, v_h = synth.make_workload_inputs(w, seed=list(WORKLOADS).index(w.name))
+    Nl = w.N // world
+    sl = slice(rank * Nl, (rank + 1) * Nl)
+    qs, ks, vs = (x[:, sl].contiguous().to(dev) for x in (q_h, k_h, v_h))
+    attn = sharded.SequenceShardedAttention(w.B, w.heads, w.head_dim, w.T, w.H, w.W, w.topk, w.tile,
+                                            linear=w.linear, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        attn(qs, ks, vs)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.fill_(i & 255)
+        starts[i].record()
+        attn(qs, ks, vs)
+        ends[i].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    # end to end: this rank's shard from pinned host memory and its output back
+    qp, kp, vp = (x[:, sl].contiguous().pin_memory() for x in (q_h, k_h, v_h))
+    out_h = torch.empty(qp.shape, dtype=qp.dtype).pin_memory()
+    bufs = [torch.empty_like(qs) for _ in range(3)]
+    e2e_steps = max(2, min(args.steps, 8))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record()
+    for _ in range(e2e_steps):
+        for b, hsrc in zip(bufs, (qp, kp, vp)):
+            b.copy_(hsrc, non_blocking=True)
+        out_h.copy_(attn(*bufs), non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
+    status = attn.attn.status()
+    if rank == 0:
+        flops = w.fine_flops()
+        ms = total_ms / args.steps
+        peaks, src = load_peaks()
+        print(json.dumps({
+            "metric": METRIC, "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) noise + per-cube N(0,1) offsets, Wan latent shapes)",
+            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "head_dim": w.head_dim,
+                       "grid": [w.T, w.H, w.W], "topk": w.topk, "linear_branch": w.linear,
+                       "fine_flops_per_step": flops,
+                       "l2": "256 MiB write between steps (outside the timed events)",
+                       "parallelism": f"sequence-sharded inputs, heads exchanged by all-to-all over {world} GPU(s)"},
+            "comm": {"all_to_all_bytes_sent_per_rank_per_step": sharded.exchange_bytes(
+                w.B, w.N, w.heads, w.head_dim, world), "collectives_per_step": 4 if world > 1 else 0},
+            "pct_of_bf16_peak": round(100 * flops / (ms * 1e-3) / 1e12 / world / peaks["bf16_tflops"], 2),
+            "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
+                    "h2d_bytes_per_step": 3 * qp.numel() * qp.element_size() * world,
+                    "d2h_bytes_per_step": out_h.numel() * out_h.element_size() * world},
+            "gpu_launches": (4 + (2 if w.linear else 0)) * args.steps,
+            "clocks": clk, "device_status": status,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
 
 
 # ------------------------------------------------------------ per-kernel lines
@@ -477,6 +580,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels", action="store_true",
                     help="print one roofline line per hot-path kernel instead of the step line")
+    ap.add_argument("--sharded", action="store_true",
+                    help="sequence-sharded inputs over the ranks, heads exchanged by all-to-all "
+                         "(strong scaling); default: one independent workload per rank")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per fine launch from an ncu capture (reported as-is)")
     args = ap.parse_args()
@@ -493,7 +599,10 @@ def main():
     else:
         if not torch.cuda.is_available():
             sys.exit("bench.py needs a CUDA device for --impl ours")
-        run_gpu(args)
+        if args.sharded:
+            run_sharded(args)
+        else:
+            run_gpu(args)
 
 
 if __name__ == "__main__":

@@ -24,14 +24,11 @@ constexpr size_t kStatusBytes = 256;     // status block at the start of the wor
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 vsa_status check_shape(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
-    if (B < 1 || heads < 1 || d < 1 || T < 1 || H < 1 || W < 1 || tt < 1 || th < 1 || tw < 1)
-        return VSA_ERR_INVALID_ARGUMENT;
-    if (d != 64 && d != 128) return VSA_ERR_UNSUPPORTED;
-    if (tt * th * tw != 64) return VSA_ERR_UNSUPPORTED;
-    // index arithmetic is 64-bit, but grid and tile counts must fit int32
-    const long long N = (long long)T * H * W;
-    if (N > (1ll << 31) || (long long)B * heads > (1ll << 24)) return VSA_ERR_INVALID_ARGUMENT;
-    return VSA_OK;
+    switch (vsa::shape_error(B, heads, d, T, H, W, tt, th, tw)) {
+        case 0: return VSA_OK;
+        case 2: return VSA_ERR_UNSUPPORTED;
+        default: return VSA_ERR_INVALID_ARGUMENT;
+    }
 }
 
 vsa::Grid grid_of(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
@@ -210,6 +207,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
         return VSA_ERR_CUDA;
     vsa::FineArgs a;
     a.g = g;
+    a.q = q;
     a.mq = &mq;
     a.mk = &mk;
     a.mv = &mv;
@@ -250,6 +248,7 @@ vsa_status vsa_sparse_attn_fwd_train(const vsa_bf16* q, const vsa_bf16* k, const
         return VSA_ERR_CUDA;
     vsa::FineArgs a;
     a.g = g;
+    a.q = q;
     a.mq = &mq;
     a.mk = &mk;
     a.mv = &mv;
@@ -357,6 +356,7 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
         return VSA_ERR_CUDA;
     vsa::FineArgs a;
     a.g = g;
+    a.q = q8;                  // unused: the E4M3 pass is the one-cube kernel
     a.mq = &mq;
     a.mk = &mk;
     a.mv = &mv;
@@ -380,7 +380,8 @@ vsa_status vsa_device_status(void* workspace, vsa_stream_t stream) {
         return VSA_ERR_CUDA;
     if (word != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
     if (word & vsa::kStatusTimeout) return VSA_ERR_TIMEOUT;
-    if (word & (vsa::kStatusBadIndex | vsa::kStatusMisaligned)) return VSA_ERR_DEVICE_CHECK;
+    if (word & (vsa::kStatusBadIndex | vsa::kStatusMisaligned | vsa::kStatusNonFinite | vsa::kStatusBadCoord))
+        return VSA_ERR_DEVICE_CHECK;
     return VSA_OK;
 }
 

@@ -12,7 +12,23 @@ enum : int {
     kStatusTimeout = 1,      // a bounded wait gave up
     kStatusBadIndex = 2,     // a block index outside [0, nt)
     kStatusMisaligned = 4,   // shared memory not aligned as the kernel needs
+    kStatusNonFinite = 8,    // debug-check build: a NaN or Inf reached an output
+    kStatusBadCoord = 16,    // debug-check build: a TMA box outside the grid
 };
+
+// Checks compiled in only with -DVSA_DEBUG_CHECKS (the library's debug-check
+// build, libvsa_debug.so): they record a status bit and let the kernel run on,
+// never trap.
+#ifdef VSA_DEBUG_CHECKS
+#define VSA_DEBUG_CHECK(cond, status, bit) \
+    do {                                   \
+        if (!(cond)) report(status, bit);  \
+    } while (0)
+#else
+#define VSA_DEBUG_CHECK(cond, status, bit) \
+    do {                                   \
+    } while (0)
+#endif
 
 // Geometry of the cube tiling of a T x H x W token grid.
 struct Grid {
@@ -24,6 +40,17 @@ struct Grid {
 };
 
 __host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+// Shape rules every entry point shares (0 = valid): 1 an invalid argument,
+// 2 an unsupported head_dim or tile volume.  Index arithmetic is 64-bit, but
+// grid and tile counts must fit int32.
+inline int shape_error(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
+    if (B < 1 || heads < 1 || d < 1 || T < 1 || H < 1 || W < 1 || tt < 1 || th < 1 || tw < 1) return 1;
+    if (d != 64 && d != 128) return 2;
+    if (tt * th * tw != 64) return 2;
+    if ((long long)T * H * W > (1ll << 31) || (long long)B * heads > (1ll << 24)) return 1;
+    return 0;
+}
 
 inline Grid make_grid(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
     Grid g;

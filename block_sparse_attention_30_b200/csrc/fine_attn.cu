@@ -520,7 +520,12 @@ cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
 }
 
-cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) { return launch_fine_single(a, stream); }
+// bf16, d = 128, sparse branch alone: the persistent two-cube kernel
+// (fine_pair.cu); the other variants run one CTA per query cube here.
+cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) {
+    if (!a.q_scale && !a.lin_image && a.g.d == 128) return launch_fine_pair(a, stream);
+    return launch_fine_single(a, stream);
+}
 
 int fine_smem_bytes(int d) { return d == 128 ? FineCfg<128>::SMEM_BYTES : FineCfg<64>::SMEM_BYTES; }
 

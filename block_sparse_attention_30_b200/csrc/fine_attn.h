@@ -10,6 +10,7 @@ namespace vsa {
 
 struct FineArgs {
     Grid g;
+    const void* q;               // bf16 q [B][N][heads][d] (the persistent kernel reads rows)
     const CUtensorMap* mq;       // 5-D maps over q, k, v (see api.cu)
     const CUtensorMap* mk;
     const CUtensorMap* mv;
@@ -28,6 +29,7 @@ struct FineArgs {
 
 cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream);
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream);
+cudaError_t launch_fine_pair(const FineArgs& a, cudaStream_t stream);
 int fine_smem_bytes(int d);
 
 }  // namespace vsa

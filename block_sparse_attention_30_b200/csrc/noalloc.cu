@@ -21,7 +21,9 @@
 //  * The first call on a device looks up the array's device address (once per
 //    device, with that device current); make that first call before any
 //    stream capture begins.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -36,21 +38,48 @@ static __device__ __align__(256) unsigned char g_select_scratch[VSA_NOALLOC_SELE
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of g_select_scratch on the current device (looked up once).
-// In host code the symbol itself is only a host-side stand-in, never a
-// device address, so the kernels must be given this pointer instead.
+// The driver's cuCtxGetCurrent, found through the runtime (no link-time
+// dependency on the driver library).
+PFN_cuCtxGetCurrent_v4000 ctx_get_fn() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    });
+    return fn;
+}
+
+// Device address of g_select_scratch on the current device, looked up once
+// per device and context.  In host code the symbol itself is only a
+// host-side stand-in, never a device address, so the kernels must be given
+// this pointer instead.  The context is remembered beside the address: after
+// a reset of the device's primary context (cudaDeviceReset) the module is
+// loaded again and the array may sit elsewhere, so the lookup is repeated
+// (also when this thread has no current context yet: the lookup binds the
+// device's primary context to it).
 cudaError_t scratch_for_current_device(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const PFN_cuCtxGetCurrent_v4000 get_ctx = ctx_get_fn();
+    if (!get_ctx) return cudaErrorInitializationError;
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
+    if (g_scratch_ptr[dev] == nullptr || ctx == nullptr || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_select_scratch);
         if (e != cudaSuccess) return e;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorInitializationError;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
@@ -66,12 +95,12 @@ extern "C" {
 vsa_status vsa_select_blocks_noalloc(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
                                      int head_dim, int T, int H, int W, int tt, int th, int tw,
                                      int topk, int32_t* block_idx, vsa_stream_t stream) {
-    if (B < 1 || heads < 1 || head_dim < 1 || T < 1 || H < 1 || W < 1 || tt < 1 || th < 1 || tw < 1)
-        return VSA_ERR_INVALID_ARGUMENT;
-    if (head_dim != 64 && head_dim != 128) return VSA_ERR_UNSUPPORTED;
-    if (tt * th * tw != 64) return VSA_ERR_UNSUPPORTED;
-    if ((long long)T * H * W > (1ll << 31) || (long long)B * heads > (1ll << 24))
-        return VSA_ERR_INVALID_ARGUMENT;
+    // the same shape rules as every other entry point (common.cuh)
+    switch (vsa::shape_error(B, heads, head_dim, T, H, W, tt, th, tw)) {
+        case 0: break;
+        case 2: return VSA_ERR_UNSUPPORTED;
+        default: return VSA_ERR_INVALID_ARGUMENT;
+    }
     const vsa::Grid g = vsa::make_grid(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(block_idx)) return VSA_ERR_INVALID_ARGUMENT;

@@ -43,12 +43,14 @@ __device__ __forceinline__ float softmax_step(float (&s)[64], uint64_t vmask, fl
     }
     float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-    for (int e = 4; e < 64; e += 8) {
+    for (int e = 4; e + 8 <= 60; e += 8) {       // s[4] .. s[59]
         m0 = max3f(m0, s[e], s[e + 1]);
         m1 = max3f(m1, s[e + 2], s[e + 3]);
         m2 = max3f(m2, s[e + 4], s[e + 5]);
         m3 = max3f(m3, s[e + 6], s[e + 7]);
     }
+    m0 = max3f(m0, s[60], s[61]);
+    m1 = max3f(m1, s[62], s[63]);
     // each half scales its own maximum (the two halves may hold key cubes
     // with different scales); for a common positive scale this equals scaling
     // the maximum of both, as rounding is monotonic

@@ -38,7 +38,15 @@
  *    allocates device memory, never frees it and never synchronises, except
  *    vsa_device_status.  It keeps no global state besides a cached driver
  *    entry point, per-device kernel attributes and the fixed device array of
- *    vsa_select_blocks_noalloc (end of this header), and is re-entrant.
+ *    vsa_select_blocks_noalloc (end of this header).  It is re-entrant, except
+ *    vsa_select_blocks_noalloc, whose calls share that array and must be
+ *    ordered on one stream.
+ *  - Faults recorded on the device: a bounded wait that gave up
+ *    (VSA_ERR_TIMEOUT), a block index out of range or a misaligned shared
+ *    memory window (VSA_ERR_DEVICE_CHECK); the debug-check build
+ *    (libvsa_debug.so, compiled with -DVSA_DEBUG_CHECKS) also records a NaN
+ *    or Inf reaching an output and a TMA box outside the grid
+ *    (VSA_ERR_DEVICE_CHECK).  Nothing traps.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream).  Argument errors are reported before any launch;
  *    launch failures return VSA_ERR_CUDA.  Faults detected on the device
@@ -78,11 +86,13 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
 /* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
  * for these shapes: a 256-byte status block followed by a scratch area that
  * holds either the selection's fp64 cube means of q and k
- * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the
- * linear branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is
- * larger (the backward passes' scratch fits it too: the sparse branch's row
- * terms and block-index transpose, the linear branch's two operand images
- * and fp32 gradient sums).  Returns 0 for invalid shapes.  The
+ * ([2][B][heads][nt][d]; the coarse scores stay in on-chip memory, except
+ * for grids whose score rows do not fit one SM's shared memory eight at a
+ * time, about nt > 1640 at d = 128, which also keep the fp64 scores
+ * [B][heads][nt][nt] here), or the linear branch's operand image (B*heads*(4*d*d + 4*d)
+ * bytes), whichever is larger (the backward passes' scratch fits it too: the
+ * sparse branch's row terms and block-index transpose, the linear branch's
+ * two operand images and fp32 gradient sums).  Returns 0 for invalid shapes.  The
  * same workspace may be passed to every call of one forward pass; calls that
  * share a workspace must be ordered on one stream. */
 size_t vsa_workspace_bytes(int B, int heads, int head_dim, int T, int H, int W,
@@ -110,7 +120,10 @@ vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int he
  * attends to).  Mean-pools q and k per cube over valid tokens (fp64), scores
  * C[i][j] = Qp[i].Kp[j]/sqrt(d) in fp64 and writes, per (b, head, i), the
  * topk key cubes with the largest C (ties -> lower j) in ascending order to
- * block_idx.  1 <= topk <= nt.  Needs vsa_workspace_bytes() of workspace. */
+ * block_idx.  1 <= topk <= nt.  Needs vsa_workspace_bytes() of workspace.
+ * Two launches: the cube means, then one kernel that scores a block of 16
+ * (or, for long rows, 8) query cubes against every key cube and selects
+ * their top-k on chip. */
 vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
                              int head_dim, int T, int H, int W, int tt, int th, int tw,
                              int topk, int32_t* block_idx, void* workspace,
@@ -250,22 +263,24 @@ vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
  * allocation, a fixed memory budget, an embedding without an allocator) and
  * so cannot provide vsa_select_blocks' workspace.  It computes exactly what
  * vsa_select_blocks computes, with the same kernels, but keeps the
- * intermediate fp64 cube means and coarse scores in one file-scope device
- * array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved on every GPU that loads
- * the library until the process exits.  It allocates and frees nothing.
+ * intermediate fp64 cube means (and, for very large grids, coarse scores) in
+ * one file-scope device array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved
+ * on every GPU that loads the library until the process exits.  It allocates and frees nothing.
  *
  *  - The caller still passes q, k (device, bf16 [B][N][heads][d]) and
  *    block_idx (device, int32 [B][heads][nt][topk]), 16-byte aligned.
- *  - Shapes whose intermediates exceed the array
- *    (2*B*heads*nt*d*8 + B*heads*nt*nt*8 bytes > the maximum) are rejected
- *    with VSA_ERR_WORKSPACE before anything is enqueued; argument errors as
+ *  - Shapes whose intermediates exceed the array are rejected with
+ *    VSA_ERR_WORKSPACE before anything is enqueued (the intermediates are the
+ *    fp64 cube means, 2*B*heads*nt*d*8 bytes, plus B*heads*nt*nt*8 bytes of
+ *    scores for grids beyond about nt = 1640 at d = 128); argument errors as
  *    for vsa_select_blocks.
  *  - All calls share the array, which keeps the last call's contents; every
  *    call rewrites what it reads, so nothing needs clearing.  Calls that
  *    overlap on the GPU (other streams, unordered host threads) race on it:
  *    order them on one stream.
- *  - The first call on each device looks up the array's device address with
- *    that device current; make that first call before any stream capture.
+ *  - The first call on each device (and the first after the device's
+ *    primary context was reset) looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
  */
 #define VSA_NOALLOC_SELECT_SCRATCH_BYTES (32u * 1024u * 1024u)
 

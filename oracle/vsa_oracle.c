@@ -539,11 +539,6 @@ void oracle_weights(const uint16_t *q, const uint16_t *kk, const int32_t *idx,
         }
 }
 
-/* ----------------------------------------------------- linear branch (step 6)
- * phi(x) = elu(x) + 1 = x + 1 for x > 0, exp(x) otherwise, applied to the raw
- * q and k (no projection, weight one).  The state sums run over ALL valid
- * tokens:  S = sum_n phi(k_n)^T v_n  (d x d),  z = sum_n phi(k_n)  (d).
- * lin_n = phi(q_n) S / (phi(q_n) . z). */
 /* ------------------------------------------------------ fine pass, backward
  * Gradients of the fine pass (trainable sparse attention: "FastVideo
  * 稀疏蒸馏技术深度解析", section "2. 视频稀疏注意力VSA", and the TurboDiffusion
@@ -632,6 +627,11 @@ void oracle_fine_bwd(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
     }
 }
 
+/* ----------------------------------------------------- linear branch (step 6)
+ * phi(x) = elu(x) + 1 = x + 1 for x > 0, exp(x) otherwise, applied to the raw
+ * q and k (no projection, weight one).  The state sums run over ALL valid
+ * tokens:  S = sum_n phi(k_n)^T v_n  (d x d),  z = sum_n phi(k_n)  (d).
+ * lin_n = phi(q_n) S / (phi(q_n) . z). */
 static REAL phi(REAL x) { return x > 0 ? x + 1 : ORACLE_EXP(x); }
 
 void oracle_linear_state(const uint16_t *kk, const uint16_t *v, int B, int heads,
@@ -678,9 +678,6 @@ void oracle_linear_apply(const uint16_t *q, const REAL *S, const REAL *z, int B,
             }
 }
 
-/* ------------------------------------------------------------ dense (pin)
- * Plain dense softmax attention over all N tokens of the grid; with k equal
- * to the tile count the block-sparse fine pass must reduce to this. */
 /* ---------------------------------------------------- linear branch, backward
  * Gradients of the linear branch (SLA: the sparse and the linear branch are
  * trained together, TurboDiffusion article, section "稀疏、蒸馏与全链路量化").
@@ -764,6 +761,9 @@ void oracle_linear_bwd(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
         }
 }
 
+/* ------------------------------------------------------------ dense (pin)
+ * Plain dense softmax attention over all N tokens of the grid; with k equal
+ * to the tile count the block-sparse fine pass must reduce to this. */
 void oracle_dense(const uint16_t *q, const uint16_t *kk, const uint16_t *v,
                   int B, int heads, int d, int64_t N, REAL *out)
 {

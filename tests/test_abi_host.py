@@ -3,6 +3,7 @@ every entry point include/vsa.h declares, and rejects bad arguments with the
 documented status codes before touching the device."""
 import ctypes
 import os
+import subprocess
 import re
 
 import pytest
@@ -54,9 +55,16 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_num_tiles(20, 28, 52, 4, 4, 4) == 455
     assert L.vsa_num_tiles(4, 32, 32, 4, 4, 4) == 64
     assert L.vsa_num_tiles(0, 4, 4, 4, 4, 4) == 0
+    # the selection keeps only the fp64 cube means in the workspace when 8 or
+    # 16 query cubes' score rows fit the fused kernel's shared memory (nt up
+    # to ~1640 at d = 128), the whole fp64 score matrix beyond
     nt, B, h, d = 455, 1, 40, 128
-    want = 256 + 2 * B * h * nt * d * 8 + B * h * nt * nt * 8
+    want = 256 + 2 * B * h * nt * d * 8
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 46) == want
+    nt = 1440                                                                 # 720P grid, ragged
+    assert L.vsa_workspace_bytes(B, h, d, 21, 45, 80, 4, 4, 4, 144) == 256 + 2 * B * h * nt * d * 8
+    nt = 2048                                                                 # 32 x 64 x 64: rows too long
+    assert L.vsa_workspace_bytes(1, 2, d, 32, 64, 64, 4, 4, 4, 8) == 256 + 2 * 2 * nt * d * 8 + 2 * nt * nt * 8
     assert L.vsa_workspace_bytes(B, h, 96, 20, 28, 52, 4, 4, 4, 46) == 0       # d unsupported
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 0) == 0         # topk < 1
@@ -150,12 +158,58 @@ def test_other_entry_points_validate(L):
 
 
 def test_library_has_no_oracle_dependency():
-    """The product library never links or names the oracle."""
-    with open(_lib.LIB_PATH, "rb") as fh:
-        blob = fh.read()
-    assert b"oracle" not in blob
+    """The product library never links or exports the oracle: its dynamic
+    dependencies (readelf's NEEDED entries) and its exported symbols (nm -D)
+    name no oracle library or function, and no package source imports it."""
+    dyn = subprocess.run(["readelf", "-d", _lib.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    needed = [ln for ln in dyn.splitlines() if "(NEEDED)" in ln]
+    assert needed and not any("oracle" in ln for ln in needed), needed
+    syms = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True,
+                          check=True).stdout
+    assert "vsa_select_blocks" in syms and "oracle" not in syms
     for root, _, files in os.walk(os.path.join(ROOT, "block_sparse_attention_30_b200")):
         for fn in files:
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(root, fn), encoding="utf-8").read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_cuda_failures_surface_as_status_codes(L):
+    """Host-side error injection into the VSA_ERR_CUDA paths: on a machine
+    without a CUDA device every CUDA runtime or driver call the library makes
+    (launches, memsets, stream synchronisation, tensor-map encoding, symbol
+    lookup) returns an error.  With arguments that pass validation, each entry
+    point must report that as VSA_ERR_CUDA, never crash, never return OK."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a CUDA device (fake pointers would reach a real launch)")
+    CUDA = 4
+    SH = (1, 2, 128, 4, 8, 8, 4, 4, 4)          # 4 cubes of 64 tokens, d = 128
+    ws = L.vsa_workspace_bytes(*SH, 2)
+    assert ws > 0
+    assert L.vsa_workspace_init(FAKE, ws, None) == CUDA
+    assert L.vsa_gather_tiles(FAKE, FAKE, *SH, None) == CUDA
+    assert L.vsa_scatter_tiles(FAKE, FAKE, *SH, None) == CUDA
+    assert L.vsa_select_blocks(FAKE, FAKE, *SH, 2, FAKE, FAKE, ws, None) == CUDA
+    assert L.vsa_select_blocks_noalloc(FAKE, FAKE, *SH, 2, FAKE, None) == CUDA
+    assert L.vsa_linear_branch_fwd(FAKE, FAKE, FAKE, FAKE, *SH[:6], FAKE, ws, None) == CUDA
+    assert L.vsa_sparse_attn_fwd(*[FAKE] * 4, None, None, FAKE, *SH, 2, FAKE, ws, None) == CUDA
+    assert L.vsa_sparse_attn_fwd(*[FAKE] * 7, *SH, 2, FAKE, ws, None) == CUDA          # with the linear branch
+    assert L.vsa_sparse_attn_fwd_train(*[FAKE] * 7, *SH, 2, FAKE, ws, None) == CUDA
+    assert L.vsa_sparse_attn_bwd(*[FAKE] * 10, *SH, 2, FAKE, ws, None) == CUDA
+    assert L.vsa_linear_branch_bwd(*[FAKE] * 9, 0, *SH[:6], FAKE, ws, None) == CUDA
+    assert L.vsa_quantize_qk_e4m3(*[FAKE] * 6, *SH, None) == CUDA
+    assert L.vsa_sparse_attn_fwd_e4m3(*[FAKE] * 7, *SH, 2, FAKE, ws, None) == CUDA
+    assert L.vsa_selftest_wait_timeout(FAKE, ws, 1000, None) == CUDA
+    assert L.vsa_device_status(FAKE, None) == CUDA
+
+
+def test_debug_check_build_exports_every_symbol():
+    """The debug-check build (-DVSA_DEBUG_CHECKS: non-finite outputs and TMA
+    boxes outside the grid are recorded in the status word) compiles for
+    sm_100a and exports the same C ABI as the product library."""
+    lib = build.build(debug_checks=True)
+    assert lib.endswith("libvsa_debug.so") and os.path.exists(lib)
+    syms = subprocess.run(["nm", "-D", "--defined-only", lib], capture_output=True, text=True, check=True).stdout
+    for name in declared_functions():
+        assert re.search(r"\b%s\b" % name, syms), name

@@ -1,6 +1,7 @@
 """Host-side logic of bench.py that needs no GPU: the roofline traffic lookup
-from the committed ncu summary and the peak table."""
+from the committed ncu capture data and the peak table."""
 import hashlib
+import json
 import os
 
 import bench
@@ -12,16 +13,15 @@ def _hash():
                                    for f in bench.FINE_SOURCES)).hexdigest()[:16]
 
 
-def test_traffic_is_reported_only_for_the_profiled_sources(tmp_path, monkeypatch):
-    prof = tmp_path / "profile.md"
-    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(prof))
-    prof.write_text(f"traffic_bytes_per_launch[wan14b_480p]: 123456\nsources_sha256: {_hash()}\n")
-    assert bench.profiled_traffic("wan14b_480p") == 123456
-    assert bench.profiled_traffic("wan1.3b_480p") is None            # not in the summary
-    prof.write_text("traffic_bytes_per_launch[wan14b_480p]: 123456\nsources_sha256: 0000000000000000\n")
-    assert bench.profiled_traffic("wan14b_480p") is None             # sources changed since
-    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(tmp_path / "missing.md"))
-    assert bench.profiled_traffic("wan14b_480p") is None
+def test_traffic_is_reported_only_for_the_profiled_sources(tmp_path):
+    data = tmp_path / "traffic.json"
+    data.write_text(json.dumps({"sources_sha256": _hash(), "bytes_per_launch": {"wan14b_480p": 123456}}))
+    assert bench.profiled_traffic("wan14b_480p", str(data)) == 123456
+    assert bench.profiled_traffic("wan1.3b_480p", str(data)) is None      # not captured
+    data.write_text(json.dumps({"sources_sha256": "0" * 16, "bytes_per_launch": {"wan14b_480p": 123456}}))
+    assert bench.profiled_traffic("wan14b_480p", str(data)) is None       # sources changed since
+    assert bench.profiled_traffic("wan14b_480p", str(tmp_path / "missing.json")) is None
+    assert bench.fine_sources_hash() == _hash()
 
 
 def test_peaks_fall_back_when_the_measured_table_is_absent(tmp_path, monkeypatch):

@@ -293,10 +293,11 @@ def test_tiny_workload_full(ops, name):
 
 
 @pytest.mark.parametrize("name,heads_sel", [("wan1.3b_480p", None), ("wan14b_480p", None),
-                                            ("wan14b_720p_ragged", (0, 4)),
+                                            ("wan14b_720p_ragged", None),
                                             ("sparse97_linear_480p", None)])
 def test_workload_selection(ops, name, heads_sel):
-    """Selection on the full-size workloads (a head subset for the largest)."""
+    """Selection on the full-size workloads, every head (the oracle's fp64
+    selection is ~21 GFLOP at 720P, seconds on the host cores)."""
     w, q, k, v, qd, kd, vd = inputs(name)
     idx, _ = run_select(ops, w, qd, kd)
     idx = idx.cpu().numpy()
@@ -311,9 +312,40 @@ def test_workload_selection(ops, name, heads_sel):
     check_indices(idx, ref_idx, scores)
 
 
+def ragged_class_rows(w, idx_np):
+    """Query cubes that name every ragged class of the grid: a cube on the last
+    t-layer only, on the last h-row only, on the last w-column only, on two or
+    three of them (the corner), and a whole query cube whose kept key cubes
+    include partial ones.  Rows are (b*heads + head)*nt + i, from head 1 (a
+    different head from the fixed samples) where the grid has it."""
+    nT, nh, nw = w.tile_grid
+    nt = nT * nh * nw
+    T_r, H_r, W_r = w.T % w.tile[0] != 0, w.H % w.tile[1] != 0, w.W % w.tile[2] != 0
+    cube = lambda it, ih, iw: (it * nh + ih) * nw + iw
+    head = min(1, w.heads - 1)
+    picks = []
+    if T_r: picks.append(cube(nT - 1, 0, 0))
+    if H_r: picks.append(cube(0, nh - 1, 0))
+    if W_r: picks.append(cube(0, 0, nw - 1))
+    if T_r and H_r: picks.append(cube(nT - 1, nh - 1, 0))
+    if T_r and H_r and W_r: picks.append(cube(nT - 1, nh - 1, nw - 1))
+    partial = set()
+    for it in range(nT):
+        for ih in range(nh):
+            for iw in range(nw):
+                if (T_r and it == nT - 1) or (H_r and ih == nh - 1) or (W_r and iw == nw - 1):
+                    partial.add(cube(it, ih, iw))
+    if partial:
+        full_rows = [i for i in range(nt) if i not in partial and set(idx_np[0, head, i].tolist()) & partial]
+        picks.append(full_rows[0])
+    return [head * nt + i for i in picks]
+
+
 @pytest.mark.parametrize("name", ["wan1.3b_480p", "wan14b_480p", "wan14b_720p_ragged"])
 def test_workload_fine_sampled(ops, name):
-    """Full-size fine pass, checked on sampled query cubes (incl. edge cubes)."""
+    """Full-size fine pass, checked on sampled query cubes plus, on ragged
+    grids, one query cube of every ragged class and one whose selection holds
+    partial key cubes."""
     w, q, k, v, qd, kd, vd = inputs(name)
     idx, ws = run_select(ops, w, qd, kd)
     out = run_fine(ops, w, qd, kd, vd, idx, ws)
@@ -321,8 +353,26 @@ def test_workload_fine_sampled(ops, name):
     nt = ops.vsa_num_tiles(w.T, w.H, w.W, w.tile)
     nT, nh, nw = w.tile_grid
     corner = (nT - 1) * nh * nw + (nh - 1) * nw + (nw - 1)     # most ragged cube of head 0
-    rows = sample_rows(nt, w.heads, w.B, 24, seed=len(name), extra=(corner,))
-    check_fine_sample(out, w, q, k, v, idx.cpu().numpy(), rows)
+    idx_np = idx.cpu().numpy()
+    classes = ragged_class_rows(w, idx_np)
+    if name == "wan14b_720p_ragged":
+        assert len(classes) == 4                                 # last-t, last-h, both, partial keys
+    rows = sample_rows(nt, w.heads, w.B, 24, seed=len(name), extra=(corner, *classes))
+    check_fine_sample(out, w, q, k, v, idx_np, rows)
+
+
+def test_headline_fine_two_heads_full(ops):
+    """Full-size 14B-480P fine pass checked on every token of heads 0 and 1:
+    910 query cubes, so each persistent CTA walks several cube pairs and one
+    pair straddles the two heads (nt = 455 is odd)."""
+    w, q, k, v, qd, kd, vd = inputs("wan14b_480p")
+    idx, ws = run_select(ops, w, qd, kd)
+    out = run_fine(ops, w, qd, kd, vd, idx, ws)
+    hs = slice(0, 2)
+    sub = lambda x: x[:, :, hs].contiguous()
+    ref = O.fine(sub(q), sub(k), sub(v), idx[:, hs].cpu().numpy(), w.B, 2, w.head_dim,
+                 w.T, w.H, w.W, w.tile)
+    check_close(to_f64(out[:, :, hs]), ref)
 
 
 # -------------------------------------------------------------- linear branch
@@ -739,3 +789,41 @@ def test_grid_smaller_than_a_cube_is_dense_attention(ops):
     q64, k64, v64 = (x.double().permute(0, 2, 1, 3) for x in (c.q, c.k, c.v))
     ref = torch.nn.functional.scaled_dot_product_attention(q64, k64, v64).permute(0, 2, 1, 3)
     check_close(to_f64(out), ref.numpy())
+
+
+def test_debug_check_build_reports_non_finite_output(ops):
+    """libvsa_debug.so (the -DVSA_DEBUG_CHECKS build) records a NaN or Inf
+    that reaches the fine pass's output in the status word, reported as
+    VSA_ERR_DEVICE_CHECK, without trapping; clean inputs stay VSA_OK and give
+    the same output as the product library."""
+    import ctypes
+    from block_sparse_attention_30_b200 import _lib, build
+    path = build.build(debug_checks=True)
+    L = ctypes.CDLL(path)
+    for name, (res, args) in _lib.SIGNATURES.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    c = Small(8, 16, 16, 2, 128, 5, seed=3)
+    qd, kd, vd = c.q.cuda(), c.k.cuda(), c.v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    shape = [1, 2, 128, 8, 16, 16, 4, 4, 4]
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def fine_debug(v):
+        out = torch.zeros_like(qd)
+        assert L.vsa_sparse_attn_fwd(qd.data_ptr(), kd.data_ptr(), v.data_ptr(), idx.data_ptr(), None, None,
+                                     out.data_ptr(), *shape, 5, ws.data_ptr(), ws.numel(), stream) == 0
+        return out, L.vsa_device_status(ws.data_ptr(), stream)
+    out, st = fine_debug(vd)
+    assert st == 0
+    assert torch.equal(out, run_fine(ops, c, qd, kd, vd, idx, ws))
+    # one value of the first token of a key cube that query cube 0 of head 1 keeps
+    j = int(idx[0, 1, 0, 0])
+    it, ih, iw = j // 16, (j // 4) % 4, j % 4          # 2 x 4 x 4 cubes
+    n = (4 * it * 16 + 4 * ih) * 16 + 4 * iw
+    bad = vd.clone()
+    bad[0, n, 1, 7] = float("inf")
+    _, st = fine_debug(bad)
+    assert st == 6, _lib.STATUS_NAMES.get(st, st)     # VSA_ERR_DEVICE_CHECK
+    _, st = fine_debug(vd)
+    assert st == 0                                     # the word was cleared by the report
