@@ -41,10 +41,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Sources of the fine kernel the step runs for bf16 d = 128 without the linear
-# branch (the persistent two-cube kernel); a DRAM-traffic figure is reported
-# only while they hash to the value recorded beside it.
-FINE_SOURCES = ["fine_pair.cu", "softmax_step.cuh", "sm100.cuh", "common.cuh"]
+# Sources of the fine kernel the headline step runs (bf16, d = 128, k = 46:
+# the one-cube-per-CTA kernel); a DRAM-traffic figure is reported only while
+# they hash to the value recorded beside it.
+FINE_SOURCES = ["fine_attn.cu", "softmax_step.cuh", "sm100.cuh", "common.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -155,9 +155,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+PAIR_MAX_TOPK = 24        # launch_fine: short rows run the persistent two-cube kernel
+
+
 def fine_kernel_name(w):
     """The fine kernel vsa_sparse_attn_fwd launches for this workload."""
-    if w.head_dim == 128 and not w.linear:
+    if w.head_dim == 128 and not w.linear and w.topk <= PAIR_MAX_TOPK:
         return "fine_pair_kernel<128>"
     return "fine_attn_kernel<%d, %s>" % (w.head_dim, "LIN" if w.linear else "-")
 

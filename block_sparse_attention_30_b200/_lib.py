@@ -34,6 +34,7 @@ SIGNATURES = {
     "vsa_linear_branch_bwd": (_i, [_p] * 9 + [_i] * 7 + [_p, _sz, _p]),
     "vsa_quantize_qk_e4m3": (_i, [_p] * 6 + _SHAPE + [_p]),
     "vsa_sparse_attn_fwd_e4m3": (_i, [_p] * 7 + _SHAPE + [_i, _p, _sz, _p]),
+    "vsa_sparse_linear_attn_fwd_e4m3": (_i, [_p] * 10 + _SHAPE + [_i, _p, _sz, _p]),
     "vsa_device_status": (_i, [_p, _p]),
     "vsa_select_blocks_noalloc": (_i, [_p, _p] + _SHAPE + [_i, _p, _p]),
     "vsa_selftest_wait_timeout": (_i, [_p, _sz, ctypes.c_uint, _p]),

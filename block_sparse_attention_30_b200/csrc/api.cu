@@ -356,7 +356,7 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
         return VSA_ERR_CUDA;
     vsa::FineArgs a;
     a.g = g;
-    a.q = q8;                  // unused: the E4M3 pass is the one-cube kernel
+    a.q = nullptr;             // no linear branch: no bf16 q needed
     a.mq = &mq;
     a.mk = &mk;
     a.mv = &mv;
@@ -369,6 +369,49 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
     a.q_scale = q_scale;
     a.k_scale = k_scale;
     a.status = static_cast<int*>(workspace);
+    return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
+}
+
+vsa_status vsa_sparse_linear_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
+                                           const float* k_scale, const vsa_bf16* q, const vsa_bf16* v,
+                                           const int32_t* block_idx, const float* lin_S,
+                                           const float* lin_z, vsa_bf16* out, int B, int heads,
+                                           int head_dim, int T, int H, int W, int tt, int th, int tw,
+                                           int topk, void* workspace, size_t workspace_bytes,
+                                           vsa_stream_t stream) {
+    vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (s != VSA_OK) return s;
+    if (head_dim != 128) return VSA_ERR_UNSUPPORTED;
+    const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
+    if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
+    for (const void* p : {(const void*)q8, (const void*)k8, (const void*)q_scale, (const void*)k_scale,
+                          (const void*)q, (const void*)v, (const void*)block_idx, (const void*)lin_S,
+                          (const void*)lin_z, (const void*)out})
+        if (!aligned16(p)) return VSA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (workspace_bytes < kStatusBytes + lin_image_bytes(g)) return VSA_ERR_WORKSPACE;
+    CUtensorMap mq, mk, mv;
+    if (!encode_grid_map_u8(&mq, q8, g) || !encode_grid_map_u8(&mk, k8, g) || !encode_grid_map(&mv, v, g))
+        return VSA_ERR_CUDA;
+    vsa::FineArgs a;
+    a.g = g;
+    a.q = q;                   // bf16 q: the linear branch's phi(q)
+    a.mq = &mq;
+    a.mk = &mk;
+    a.mv = &mv;
+    a.block_idx = block_idx;
+    a.topk = topk;
+    a.out = out;
+    a.out32 = nullptr;
+    a.lse = nullptr;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.status = static_cast<int*>(workspace);
+    // the bf16 hi/lo operand image of (S, z) goes into the workspace scratch
+    a.lin_image = static_cast<uint8_t*>(workspace) + kStatusBytes;
+    cudaError_t e = vsa::launch_linear_pack(g, lin_S, lin_z, const_cast<void*>(a.lin_image),
+                                            (cudaStream_t)stream);
+    if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(vsa::launch_fine(a, (cudaStream_t)stream));
 }
 

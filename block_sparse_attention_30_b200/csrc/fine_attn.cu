@@ -34,7 +34,10 @@
 // one scale per (b, head, cube) (quant.cu); Q K^T runs as tcgen05
 // kind::f8f6f4 (K = 32 per MMA, one 128-byte row per token), the softmax
 // multiplies each half row by its query and key cube scales, P V stays bf16.
-// The halved Q and K tiles make room for a second V stage.
+// The halved Q and K tiles make room for a second V stage.  With the linear
+// branch (SageSLA: the sparse + linear attention on quantised products), the
+// branch itself stays bf16 hi + lo: phi(q) comes from the bf16 q in global
+// memory and goes into the K ring, the (S, z) image into the V ring.
 //
 // Every wait is bounded; on a timeout the CTA records kStatusTimeout in the
 // status word, drains its own copies and MMAs, frees TMEM and exits.
@@ -80,8 +83,10 @@ struct FineCfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int Z_BYTES = D * 4;              // linear branch: z (fp32)
     static constexpr int SMEM_BYTES = Q_BYTES + NK * K_PAIR_BYTES + NV * V_PAIR_BYTES + BAR_BYTES + Z_BYTES;
-    // the linear branch's S hi + lo image must fit the K ring, phi(Q) lo the V ring
-    static_assert(Q8 || (4 * D * D <= NK * K_PAIR_BYTES && Q_BYTES <= NV * V_PAIR_BYTES), "linear operands");
+    // the linear branch's S hi + lo image must fit the K ring, phi(Q) lo the V
+    // ring (bf16); low precision: phi(Q) hi + lo the K ring, the image the V ring
+    static_assert(Q8 ? (2 * 64 * D * 2 <= NK * K_PAIR_BYTES && 4 * D * D <= NV * V_PAIR_BYTES)
+                     : (4 * D * D <= NK * K_PAIR_BYTES && Q_BYTES <= NV * V_PAIR_BYTES), "linear operands");
 };
 
 template <int D, bool Q8 = false>
@@ -107,9 +112,9 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                  const int ragged, const uint8_t* __restrict__ lin_image,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ out32, float* __restrict__ lse,
                  const float* __restrict__ q_scale, const float* __restrict__ k_scale,
-                 int* status) {
+                 const __nv_bfloat16* __restrict__ q_bf16, int* status) {
     using C = FineCfg<D, Q8>;
-    static_assert(!(Q8 && LIN), "the low-precision variant has no linear branch");
+    static_assert(!Q8 || D == 128, "the low-precision variant is d = 128");
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
         if (threadIdx.x == 0) report(status, kStatusMisaligned);
@@ -131,13 +136,15 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     constexpr bool lin = LIN;
     // Linear-branch operands reuse the buffers of the sparse pass:
     //   S hi / lo (B, MN-major) + z: one bulk copy of the (b, head) image into
-    //     the K ring once the last Q K^T is done, z into its own 512 bytes;
-    //   phi(Q) hi / lo (A, K-major like Q): hi over Q in place, lo in the V
-    //     ring, once the last P V is done.
-    uint8_t* sPhiHi = sQ;
-    uint8_t* sPhiLo = sV;
-    uint8_t* sSHi = sK;
-    uint8_t* sSLo = sK + D * D * 2;
+    //     the K ring once the last Q K^T is done (bf16 q, k) or into the V
+    //     ring once the last P V is done (E4M3 q, k), z into its own 512 bytes;
+    //   phi(Q) hi / lo (A, K-major like a bf16 Q): bf16 q, k: hi over Q in
+    //     place, lo in the V ring, once the last P V is done; E4M3 q, k: both
+    //     in the K ring, from the bf16 q in global memory.
+    uint8_t* sPhiHi = Q8 ? sK : sQ;
+    uint8_t* sPhiLo = Q8 ? sK + 64 * D * 2 : sV;
+    uint8_t* sSHi = Q8 ? sV : sK;
+    uint8_t* sSLo = sSHi + D * D * 2;
     float* sZ = reinterpret_cast<float*>(sV + C::NV * C::V_PAIR_BYTES + C::BAR_BYTES);
 
     if (tid == 0) {
@@ -217,13 +224,15 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 ++issued;
             }
             bool lin_issued = false;
-            if (lin && is_k && issued == n_pairs && !*abort_flag) {
-                // the (S, z) image goes into the K ring once the last Q K^T
-                // MMAs (each stage's last use) are done
+            if (lin && is_k != Q8 && issued == n_pairs && !*abort_flag) {
+                // the (S, z) image goes into the K ring (bf16) or the V ring
+                // (E4M3) once the last MMAs reading each of its stages are done
                 bool free = true;
-                for (int p = max(0, n_pairs - nst); p < n_pairs && free; ++p)
-                    free = C::K_ON_S ? mbar_wait(&bars->s_full[p & 1], (p >> 1) & 1, abort_flag)
-                                     : mbar_wait(&empty[p % nst], (p / nst) & 1, abort_flag);
+                for (int p = max(0, n_pairs - nst); p < n_pairs && free; ++p) {
+                    if (is_k && C::K_ON_S) free = mbar_wait(&bars->s_full[p & 1], (p >> 1) & 1, abort_flag);
+                    else if (!is_k && C::V_ON_O) free = mbar_wait(&bars->o_ready[p & 1], (p >> 1) & 1, abort_flag);
+                    else free = mbar_wait(&empty[p % nst], (p / nst) & 1, abort_flag);
+                }
                 if (free) {
                     const uint8_t* img = lin_image + (long long)bh * (4 * D * D + 4 * D);
                     mbar_arrive_expect_tx(&bars->lin_full, 4 * D * D + 4 * D);
@@ -382,6 +391,11 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             mbar_arrive(&bars->p_full[x]);
         }
         if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_ready[(n_pairs - 1) & 1], ((n_pairs - 1) >> 1) & 1, abort_flag))) ok = false;
+        // this thread's query slot: token n of the grid, if the slot is valid
+        const TileCoord qc = tile_coord(g, i);
+        const int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
+        const bool valid = dt < qc.vt && dh < qc.vh && dw < qc.vw;
+        const long long n = ((long long)(qc.t0 + dt) * g.H + (qc.h0 + dh)) * g.W + (qc.w0 + dw);
         // ------------------------------------------------------- linear branch
         // phi(q) = elu(q) + 1 (SparkDiffusion RoLA / TurboDiffusion SLA linear
         // branch).  Each thread owns half a query row: D/2 features.
@@ -392,14 +406,21 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             const float* zb = sZ + hf * (D / 2);
             float dpart = 0.f;
             // phi(Q) hi/lo: this thread's D/2 features sit in chunk (hf*(D/2))/64
-            // of the Q cube, 16-byte units u0 .. u0 + D/16 - 1 of row r; hi
-            // replaces q in place, lo goes to the same offset in the V ring.
+            // of a bf16 Q cube, 16-byte units u0 .. u0 + D/16 - 1 of row r.
+            // bf16 q, k: q is read from the Q tile, hi replaces it in place and
+            // lo goes to the same offset in the V ring.  E4M3 q, k: q is read
+            // from global memory (0 for padded slots), hi and lo go to the two
+            // halves of the K ring, which the last Q K^T no longer needs.
             const int chunk = (hf * (D / 2)) / 64, u0 = ((hf * (D / 2)) % 64) / 8;
+            const uint4* qrow = reinterpret_cast<const uint4*>(
+                q_bf16 + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2));
 #pragma unroll
             for (int u = 0; u < D / 16; ++u) {
                 const int uu = u0 + u;
                 const uint32_t off = chunk * 8192 + r * 128 + (((uu) ^ (r & 7)) << 4);
-                const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
+                uint4 raw;
+                if constexpr (Q8) raw = valid ? __ldg(qrow + u) : make_uint4(0u, 0u, 0u, 0u);
+                else raw = *reinterpret_cast<const uint4*>(sQ + off);
                 const float4 z0 = reinterpret_cast<const float4*>(zb + u * 8)[0];
                 const float4 z1 = reinterpret_cast<const float4*>(zb + u * 8)[1];
                 const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
@@ -429,10 +450,6 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             const float l = sm.l_run + __shfl_xor_sync(0xffffffffu, sm.l_run, 16);
             const float inv = 1.f / l;
             const float inv_den = 1.f / den;
-            const TileCoord qc = tile_coord(g, i);
-            const int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
-            const bool valid = dt < qc.vt && dh < qc.vh && dw < qc.vw;
-            const long long n = ((long long)(qc.t0 + dt) * g.H + (qc.h0 + dh)) * g.W + (qc.w0 + dw);
             __nv_bfloat16* orow = out + (((long long)b * g.N + n) * g.heads + head) * D + hf * (D / 2);
             // log2 of the softmax normaliser of the scaled scores (for the
             // backward pass); +inf marks padded query slots (zero weight there)
@@ -509,21 +526,28 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
     fine_attn_kernel<D, LIN, Q8><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(
         *a.mq, *a.mk, *a.mv, a.g, a.block_idx, a.topk, scale_log2, ragged,
         static_cast<const uint8_t*>(a.lin_image), reinterpret_cast<__nv_bfloat16*>(a.out), a.out32, a.lse,
-        a.q_scale, a.k_scale, a.status);
+        a.q_scale, a.k_scale, static_cast<const __nv_bfloat16*>(a.q), a.status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
-    if (a.q_scale) return launch_fine_impl<128, false, true>(a, stream);   // E4M3 q, k (d = 128)
     const bool lin = a.lin_image != nullptr;
+    if (a.q_scale)                                                      // E4M3 q, k (d = 128)
+        return lin ? launch_fine_impl<128, true, true>(a, stream) : launch_fine_impl<128, false, true>(a, stream);
     if (a.g.d == 128) return lin ? launch_fine_impl<128, true>(a, stream) : launch_fine_impl<128, false>(a, stream);
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
 }
 
-// bf16, d = 128, sparse branch alone: the persistent two-cube kernel
-// (fine_pair.cu); the other variants run one CTA per query cube here.
+// Kernel choice for the bf16, d = 128 sparse branch.  Short rows (few kept
+// cubes per query cube) go to the persistent two-cube kernel (fine_pair.cu),
+// which pays a CTA's set-up and pipeline fill once per SM instead of once
+// per query cube; long rows amortise that set-up and run faster here, with
+// one CTA per query cube and two CTAs per SM (measured on B200 at the 97 %
+// shape, k = 11: 0.196 vs 0.212 ms; at 14B-480P, k = 46: 2.63 vs 2.42 ms).
+constexpr int kPairMaxTopk = 24;
+
 cudaError_t launch_fine(const FineArgs& a, cudaStream_t stream) {
-    if (!a.q_scale && !a.lin_image && a.g.d == 128) return launch_fine_pair(a, stream);
+    if (!a.q_scale && !a.lin_image && a.g.d == 128 && a.topk <= kPairMaxTopk) return launch_fine_pair(a, stream);
     return launch_fine_single(a, stream);
 }
 

@@ -250,9 +250,8 @@ __device__ void warp_topk(const unsigned long long* __restrict__ keys, const int
     }
 }
 
-// One warp per (b, head, i) row of a score matrix in global memory;
-// rows_per_cta warps per CTA (the path for grids whose score rows do not fit
-// the fused kernel's shared memory).
+// One warp per (b, head, i) row of the score matrix in global memory;
+// rows_per_cta warps per CTA.
 __global__ void __launch_bounds__(256)
 topk_kernel(const double* __restrict__ scores, const int nt, const int k, const long long rows,
             int32_t* __restrict__ idx) {
@@ -269,151 +268,10 @@ topk_kernel(const double* __restrict__ scores, const int nt, const int k, const 
     warp_topk(keys, nt, k, hist, idx + row * k, lane);
 }
 
-// ---------------------------------------------- fused coarse scores + top-k
-// One CTA per (b, head, block of R query cubes), 8 warps: the fp64 scores of
-// its rows against every key cube of the head are computed on the fp64 tensor
-// cores (mma.sync m8n8k4) and kept in shared memory as order-preserving keys;
-// each warp then selects the top-k of its rows with warp_topk.  No score
-// matrix goes through global memory.  Kp streams through shared memory in
-// slices of kSelChunk features of a kSelTile-key tile, kSelStages slices in
-// flight (cp.async); warp w scores keys 32w..32w+31 of a tile.  R = 16 rows
-// (two 8-row MMA tiles) when their score rows fit, 8 for longer rows.
-constexpr int kSelWarps = 8;
-constexpr int kSelTile = 32 * kSelWarps;         // key cubes per tile
-constexpr int kSelChunk = 16;                    // features per staged slice
-constexpr int kSelKs = kSelChunk + 2;            // doubles per staged key row (bank spread, 16-byte rows)
-constexpr int kSelStages = 3;
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
-    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-    const int n = valid ? 16 : 0;                // 0 source bytes: the 16 bytes are zero-filled
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(gsrc), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-size_t select_fused_smem_bytes(const Grid& g, int R) {
-    return (size_t)R * g.nt * 8                               // score keys
-           + (size_t)R * (g.d + 4) * 8                         // Qp rows
-           + (size_t)kSelStages * kSelTile * kSelKs * 8        // staged Kp slices
-           + (size_t)kSelWarps * 256 * 4;                      // per-warp histograms
-}
-
-// Rows per CTA of the fused kernel for this grid (16 or 8), or 0 when even
-// 8 score rows do not fit one SM's shared memory.
-int select_fused_rows(const Grid& g) {
-    const size_t cap = 227u * 1024u;
-    if (select_fused_smem_bytes(g, 16) <= cap) return 16;
-    if (select_fused_smem_bytes(g, 8) <= cap) return 8;
-    return 0;
-}
-
-template <int R>
-__global__ void __launch_bounds__(32 * kSelWarps, 1)
-select_fused_kernel(const double* __restrict__ qp, const double* __restrict__ kp, const Grid g,
-                    const double inv_sqrt_d, const int topk, int32_t* __restrict__ idx) {
-    constexpr int MT = R / 8;                                  // 8-row MMA tiles
-    extern __shared__ __align__(16) unsigned char sel_smem[];
-    const int nt = g.nt, d = g.d;
-    const int qs_stride = d + 4;
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(sel_smem);            // [R][nt]
-    double* qs = reinterpret_cast<double*>(keys + (size_t)R * nt);                          // [R][d + 4]
-    double* ks = qs + R * qs_stride;                                                        // [stages][tile][kSelKs]
-    unsigned int* hist = reinterpret_cast<unsigned int*>(ks + kSelStages * kSelTile * kSelKs);
-    const int bh = blockIdx.y;
-    const int i0 = blockIdx.x * R;
-    const double* Q = qp + (long long)bh * nt * d;
-    const double* K = kp + (long long)bh * nt * d;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int gr = lane >> 2, tq = lane & 3;                  // MMA fragment coordinates
-
-    // the block's query rows (zero past nt)
-    for (int l = tid; l < R * d / 2; l += blockDim.x) {
-        const int rr = l / (d / 2), cc = 2 * (l % (d / 2));
-        const double2 v = i0 + rr < nt ? *reinterpret_cast<const double2*>(Q + (long long)(i0 + rr) * d + cc)
-                                       : make_double2(0.0, 0.0);
-        *reinterpret_cast<double2*>(&qs[rr * qs_stride + cc]) = v;
-    }
-    const int n_tiles = (nt + kSelTile - 1) / kSelTile;
-    const int n_chunks = d / kSelChunk;
-    const int steps = n_tiles * n_chunks;
-    // slice s: tile s / n_chunks, features (s % n_chunks) * kSelChunk ..; 16 bytes per cp.async
-    auto stage = [&](int s) {
-        const int t = s / n_chunks, f0 = (s % n_chunks) * kSelChunk;
-        double* dst = ks + (s % kSelStages) * kSelTile * kSelKs;
-#pragma unroll
-        for (int e = 0; e < kSelTile * kSelChunk / 2 / (32 * kSelWarps); ++e) {
-            const int l = tid + 32 * kSelWarps * e;
-            const int kr = l / (kSelChunk / 2), cc = 2 * (l % (kSelChunk / 2));
-            const int j = t * kSelTile + kr;
-            const double* src = K + (long long)min(j, nt - 1) * d + f0 + cc;
-            cp_async16(dst + kr * kSelKs + cc, src, j < nt);
-        }
-        cp_async_commit();
-    };
-    double acc[MT][4][2];
-#pragma unroll
-    for (int a = 0; a < MT; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c][0] = acc[a][c][1] = 0.0;
-    stage(0);
-    if (steps > 1) stage(1);
-    for (int s = 0; s < steps; ++s) {
-        if (s + 2 < steps) {
-            stage(s + 2);
-            cp_async_wait<2>();
-        } else if (s + 1 < steps) {
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const double* kb = ks + (s % kSelStages) * kSelTile * kSelKs;
-        const int f0 = (s % n_chunks) * kSelChunk;
-#pragma unroll
-        for (int kk = 0; kk < kSelChunk / 4; ++kk) {
-            double a[MT], b[4];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) a[mt] = qs[(8 * mt + gr) * qs_stride + f0 + 4 * kk + tq];
-#pragma unroll
-            for (int n8 = 0; n8 < 4; ++n8) b[n8] = kb[(32 * warp + 8 * n8 + gr) * kSelKs + 4 * kk + tq];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int n8 = 0; n8 < 4; ++n8) dmma_8x8x4(acc[mt][n8][0], acc[mt][n8][1], a[mt], b[n8]);
-        }
-        if (s % n_chunks == n_chunks - 1) {
-            // the tile's scores are complete: store them as keys, restart
-            const int t = s / n_chunks;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int n8 = 0; n8 < 4; ++n8)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int j = t * kSelTile + 32 * warp + 8 * n8 + 2 * tq + e;
-                        if (j < nt) keys[(8 * mt + gr) * nt + j] = ordered_key(acc[mt][n8][e] * inv_sqrt_d);
-                        acc[mt][n8][e] = 0.0;
-                    }
-        }
-        __syncthreads();                                  // the slice's buffer is refilled next
-    }
-    // top-k of each row: warp w takes rows w, w + 8, ...
-    for (int rr = warp; rr < R; rr += kSelWarps) {
-        const int i = i0 + rr;
-        if (i >= nt) break;
-        warp_topk(keys + (size_t)rr * nt, nt, topk, hist + warp * 256, idx + ((long long)bh * nt + i) * topk, lane);
-    }
-}
-
 // ------------------------------------------------------------------ launchers
 
 size_t select_scratch_bytes(const Grid& g) {
     const size_t pooled = 2ull * g.B * g.heads * g.nt * g.d * sizeof(double);
-    if (select_fused_rows(g) > 0) return pooled;
-    // grids whose score rows exceed the fused kernel's shared memory keep
-    // the whole score matrix in the workspace
     const size_t scores = (size_t)g.B * g.heads * g.nt * g.nt * sizeof(double);
     return pooled + scores;
 }
@@ -435,23 +293,6 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const double* qp = pooled;
     const double* kp = pooled + (size_t)g.B * g.heads * g.nt * g.d;
-    const int R = select_fused_rows(g);
-    if (R > 0) {
-        const size_t smem = select_fused_smem_bytes(g, R);
-        const double inv_sqrt_d = 1.0 / sqrt((double)g.d);
-        if (R == 16) {
-            e = cudaFuncSetAttribute(select_fused_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            select_fused_kernel<16><<<dim3(ceil_div_i(g.nt, 16), g.B * g.heads), 32 * kSelWarps, smem, stream>>>(
-                qp, kp, g, inv_sqrt_d, a.topk, a.block_idx);
-        } else {
-            e = cudaFuncSetAttribute(select_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            select_fused_kernel<8><<<dim3(ceil_div_i(g.nt, 8), g.B * g.heads), 32 * kSelWarps, smem, stream>>>(
-                qp, kp, g, inv_sqrt_d, a.topk, a.block_idx);
-        }
-        return cudaGetLastError();
-    }
     const int tiles = ceil_div_i(g.nt, 64);
     coarse_kernel<<<dim3(tiles, tiles, g.B * g.heads), 128, 0, stream>>>(qp, kp, g, 1.0 / sqrt((double)g.d), scores);
     e = cudaGetLastError();

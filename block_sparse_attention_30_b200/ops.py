@@ -149,6 +149,18 @@ def vsa_sparse_attn_fwd_e4m3(q8, k8, q_scale, k_scale, v, block_idx, out, T, H, 
         workspace.data_ptr(), workspace.numel(), _stream(stream)))
 
 
+def vsa_sparse_linear_attn_fwd_e4m3(q8, k8, q_scale, k_scale, q, v, block_idx, lin_S, lin_z, out, T, H,
+                                    W, topk, workspace, tile=(4, 4, 4), stream=None):
+    """Fine pass with Q K^T in E4M3 plus the bf16 linear branch phi(q)S/(phi(q).z)
+    (lin_S, lin_z from vsa_linear_branch_fwd)."""
+    B, heads, d = _grid_of(v, T, H, W)
+    _lib.check("vsa_sparse_linear_attn_fwd_e4m3", _lib.lib().vsa_sparse_linear_attn_fwd_e4m3(
+        q8.data_ptr(), k8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(), q.data_ptr(),
+        v.data_ptr(), block_idx.data_ptr(), lin_S.data_ptr(), lin_z.data_ptr(), out.data_ptr(),
+        *_shape(B, heads, d, T, H, W, tile), topk, workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
+
+
 def vsa_device_status(workspace, stream=None) -> int:
     """Synchronise and return the device status code (0 = VSA_OK)."""
     return _lib.lib().vsa_device_status(workspace.data_ptr(), _stream(stream))

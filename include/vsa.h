@@ -86,10 +86,7 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
 /* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
  * for these shapes: a 256-byte status block followed by a scratch area that
  * holds either the selection's fp64 cube means of q and k
- * ([2][B][heads][nt][d]; the coarse scores stay in on-chip memory, except
- * for grids whose score rows do not fit one SM's shared memory eight at a
- * time, about nt > 1640 at d = 128, which also keep the fp64 scores
- * [B][heads][nt][nt] here), or the linear branch's operand image (B*heads*(4*d*d + 4*d)
+ * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the linear branch's operand image (B*heads*(4*d*d + 4*d)
  * bytes), whichever is larger (the backward passes' scratch fits it too: the
  * sparse branch's row terms and block-index transpose, the linear branch's
  * two operand images and fp32 gradient sums).  Returns 0 for invalid shapes.  The
@@ -121,9 +118,7 @@ vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int he
  * C[i][j] = Qp[i].Kp[j]/sqrt(d) in fp64 and writes, per (b, head, i), the
  * topk key cubes with the largest C (ties -> lower j) in ascending order to
  * block_idx.  1 <= topk <= nt.  Needs vsa_workspace_bytes() of workspace.
- * Two launches: the cube means, then one kernel that scores a block of 16
- * (or, for long rows, 8) query cubes against every key cube and selects
- * their top-k on chip. */
+ * Three launches: the cube means, the coarse scores, the top-k. */
 vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
                              int head_dim, int T, int H, int W, int tt, int th, int tw,
                              int topk, int32_t* block_idx, void* workspace,
@@ -232,7 +227,8 @@ vsa_status vsa_quantize_qk_e4m3(const vsa_bf16* q, const vsa_bf16* k, uint8_t* q
  * Q K^T on the tensor cores in E4M3 (fp32 accumulation), scores rescaled by
  * q_scale[query cube] * k_scale[key cube], softmax and P V as in the bf16
  * pass (bf16 P and v), output bf16 in grid order.  head_dim 128 only
- * (VSA_ERR_UNSUPPORTED otherwise); no linear branch.  Needs
+ * (VSA_ERR_UNSUPPORTED otherwise); the linear branch is added by
+ * vsa_sparse_linear_attn_fwd_e4m3 below.  Needs
  * vsa_workspace_bytes() of workspace (status word only). */
 vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
                                     const float* k_scale, const vsa_bf16* v,
@@ -240,6 +236,26 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
                                     int head_dim, int T, int H, int W, int tt, int th, int tw,
                                     int topk, void* workspace, size_t workspace_bytes,
                                     vsa_stream_t stream);
+
+/* Low-precision sparse + linear attention (SageSLA: SLA built on SageAttention's
+ * quantised products, TurboDiffusion article, section "稀疏、蒸馏与全链路量化"):
+ * vsa_sparse_attn_fwd_e4m3 plus the linear branch of vsa_sparse_attn_fwd,
+ *     out = softmax-pass(E4M3 Q K^T, bf16 P V) + phi(q) S / (phi(q) . z),
+ * with lin_S, lin_z from vsa_linear_branch_fwd (fp32) and phi(q) computed
+ * from the bf16 q (the quantisation covers the sparse branch's Q K^T only;
+ * the branch's products run as bf16 hi + lo pairs, fp32-level, as in
+ * vsa_sparse_attn_fwd).  q8, k8, q_scale, k_scale from vsa_quantize_qk_e4m3;
+ * q, v bf16 [B][N][heads][d].  head_dim 128 only (VSA_ERR_UNSUPPORTED
+ * otherwise).  All pointers 16-byte aligned (VSA_ERR_INVALID_ARGUMENT).
+ * Needs vsa_workspace_bytes() of workspace: the status word plus the
+ * operand image of (S, z) (VSA_ERR_WORKSPACE when smaller). */
+vsa_status vsa_sparse_linear_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
+                                           const float* k_scale, const vsa_bf16* q, const vsa_bf16* v,
+                                           const int32_t* block_idx, const float* lin_S,
+                                           const float* lin_z, vsa_bf16* out, int B, int heads,
+                                           int head_dim, int T, int H, int W, int tt, int th, int tw,
+                                           int topk, void* workspace, size_t workspace_bytes,
+                                           vsa_stream_t stream);
 
 /* Self-test of the device failure path (no counterpart on the pages): a
  * one-warp kernel waits on a barrier nobody arrives at, gives up after
@@ -263,16 +279,15 @@ vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
  * allocation, a fixed memory budget, an embedding without an allocator) and
  * so cannot provide vsa_select_blocks' workspace.  It computes exactly what
  * vsa_select_blocks computes, with the same kernels, but keeps the
- * intermediate fp64 cube means (and, for very large grids, coarse scores) in
- * one file-scope device array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved
- * on every GPU that loads the library until the process exits.  It allocates and frees nothing.
+ * intermediate fp64 cube means and coarse scores in one file-scope device
+ * array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved on every GPU that loads
+ * the library until the process exits.  It allocates and frees nothing.
  *
  *  - The caller still passes q, k (device, bf16 [B][N][heads][d]) and
  *    block_idx (device, int32 [B][heads][nt][topk]), 16-byte aligned.
- *  - Shapes whose intermediates exceed the array are rejected with
- *    VSA_ERR_WORKSPACE before anything is enqueued (the intermediates are the
- *    fp64 cube means, 2*B*heads*nt*d*8 bytes, plus B*heads*nt*nt*8 bytes of
- *    scores for grids beyond about nt = 1640 at d = 128); argument errors as
+ *  - Shapes whose intermediates exceed the array
+ *    (2*B*heads*nt*d*8 + B*heads*nt*nt*8 bytes > the maximum) are rejected
+ *    with VSA_ERR_WORKSPACE before anything is enqueued; argument errors as
  *    for vsa_select_blocks.
  *  - All calls share the array, which keeps the last call's contents; every
  *    call rewrites what it reads, so nothing needs clearing.  Calls that

@@ -55,16 +55,9 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_num_tiles(20, 28, 52, 4, 4, 4) == 455
     assert L.vsa_num_tiles(4, 32, 32, 4, 4, 4) == 64
     assert L.vsa_num_tiles(0, 4, 4, 4, 4, 4) == 0
-    # the selection keeps only the fp64 cube means in the workspace when 8 or
-    # 16 query cubes' score rows fit the fused kernel's shared memory (nt up
-    # to ~1640 at d = 128), the whole fp64 score matrix beyond
     nt, B, h, d = 455, 1, 40, 128
-    want = 256 + 2 * B * h * nt * d * 8
+    want = 256 + 2 * B * h * nt * d * 8 + B * h * nt * nt * 8
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 46) == want
-    nt = 1440                                                                 # 720P grid, ragged
-    assert L.vsa_workspace_bytes(B, h, d, 21, 45, 80, 4, 4, 4, 144) == 256 + 2 * B * h * nt * d * 8
-    nt = 2048                                                                 # 32 x 64 x 64: rows too long
-    assert L.vsa_workspace_bytes(1, 2, d, 32, 64, 64, 4, 4, 4, 8) == 256 + 2 * 2 * nt * d * 8 + 2 * nt * nt * 8
     assert L.vsa_workspace_bytes(B, h, 96, 20, 28, 52, 4, 4, 4, 46) == 0       # d unsupported
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 0) == 0         # topk < 1

@@ -362,12 +362,27 @@ def test_workload_fine_sampled(ops, name):
 
 
 def test_headline_fine_two_heads_full(ops):
-    """Full-size 14B-480P fine pass checked on every token of heads 0 and 1:
-    910 query cubes, so each persistent CTA walks several cube pairs and one
-    pair straddles the two heads (nt = 455 is odd)."""
+    """Full-size 14B-480P fine pass checked on every token of heads 0 and 1
+    (910 query cubes; nt = 455 is odd, so cube pairs of the persistent kernel
+    would straddle the two heads)."""
     w, q, k, v, qd, kd, vd = inputs("wan14b_480p")
     idx, ws = run_select(ops, w, qd, kd)
     out = run_fine(ops, w, qd, kd, vd, idx, ws)
+    hs = slice(0, 2)
+    sub = lambda x: x[:, :, hs].contiguous()
+    ref = O.fine(sub(q), sub(k), sub(v), idx[:, hs].cpu().numpy(), w.B, 2, w.head_dim,
+                 w.T, w.H, w.W, w.tile)
+    check_close(to_f64(out[:, :, hs]), ref)
+
+
+def test_short_rows_persistent_two_heads_full(ops):
+    """The 97 %-sparse shape (k = 11) without the linear branch, checked on
+    every token of heads 0 and 1: short rows run the persistent two-cube
+    kernel, whose CTAs each walk ~15 cube pairs at this size."""
+    w, q, k, v, qd, kd, vd = inputs("sparse97_linear_480p")
+    idx, ws = run_select(ops, w, qd, kd)
+    out = run_fine(ops, w, qd, kd, vd, idx, ws)            # no (S, z): sparse branch alone
+    assert not torch.isnan(out).any(), "every valid token must be written"
     hs = slice(0, 2)
     sub = lambda x: x[:, :, hs].contiguous()
     ref = O.fine(sub(q), sub(k), sub(v), idx[:, hs].cpu().numpy(), w.B, 2, w.head_dim,
@@ -743,6 +758,91 @@ def test_e4m3_headline_workload_sampled(ops):
         ok = slots[i] >= 0
         ref.append(part[r][ok])
         got.append(to_f64(out[0, torch.as_tensor(slots[i][ok]), head]))
+    check_close(np.concatenate(got), np.concatenate(ref))
+
+
+# ------------------------------------- low precision + linear branch (SageSLA)
+
+def run_e4m3_linear(ops, q, k, v, T, H, W, topk):
+    """Selection, E4M3 quantisation, linear state, then the E4M3 sparse pass
+    with the linear branch added."""
+    B, N, heads, d = q.shape
+    c = types.SimpleNamespace(T=T, H=H, W=W, topk=topk, tile=(4, 4, 4))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    idx, ws = run_select(ops, c, qd, kd)
+    nt = ops.vsa_num_tiles(T, H, W)
+    q8, k8 = (torch.zeros(q.shape, dtype=torch.uint8, device="cuda") for _ in range(2))
+    sq, sk = (torch.empty((B, heads, nt), dtype=torch.float32, device="cuda") for _ in range(2))
+    ops.vsa_quantize_qk_e4m3(qd, kd, q8, k8, sq, sk, T, H, W)
+    S = torch.empty((B, heads, d, d), dtype=torch.float32, device="cuda")
+    z = torch.empty((B, heads, d), dtype=torch.float32, device="cuda")
+    ops.vsa_linear_branch_fwd(kd, vd, S, z, T, H, W, ws)
+    out = torch.full_like(vd, float("nan"))
+    ops.vsa_sparse_linear_attn_fwd_e4m3(q8, k8, sq, sk, qd, vd, idx, S, z, out, T, H, W, topk, ws)
+    assert ops.vsa_device_status(ws) == 0
+    return idx, out
+
+
+@pytest.mark.parametrize("case", E4M3_CASES)
+def test_e4m3_linear_small_full(ops, case):
+    """SageSLA (TurboDiffusion article, section "稀疏、蒸馏与全链路量化"): the
+    E4M3 sparse pass plus the bf16 linear branch, every output element against
+    the oracle's fine pass on the dequantised q, k plus its linear branch on
+    the bf16 q, k, v (the bf16 bar), and against the exact oracle (fine pass on
+    bf16 q, k) within the stated E4M3 bound."""
+    B, T, H, W, heads, topk = case
+    q, k, v = synth.make_qkv(B, heads, 128, T, H, W, amplitude=0.7, seed=sum(case) + 3)
+    idx, out = run_e4m3_linear(ops, q, k, v, T, H, W, topk)
+    idx_np = idx.cpu().numpy()
+    N = T * H * W
+    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, 128, T, H, W)
+    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, 128, T, H, W)
+    qh = O.dequant_e4m3_cubes(cq, sq_ref, T, H, W)
+    kh = O.dequant_e4m3_cubes(ck, sk_ref, T, H, W)
+    Sr, zr = O.linear_state(k, v, B, heads, 128, N)
+    lin = O.linear_apply(q, Sr, zr, B, heads, 128, N)
+    got = to_f64(out)
+    assert not np.isnan(got).any()
+    check_close(got, O.fine_real(qh, kh, v, idx_np, B, heads, 128, T, H, W) + lin)
+    ref = O.fine(q, k, v, idx_np, B, heads, 128, T, H, W) + lin
+    err = np.abs(got - ref).max()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert err <= E4M3_MAX_REL * np.abs(ref).max() and rel <= E4M3_REL_FRO, (err, rel)
+
+
+def test_e4m3_linear_sparse97_sampled(ops):
+    """The 97 %-sparsity + linear-branch workload with E4M3 Q K^T: sampled query
+    cubes against the oracle on the dequantised q, k plus the linear branch on
+    bf16 q, k, v."""
+    w, q, k, v, qd, kd, vd = inputs("sparse97_linear_480p")
+    idx, out = run_e4m3_linear(ops, q, k, v, w.T, w.H, w.W, w.topk)
+    nt = w.num_tiles
+    rows = sample_rows(nt, w.heads, w.B, 12, seed=11, extra=ragged_class_rows(w, idx.cpu().numpy()))
+    heads_used = sorted({int(r) // nt % w.heads for r in rows})
+    b_used = sorted({int(r) // nt // w.heads for r in rows})
+    assert b_used == [0]
+    sub = lambda x: x[:, :, heads_used].contiguous()
+    hsub = len(heads_used)
+    cq, sq_ref = O.quant_e4m3_cubes(sub(q), 1, hsub, 128, w.T, w.H, w.W)
+    ck, sk_ref = O.quant_e4m3_cubes(sub(k), 1, hsub, 128, w.T, w.H, w.W)
+    qh = O.dequant_e4m3_cubes(cq, sq_ref, w.T, w.H, w.W)
+    kh = O.dequant_e4m3_cubes(ck, sk_ref, w.T, w.H, w.W)
+    Sr, zr = O.linear_state(sub(k), sub(v), 1, hsub, 128, w.N)
+    hmap = {h: j for j, h in enumerate(heads_used)}
+    srows = np.array([hmap[int(r) // nt] * nt + int(r) % nt for r in rows], np.int64)
+    idx_sub = idx[:, heads_used].cpu().numpy()
+    part = O.fine_tiles_real(qh, kh, sub(v), idx_sub, srows, 1, hsub, 128, w.T, w.H, w.W)
+    slots = O.tile_slots(w.T, w.H, w.W)
+    got, ref = [], []
+    for r, row in enumerate(rows):
+        head, i = divmod(int(row), nt)
+        ok = slots[i] >= 0
+        toks = slots[i][ok]
+        qrow = q[:, torch.as_tensor(toks), head:head + 1].contiguous()
+        j = hmap[head]
+        lin = O.linear_apply(qrow, Sr[:, j:j + 1], zr[:, j:j + 1], 1, 1, 128, len(toks))[0, :, 0]
+        ref.append(part[r][ok] + lin)
+        got.append(to_f64(out[0, torch.as_tensor(toks), head]))
     check_close(np.concatenate(got), np.concatenate(ref))
 
 

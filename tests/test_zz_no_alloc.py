@@ -51,7 +51,7 @@ def _select_both(L, w, seed):
 
 
 def test_noalloc_select_matches_workspace_select_twice(L):
-    w = WORKLOADS["wan1.3b_480p"]            # 9 MB of fp64 cube means: fits the array
+    w = WORKLOADS["wan1.3b_480p"]            # 21.6 MB of intermediates: fits the array
     for seed in (101, 202):                  # two calls in a row, different inputs
         ref, got = _select_both(L, w, seed)
         assert (ref >= 0).all()
@@ -59,7 +59,7 @@ def test_noalloc_select_matches_workspace_select_twice(L):
 
 
 def test_noalloc_select_rejects_shapes_beyond_the_array(L):
-    w = WORKLOADS["wan14b_480p"]             # 37 MB of fp64 cube means: too large
+    w = WORKLOADS["wan14b_480p"]             # 103 MB of intermediates: too large
     tt, th, tw = w.tile
     fake = 0x10000                           # never dereferenced: refused before launch
     code = L.vsa_select_blocks_noalloc(fake, fake, w.B, w.heads, w.head_dim, w.T, w.H, w.W,
