@@ -167,6 +167,7 @@ vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int he
     a.topk = topk;
     a.block_idx = block_idx;
     a.scratch = static_cast<uint8_t*>(workspace) + kStatusBytes;
+    a.status = static_cast<int*>(workspace);
     return from_cuda(vsa::launch_select(a, (cudaStream_t)stream));
 }
 

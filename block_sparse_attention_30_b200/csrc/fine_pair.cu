@@ -36,13 +36,16 @@
 //   gs % NS, lanes 16X; softmax writes P as bf16 over S; O += P V (A = P
 //   from TMEM, B = V MN-major).  S of step gs + NS is issued right after P V
 //   of step gs, so the softmax finds the next S ready.
-// Ring items are numbered 2 gs + X in load order; item i uses slot i % 3,
-// signals the slot's barrier of cube X (phase gs / 3) and is released by its
-// own cube's MMA completion: a K item by the commit of its S (s_full[X]), a
-// V item by the commit of its P V (o_ready[X]).  Per-step barriers come in
+// Ring items are numbered 2 gs + X in load order; item i uses slot i % R
+// (K: R = 4, so cube X owns slots X and X + 2 and each slot serves every
+// second step of its cube; V: R = 3, shared by the cubes in turn), signals
+// the slot's barrier of cube X (phase gs / 2 for K, gs / 3 for V) and is
+// released by its own cube's MMA completion: a K item by the commit of its S
+// (s_full[X]), a V item by the commit of its P V (o_ready[X]).  Per-step barriers come in
 // NS copies (step gs uses copy gs % NS) and each role observes a barrier's
 // phases in order, so every wait is for a phase that is neither overtaken
-// nor two phases ahead (a parity wait only tells the last two phases apart).  The softmax of step gs, for instance, may run while P V
+// nor two phases ahead (a parity wait only tells the last two phases
+// apart).  The softmax of step gs, for instance, may run while P V
 // of steps gs - 2 and gs - 1 are still pending (S of gs only implies P V of
 // gs - 3); with NS copies the copy it waits on has completed step gs - 1 - NS
 // already and cannot complete gs - 1 + NS before this softmax step is done.

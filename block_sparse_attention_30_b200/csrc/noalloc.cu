@@ -1,7 +1,7 @@
 // noalloc.cu -- block selection for callers that cannot allocate device memory.
 //
 // vsa_select_blocks needs a caller-allocated workspace for its intermediate
-// cube means and coarse scores.  Some callers cannot obtain one: code that
+// work counters and cube means.  Some callers cannot obtain one: code that
 // runs where cudaMalloc is not permitted or not wanted (inside a framework
 // callback that forbids allocation, behind a fixed memory budget, or in an
 // embedding that has no allocator of its own).  For them this file keeps the
@@ -14,7 +14,8 @@
 //  * Shapes whose intermediates do not fit are rejected with
 //    VSA_ERR_WORKSPACE before anything is enqueued.
 //  * Every call shares the array and it keeps the last call's contents; each
-//    call writes all the bytes it later reads, so nothing needs clearing.
+//    call clears the selection kernel's work counters (a memset it enqueues)
+//    and writes all the other bytes it later reads.
 //    Calls whose work overlaps on the GPU (different streams, or different
 //    host threads without ordering) race on the array and may produce wrong
 //    indices: order them on one stream.
@@ -115,6 +116,7 @@ vsa_status vsa_select_blocks_noalloc(const vsa_bf16* q, const vsa_bf16* k, int B
     a.topk = topk;
     a.block_idx = block_idx;
     a.scratch = scratch;
+    a.status = nullptr;        // no caller-visible status word (see the header)
     return vsa::launch_select(a, (cudaStream_t)stream) == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

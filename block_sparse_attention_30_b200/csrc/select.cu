@@ -6,24 +6,60 @@
 // scores Qp[i].Kp[j]/sqrt(d), top-k per query cube, ties to the lower cube id,
 // indices emitted ascending) is this library's reading of that outline.
 //
-// Three HBM-friendly kernels, all in fp64 so the chosen cubes match an exact
-// evaluation except for genuine ties:
-//   pool_kernel    one CTA per (cube, batch, q|k): 16-byte vector loads of the
-//                  cube's valid token rows (all heads at once), fp64 sums,
-//                  divide by the valid count -> pooled [2][B][heads][nt][d].
-//   coarse_kernel  per (b, head) a 64x64 tile of C = Qp Kp^T / sqrt(d) on the
-//                  fp64 tensor cores -> scores [B][heads][nt][nt].
-//   topk_kernel    one warp per score row: 8-pass MSD radix select on
-//                  order-preserving 64-bit keys finds the k-th largest score,
-//                  then a ballot sweep in ascending j emits the kept cubes
-//                  (equal keys taken lowest j first).
+// One persistent kernel, select_kernel, does the whole selection.  Its CTAs
+// claim work items from an atomic counter, per group of up to 8 heads:
+//   pool items   one per (cubes j0 .. j0 + cpi - 1, batch, q|k) of the group:
+//                16-byte vector loads of the cubes' valid token rows (the
+//                group's heads, contiguous within a token row), fp64 sums,
+//                divide by the valid count; the mean is stored as an fp32
+//                pair hi + lo (hi = RN(mean), lo = RN(mean - hi), together
+//                within 2^-48 of the fp64 mean) -> pooled [2][2][B][heads][nt][d].
+//   score items  one per (b, head, block of 16 query cubes): the coarse
+//                scores of the 16 rows against all nt key cubes,
+//                C = Qp Kp^T / sqrt(d), in fp32 (packed fp32x2 FMA, the 16
+//                rows' Qp in shared memory, four key cubes per lane, the
+//                features split over two warps) into shared memory -- the nt x nt
+//                score matrix never reaches HBM -- then per row (one warp)
+//                the exact top-k:
+//                  1. a bracket [lo, hi] around the k-th largest fp32 score
+//                     (two levels of 256 value bins, about 1/65536 of the
+//                     row's range wide);
+//                  2. every score above hi + 2 eps is kept, every score
+//                     below lo - 2 eps dropped, where eps bounds the fp32
+//                     error of a score (forward error of a d-term fp32 dot
+//                     product: (d + 8) 2^-24 |Qp_i| max_j |Kp_j| / sqrt(d),
+//                     doubled);
+//                  3. the few scores in between are recomputed in fp64 from
+//                     hi + lo and ranked (larger first, then lower cube id)
+//                     for the remaining places (more than 64 of them, e.g.
+//                     exact ties: fp64 keys for the whole row and a 64-bit
+//                     radix select);
+//                  4. a ballot sweep in ascending j writes the kept cubes.
+//                Since every fp32 score is within eps of its fp64 value, the
+//                kept set is the one the fp64 scores give, up to the rounding
+//                of the fp64 dot products themselves.
+// Claim order P_0, P_1, S_0, P_2, S_1, ... (pool and score items of head
+// group g): the pooling of the next group (HBM bound) runs while the current
+// group is scored (compute bound).  A score item waits for its group's pool
+// items with a bounded spin on the group's counter; items are claimed in
+// order, so every pool item it needs is held by a running CTA that never
+// waits, and the wait ends without any assumption about which CTAs are
+// resident.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "select.h"
+#include "sm100.cuh"
 
 namespace vsa {
+
+constexpr int kSelThreads = 256;                 // 8 warps
+constexpr int kSelRows = 16;                     // query cubes per score item
+constexpr int kSelMaxCand = 64;                  // fp64-refined candidates per row (fast path)
+constexpr int kSelMaxCtas = 1024;                // grid bound (fallback scratch rows)
 
 // ------------------------------------------------------------------ pooling
 
@@ -36,20 +72,28 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 raw) {
     }
 }
 
-__global__ void __launch_bounds__(320)
-pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g,
-            double* __restrict__ pooled) {
-    const int j = blockIdx.x, b = blockIdx.y, which = blockIdx.z;
+// Means of cubes j0 .. j0 + cpi - 1 (those < nt) of batch b of q (which = 0)
+// or k (which = 1), heads h0 .. h0 + nh - 1, written as fp32 hi + lo into
+// pooled[which][0|1][b][head][j][d].  Thread t takes (cube, 16-byte vector)
+// pairs t, t + 256, ...
+__device__ void pool_item(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid& g,
+                          const int j0, const int cpi, const int b, const int which, const int h0, const int nh,
+                          float* __restrict__ pooled) {
     const uint16_t* x = which ? k : q;
-    const int it = j / (g.nh * g.nw), ih = (j / g.nw) % g.nh, iw = j % g.nw;
-    const int t0 = it * g.tt, h0 = ih * g.th, w0 = iw * g.tw;
-    const int vt = min(g.tt, g.T - t0), vh = min(g.th, g.H - h0), vw = min(g.tw, g.W - w0);
-    const double count = (double)(vt * vh * vw);
     const int row_elems = g.heads * g.d;              // one token: all heads
-    const int nvec = row_elems / 8;
-    const bool full444 = vt == 4 && vh == 4 && vw == 4 && g.tt == 4 && g.th == 4 && g.tw == 4;
-    double* out = pooled + ((long long)which * g.B + b) * g.heads * (long long)g.nt * g.d;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    const int nvec = nh * g.d / 8;                    // per cube: heads h0 .. h0 + nh - 1
+    const uint16_t* xg = x + (long long)h0 * g.d;
+    const long long plane = (long long)g.B * g.heads * g.nt * g.d;
+    float* hi = pooled + (2ll * which) * plane + (long long)b * g.heads * g.nt * g.d;
+    float* lo = hi + plane;
+    for (int u = threadIdx.x; u < cpi * nvec; u += blockDim.x) {
+        const int j = j0 + u / nvec, v = u % nvec;
+        if (j >= g.nt) break;
+        const int it = j / (g.nh * g.nw), ih = (j / g.nw) % g.nh, iw = j % g.nw;
+        const int t0 = it * g.tt, h0c = ih * g.th, w0 = iw * g.tw;
+        const int vt = min(g.tt, g.T - t0), vh = min(g.th, g.H - h0c), vw = min(g.tw, g.W - w0);
+        const double count = (double)(vt * vh * vw);
+        const bool full444 = vt == 4 && vh == 4 && vw == 4 && g.tt == 4 && g.th == 4 && g.tw == 4;
         double acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0;
@@ -59,8 +103,8 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, cons
                 uint4 raw[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    const long long n = ((long long)(t0 + dt) * g.H + (h0 + (r >> 2))) * g.W + w0 + (r & 3);
-                    raw[r] = __ldg(reinterpret_cast<const uint4*>(x + ((long long)b * g.N + n) * row_elems) + v);
+                    const long long n = ((long long)(t0 + dt) * g.H + (h0c + (r >> 2))) * g.W + w0 + (r & 3);
+                    raw[r] = __ldg(reinterpret_cast<const uint4*>(xg + ((long long)b * g.N + n) * row_elems) + v);
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) add_bf16x8(acc, raw[r]);
@@ -68,91 +112,24 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, cons
         } else {
             for (int dt = 0; dt < vt; ++dt)
                 for (int dh = 0; dh < vh; ++dh) {
-                    const long long n0 = ((long long)(t0 + dt) * g.H + (h0 + dh)) * g.W + w0;
-                    const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)b * g.N + n0) * row_elems) + v;
-                    for (int dw = 0; dw < vw; ++dw) add_bf16x8(acc, __ldg(src + (long long)dw * nvec));
+                    const long long n0 = ((long long)(t0 + dt) * g.H + (h0c + dh)) * g.W + w0;
+                    const uint4* src = reinterpret_cast<const uint4*>(xg + ((long long)b * g.N + n0) * row_elems) + v;
+                    for (int dw = 0; dw < vw; ++dw) add_bf16x8(acc, __ldg(src + (long long)dw * (row_elems / 8)));
                 }
         }
-        const int e0 = v * 8, head = e0 / g.d, c0 = e0 % g.d;
-        double* dst = out + ((long long)head * g.nt + j) * g.d + c0;
+        const int e0 = v * 8, head = h0 + e0 / g.d, c0 = e0 % g.d;
+        const long long off = ((long long)head * g.nt + j) * g.d + c0;
+        float h8[8], l8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst[e] = acc[e] / count;
-    }
-}
-
-// ------------------------------------------------------------ coarse scores
-// C[i][j] = (sum_c Qp[i][c] Kp[j][c]) / sqrt(d), per (b, head), in fp64 on
-// the fp64 tensor cores (mma.sync m8n8k4, exact products, fp64 accumulation;
-// tcgen05 has no fp64 kind).  64x64 tiles of C per CTA, 4 warps of 32x32
-// (4x4 MMA tiles), operands staged 32 features at a time in shared memory.
-// The summation order differs from a sequential dot product only at the fp64
-// rounding level, far inside the near-tie tolerance of the selection.
-__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
-    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                 : "+d"(d0), "+d"(d1)
-                 : "d"(a), "d"(b));
-}
-
-constexpr int kCoarseChunk = 32;                 // features staged per step
-constexpr int kCoarseStride = kCoarseChunk + 4;  // doubles per smem row: 8-byte loads of a
-                                                 // half-warp (4 rows x 4 features) hit distinct banks
-
-__global__ void __launch_bounds__(128)
-coarse_kernel(const double* __restrict__ qp, const double* __restrict__ kp, const Grid g,
-              const double inv_sqrt_d, double* __restrict__ scores) {
-    __shared__ __align__(16) double As[64 * kCoarseStride];
-    __shared__ __align__(16) double Bs[64 * kCoarseStride];
-    const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
-    const int nt = g.nt, d = g.d;
-    const double* Q = qp + (long long)bh * nt * d;
-    const double* K = kp + (long long)bh * nt * d;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wm = warp >> 1, wn = warp & 1;         // warp tile: rows 32*wm.., cols 32*wn..
-    const int gr = lane >> 2, tq = lane & 3;         // MMA fragment coordinates
-    double acc[4][4][2];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c][0] = acc[a][c][1] = 0.0;
-    for (int e0 = 0; e0 < d; e0 += kCoarseChunk) {
-        // 64 rows x 32 features of each operand, 16-byte loads, zero rows past nt
-        for (int l = threadIdx.x; l < 64 * kCoarseChunk / 2; l += 128) {
-            const int rr = l / (kCoarseChunk / 2), cc = 2 * (l % (kCoarseChunk / 2));
-            const double2 qa = i0 + rr < nt ? *reinterpret_cast<const double2*>(Q + (long long)(i0 + rr) * d + e0 + cc)
-                                            : make_double2(0.0, 0.0);
-            const double2 kb = j0 + rr < nt ? *reinterpret_cast<const double2*>(K + (long long)(j0 + rr) * d + e0 + cc)
-                                            : make_double2(0.0, 0.0);
-            *reinterpret_cast<double2*>(&As[rr * kCoarseStride + cc]) = qa;
-            *reinterpret_cast<double2*>(&Bs[rr * kCoarseStride + cc]) = kb;
+        for (int e = 0; e < 8; ++e) {
+            const double m = acc[e] / count;
+            h8[e] = (float)m;
+            l8[e] = (float)(m - (double)h8[e]);
         }
-        __syncthreads();
-#pragma unroll
-        for (int ks = 0; ks < kCoarseChunk / 4; ++ks) {
-            double a[4], b[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                a[t] = As[(32 * wm + 8 * t + gr) * kCoarseStride + 4 * ks + tq];   // A[row][k]
-                b[t] = Bs[(32 * wn + 8 * t + gr) * kCoarseStride + 4 * ks + tq];   // B[k][col] = Kp[col][k]
-            }
-#pragma unroll
-            for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-                for (int ct = 0; ct < 4; ++ct) dmma_8x8x4(acc[rt][ct][0], acc[rt][ct][1], a[rt], b[ct]);
-        }
-        __syncthreads();
-    }
-    double* S = scores + (long long)bh * nt * nt;
-#pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-        const int ii = i0 + 32 * wm + 8 * rt + gr;
-        if (ii >= nt) continue;
-#pragma unroll
-        for (int ct = 0; ct < 4; ++ct) {
-            const int jj = j0 + 32 * wn + 8 * ct + 2 * tq;
-            if (jj < nt) S[(long long)ii * nt + jj] = acc[rt][ct][0] * inv_sqrt_d;
-            if (jj + 1 < nt) S[(long long)ii * nt + jj + 1] = acc[rt][ct][1] * inv_sqrt_d;
-        }
+        reinterpret_cast<float4*>(hi + off)[0] = make_float4(h8[0], h8[1], h8[2], h8[3]);
+        reinterpret_cast<float4*>(hi + off)[1] = make_float4(h8[4], h8[5], h8[6], h8[7]);
+        reinterpret_cast<float4*>(lo + off)[0] = make_float4(l8[0], l8[1], l8[2], l8[3]);
+        reinterpret_cast<float4*>(lo + off)[1] = make_float4(l8[4], l8[5], l8[6], l8[7]);
     }
 }
 
@@ -163,10 +140,10 @@ __device__ __forceinline__ unsigned long long ordered_key(double x) {
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// Top-k of one row of nt order-preserving keys in shared memory, by one warp
-// (hist: 256 bins of this warp's own): MSD radix select of the k-th largest
-// key, then the kept indices in ascending order (equal keys lowest j first)
-// written to out[0..k).
+// Top-k of one row of nt order-preserving 64-bit keys, by one warp (hist:
+// 256 shared-memory bins of this warp's own): MSD radix select of the k-th
+// largest key, then the kept indices in ascending order (equal keys lowest j
+// first) written to out[0..k).
 __device__ void warp_topk(const unsigned long long* __restrict__ keys, const int nt, const int k,
                           unsigned int* __restrict__ hist, int32_t* __restrict__ out, const int lane) {
     // Skip the leading bytes every key shares (for scores of one magnitude
@@ -250,62 +227,514 @@ __device__ void warp_topk(const unsigned long long* __restrict__ keys, const int
     }
 }
 
-// One warp per (b, head, i) row of the score matrix in global memory;
-// rows_per_cta warps per CTA.
-__global__ void __launch_bounds__(256)
-topk_kernel(const double* __restrict__ scores, const int nt, const int k, const long long rows,
-            int32_t* __restrict__ idx) {
-    extern __shared__ unsigned long long tk_smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
-    const long long row = (long long)blockIdx.x * nwarps + warp;
-    unsigned long long* keys = tk_smem + (long long)warp * nt;
-    unsigned int* hist = reinterpret_cast<unsigned int*>(tk_smem + (long long)nwarps * nt) + warp * 256;
-    if (row >= rows) return;                          // whole warp leaves together
-    const double* src = scores + row * nt;
-    for (int j = lane; j < nt; j += 32) keys[j] = ordered_key(src[j]);
+
+// In a warp's 256-bin histogram (counts in descending bin order = descending
+// values), the bin holding the remaining-th largest value: its index and the
+// count of all higher bins.
+__device__ __forceinline__ void warp_hist_pick(const unsigned int* __restrict__ hist, const int remaining,
+                                               const int lane, int& bin, int& above) {
+    int cnt[8], lsum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { cnt[e] = (int)hist[255 - 8 * lane - e]; lsum += cnt[e]; }
+    int incl = lsum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const unsigned ball = __ballot_sync(0xffffffffu, incl >= remaining);
+    const int owner = ball ? __ffs(ball) - 1 : 31;
+    int b = 0, a = 0;
+    if (lane == owner) {
+        int run = incl - lsum;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (run + cnt[e] >= remaining) { b = 255 - 8 * lane - e; a = run; break; }
+            run += cnt[e];
+        }
+    }
+    bin = __shfl_sync(0xffffffffu, b, owner);
+    above = __shfl_sync(0xffffffffu, a, owner);
+}
+
+// Bin index 0..255 of x in [0, 256]: x rounded to an integer by the fp32
+// adder (add 1.5 * 2^23 and read the low mantissa bits), non-decreasing in x,
+// on the FMA/ALU pipes rather than a float-to-int conversion.
+__device__ __forceinline__ int bin256(float x) {
+    const int n = __float_as_int((x - 0.5f) + 12582912.f) - 0x4B400000;
+    return min(255, max(0, n));
+}
+
+// A bracket [lo, hi] that holds the k-th largest of the nt fp32 values
+// row[0..nt) (shared memory), by one warp: two levels of 256 equal-width
+// value bins over [min, max] (x = (s - min) * 256 / (max - min), bin
+// round(x - 1/2) clamped to 0..255, level 2 the same on 256 (x - t1) within
+// bin t1; both non-decreasing in s, so the k-th largest value lies in the
+// chosen bins), so the bracket is about (max - min) / 65536 wide: bin t1, t2
+// holds x in [t1 + t2 / 256, t1 + (t2 + 1) / 256] up to the rounding of x
+// (3.1 ulp relative, at most 3.2 * 2^-24 * (max - min) in s); the bracket is
+// widened by 8 * 2^-24 * (|min| + |max| + max - min).
+__device__ void warp_bracket(const float* __restrict__ row, const int nt, const int k,
+                             unsigned int* __restrict__ hist, const int lane, double& lo, double& hi) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int j0 = 0; j0 < nt; j0 += 128) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 32 * u + lane;
+            if (j < nt) { const float v = row[j]; mn = fminf(mn, v); mx = fmaxf(mx, v); }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    if (!(mx - mn > 1e-30f)) { lo = mn; hi = mx; return; }      // (nearly) one value
+    const float sc1 = 256.f / (mx - mn);
+    // level 1
+    for (int h = lane; h < 256; h += 32) hist[h] = 0;
     __syncwarp();
-    warp_topk(keys, nt, k, hist, idx + row * k, lane);
+    for (int j0 = 0; j0 < nt; j0 += 128) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 32 * u + lane;
+            if (j < nt) atomicAdd(&hist[bin256((row[j] - mn) * sc1)], 1u);
+        }
+    }
+    __syncwarp();
+    int t1, above1;
+    warp_hist_pick(hist, k, lane, t1, above1);
+    __syncwarp();
+    // level 2: the values in bin t1
+    for (int h = lane; h < 256; h += 32) hist[h] = 0;
+    __syncwarp();
+    for (int j0 = 0; j0 < nt; j0 += 128) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 32 * u + lane;
+            if (j < nt) {
+                const float x = (row[j] - mn) * sc1;
+                if (bin256(x) == t1) atomicAdd(&hist[bin256((x - (float)t1) * 256.f)], 1u);
+            }
+        }
+    }
+    __syncwarp();
+    int t2, above2;
+    warp_hist_pick(hist, k - above1, lane, t2, above2);
+    __syncwarp();
+    const double w1 = ((double)mx - (double)mn) / 256.0;
+    const double margin = 8.0 * 0x1p-24 * (fabs((double)mn) + fabs((double)mx) + ((double)mx - (double)mn));
+    lo = (double)mn + ((double)t1 + t2 / 256.0) * w1 - margin;
+    hi = (double)mn + ((double)t1 + (t2 + 1) / 256.0) * w1 + margin;
+}
+
+// fp64 coarse scores against one query cube row, by one warp: lane l holds
+// features fpl*l .. fpl*l + fpl - 1 (fpl = d / 32) of the row as fp64
+// (hi + lo); score(j) sums its lane's products in feature order and the 32
+// lane partials in a butterfly; the same value on every lane.
+struct RowF64 {
+    double q[4];
+    int fpl;
+    __device__ void load(const float* __restrict__ qh, const float* __restrict__ ql, int d, int lane) {
+        fpl = d / 32;
+        const int c = lane * fpl;
+        if (fpl == 4) {
+            const float4 h = __ldcg(reinterpret_cast<const float4*>(qh + c)), l = __ldcg(reinterpret_cast<const float4*>(ql + c));
+            q[0] = (double)h.x + l.x; q[1] = (double)h.y + l.y; q[2] = (double)h.z + l.z; q[3] = (double)h.w + l.w;
+        } else {
+            const float2 h = __ldcg(reinterpret_cast<const float2*>(qh + c)), l = __ldcg(reinterpret_cast<const float2*>(ql + c));
+            q[0] = (double)h.x + l.x; q[1] = (double)h.y + l.y; q[2] = q[3] = 0.0;
+        }
+    }
+    // this lane's partial of key cube row (kh, kl)
+    __device__ double partial(const float* __restrict__ kh, const float* __restrict__ kl, int lane) const {
+        const int c = lane * fpl;
+        if (fpl == 4) {
+            const float4 h = __ldcg(reinterpret_cast<const float4*>(kh + c)), l = __ldcg(reinterpret_cast<const float4*>(kl + c));
+            double s = q[0] * ((double)h.x + l.x);
+            s = fma(q[1], (double)h.y + l.y, s);
+            s = fma(q[2], (double)h.z + l.z, s);
+            return fma(q[3], (double)h.w + l.w, s);
+        }
+        const float2 h = __ldcg(reinterpret_cast<const float2*>(kh + c)), l = __ldcg(reinterpret_cast<const float2*>(kl + c));
+        return fma(q[1], (double)h.y + l.y, q[0] * ((double)h.x + l.x));
+    }
+};
+
+__device__ __forceinline__ double warp_sum_f64(double s) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s;
+}
+
+__device__ __forceinline__ unsigned long long f64_key(double x) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(x);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+struct SelShared {
+    int item;
+    int ready;                  // the current item's pooling is done (1) or timed out (-1)
+    int lock;                   // fallback scratch row of this CTA
+    float kmax2[2];             // max_j of |Kp_j|^2 over each half of the features
+};
+
+// Dynamic shared memory of a score item: SelShared, Qp^T [d][16] fp32, the
+// scores [16][ntp] fp32, per warp 256 histogram bins and kSelMaxCand
+// candidates (cube id + fp64 score).
+__host__ __device__ inline int sel_ntp(int nt) { return (nt + 3) & ~3; }
+__host__ __device__ inline size_t sel_smem_bytes(int nt, int d) {
+    return 128 + (size_t)d * kSelRows * 4 + (size_t)kSelRows * sel_ntp(nt) * 4 +
+           (kSelThreads / 32) * (256 * 4 + kSelMaxCand * 12);
+}
+
+__device__ void score_item(const Grid& g, const int topk, const int item, const float* __restrict__ pooled,
+                           unsigned long long* __restrict__ fallback, int32_t* __restrict__ idx,
+                           uint8_t* smem, int* status) {
+    SelShared* sh = reinterpret_cast<SelShared*>(smem);
+    const int d = g.d, nt = g.nt, ntp = sel_ntp(nt);
+    float* sQ = reinterpret_cast<float*>(smem + 128);                   // [d][16]
+    float* sc = sQ + d * kSelRows;                                       // [16][ntp]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int kWarps = kSelThreads / 32;
+    unsigned int* hist_all = reinterpret_cast<unsigned int*>(sc + kSelRows * ntp);   // [8][256]
+    double* cs_all = reinterpret_cast<double*>(hist_all + kWarps * 256);            // [8][64]
+    int* ci_all = reinterpret_cast<int*>(cs_all + kWarps * kSelMaxCand);            // [8][64]
+    unsigned int* hist = hist_all + warp * 256;
+    double* cs = cs_all + warp * kSelMaxCand;
+    int* ci = ci_all + warp * kSelMaxCand;
+    const int rblocks = ceil_div_i(nt, kSelRows);
+    const int bh = item / rblocks, i0 = (item % rblocks) * kSelRows;
+    const long long plane = (long long)g.B * g.heads * nt * d;
+    const float* Qh = pooled + (long long)bh * nt * d;                   // q hi
+    const float* Ql = Qh + plane;                                        // q lo
+    const float* Kh = pooled + 2 * plane + (long long)bh * nt * d;       // k hi
+    const float* Kl = Kh + plane;                                        // k lo
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    const float inv_sqrt_d_f = (float)inv_sqrt_d;
+
+    // Qp hi of the 16 rows, transposed (rows past nt are zero)
+    for (int e = tid; e < kSelRows * d; e += kSelThreads) {
+        const int r = e / d, c = e % d;
+        sQ[c * kSelRows + r] = i0 + r < nt ? __ldcg(Qh + (long long)(i0 + r) * d + c) : 0.f;
+    }
+    if (tid == 0) sh->kmax2[0] = sh->kmax2[1] = 0.f;
+    __syncthreads();
+
+    // ---- coarse scores, fp32: each lane four key cubes and all 16 rows
+    // (acc[b][p] holds rows 2p, 2p+1 of key b; one packed fp32x2 FMA per row
+    // pair); warps w and w + 4 take the two halves of the features of the
+    // same 128 keys, each half summed in feature order, and the two partial
+    // sums meet in shared memory (C = (half 0 + half 1) / sqrt(d)).
+    const int half = warp >> 2, kw = warp & 3, dh = d / 2, c0 = half * dh;
+    const int passes = ceil_div_i(nt, 512);
+    float kmax2 = 0.f;                                    // max_j of this half's |Kp_j|^2
+    for (int ps = 0; ps < passes; ++ps) {
+        const int j0 = ps * 512 + kw * 128 + 4 * lane;
+        const float* kbase = Kh + (long long)j0 * d + c0;
+        uint64_t acc[4][kSelRows / 2];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int p = 0; p < kSelRows / 2; ++p) acc[b][p] = 0ull;
+        float nrm[4] = {0.f, 0.f, 0.f, 0.f};
+        float4 cur[4];
+        for (int dc = 0; dc < dh; dc += 4) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                cur[b] = j0 + b < nt ? __ldcg(reinterpret_cast<const float4*>(kbase + (long long)b * d + dc))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4* qq = reinterpret_cast<const float4*>(sQ + (c0 + dc + c) * kSelRows);
+                uint64_t kd[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float kv = c == 0 ? cur[b].x : c == 1 ? cur[b].y : c == 2 ? cur[b].z : cur[b].w;
+                    nrm[b] = fmaf(kv, kv, nrm[b]);
+                    kd[b] = f32x2(kv, kv);
+                }
+#pragma unroll
+                for (int p4 = 0; p4 < kSelRows / 4; ++p4) {
+                    const float4 q4 = qq[p4];
+                    const uint64_t qlo = f32x2(q4.x, q4.y), qhi = f32x2(q4.z, q4.w);
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        acc[b][2 * p4] = fma_f32x2(qlo, kd[b], acc[b][2 * p4]);
+                        acc[b][2 * p4 + 1] = fma_f32x2(qhi, kd[b], acc[b][2 * p4 + 1]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            if (j0 + b < nt) kmax2 = fmaxf(kmax2, nrm[b]);
+        if (half == 0) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (j0 + b >= nt) continue;
+#pragma unroll
+                for (int p = 0; p < kSelRows / 2; ++p) {
+                    float r0, r1;
+                    unf32x2(acc[b][p], r0, r1);
+                    sc[(2 * p) * ntp + j0 + b] = r0;
+                    sc[(2 * p + 1) * ntp + j0 + b] = r1;
+                }
+            }
+        }
+        __syncthreads();
+        if (half == 1) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (j0 + b >= nt) continue;
+#pragma unroll
+                for (int p = 0; p < kSelRows / 2; ++p) {
+                    float r0, r1;
+                    unf32x2(acc[b][p], r0, r1);
+                    float* c0p = sc + (2 * p) * ntp + j0 + b;
+                    float* c1p = sc + (2 * p + 1) * ntp + j0 + b;
+                    *c0p = (*c0p + r0) * inv_sqrt_d_f;
+                    *c1p = (*c1p + r1) * inv_sqrt_d_f;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kmax2 = fmaxf(kmax2, __shfl_xor_sync(0xffffffffu, kmax2, off));
+    if (lane == 0) atomicMax(reinterpret_cast<int*>(&sh->kmax2[half]), __float_as_int(kmax2));   // >= 0: int order
+    __syncthreads();
+
+    // ---- per row (one warp each): exact top-k
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int r = warp; r < kSelRows; r += kSelThreads / 32) {
+        const int i = i0 + r;
+        if (i >= nt) break;
+        float* row = sc + r * ntp;
+        int32_t* out = idx + ((long long)bh * nt + i) * topk;
+        if (topk == nt) {                                   // every cube kept
+            for (int j = lane; j < nt; j += 32) out[j] = j;
+            continue;
+        }
+        float qn2 = 0.f;
+        for (int c = lane; c < d; c += 32) qn2 = fmaf(sQ[c * kSelRows + r], sQ[c * kSelRows + r], qn2);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) qn2 += __shfl_xor_sync(0xffffffffu, qn2, off);
+        // bound on |fp32 score - fp64 score|, doubled, plus an absolute term
+        // for products in the subnormal range
+        // (max_j |Kp_j|^2 <= the sum of the two halves' maxima)
+        const double eps = 2.0 * (d + 8) * 0x1p-24 *
+                           sqrt((double)qn2 * ((double)sh->kmax2[0] + (double)sh->kmax2[1])) * 1.0001 * inv_sqrt_d + 1e-30;
+        double blo, bhi;
+        warp_bracket(row, nt, topk, hist, lane, blo, bhi);
+        // every score above hi is kept, every score below lo dropped: fp32
+        // thresholds rounded outward from the bracket widened by 2 eps
+        const float hi = __double2float_ru(bhi + 2.0 * eps), lo = __double2float_rd(blo - 2.0 * eps);
+        int above = 0, nc = 0;
+        for (int j0 = 0; j0 < nt; j0 += 32) {
+            const int j = j0 + lane;
+            const float v = j < nt ? row[j] : -INFINITY;
+            const bool gt = v > hi, band = j < nt && !gt && v >= lo;
+            above += __popc(__ballot_sync(0xffffffffu, gt));
+            const unsigned bb = __ballot_sync(0xffffffffu, band);
+            const int pos = nc + __popc(bb & lt_mask);
+            if (band && pos < kSelMaxCand) ci[pos] = j;
+            nc += __popc(bb);
+        }
+        const int need = topk - above;                      // 1 <= need <= nc
+        RowF64 qrow;
+        qrow.load(Qh + (long long)i * d, Ql + (long long)i * d, d, lane);
+        if (nc <= kSelMaxCand) {
+            __syncwarp();
+            for (int c = 0; c < nc; c += 2) {               // two candidates' loads in flight
+                const int ja = ci[c], jb = c + 1 < nc ? ci[c + 1] : ja;
+                const double pa = qrow.partial(Kh + (long long)ja * d, Kl + (long long)ja * d, lane);
+                const double pb = qrow.partial(Kh + (long long)jb * d, Kl + (long long)jb * d, lane);
+                const double sa = warp_sum_f64(pa) * inv_sqrt_d, sb = warp_sum_f64(pb) * inv_sqrt_d;
+                if (lane == 0) { cs[c] = sa; if (c + 1 < nc) cs[c + 1] = sb; }
+            }
+            __syncwarp();
+            for (int c = lane; c < nc; c += 32) {
+                const double s = cs[c];
+                const int j = ci[c];
+                int rank = 0;
+                for (int o = 0; o < nc; ++o) rank += (cs[o] > s || (cs[o] == s && ci[o] < j)) ? 1 : 0;
+                row[j] = rank < need ? INFINITY : -INFINITY;
+            }
+            __syncwarp();
+            int base = 0;
+            for (int j0 = 0; j0 < nt; j0 += 32) {
+                const int j = j0 + lane;
+                const bool take = j < nt && row[j] > hi;
+                const unsigned tb = __ballot_sync(0xffffffffu, take);
+                const int pos = base + __popc(tb & lt_mask);
+                if (take && pos < topk) out[pos] = j;       // exactly topk are taken for finite scores
+                base += __popc(tb);
+            }
+        } else {
+            // Many scores within the error band (ties, or many nearly equal
+            // cubes): fp64 keys for the whole row in this CTA's global
+            // scratch row, then the 64-bit radix select.  One warp of the
+            // CTA at a time owns the scratch row; the owner waits on nothing.
+            bool got = false;
+            const unsigned long long t0 = clock64();
+            while (true) {
+                int v = 0;
+                if (lane == 0) v = atomicCAS(&sh->lock, 0, 1) == 0;
+                got = __shfl_sync(0xffffffffu, v, 0);
+                if (got || clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) break;
+                __nanosleep(256);
+            }
+            if (!got) { if (lane == 0) report(status, kStatusTimeout); continue; }
+            unsigned long long* keys = fallback + (long long)blockIdx.x * nt;
+            for (int j0 = 0; j0 < nt; j0 += 32) {
+                const int j = j0 + lane;
+                const float v = j < nt ? row[j] : -INFINITY;
+                const bool gt = v > hi, band = j < nt && !gt && v >= lo;
+                unsigned bb = __ballot_sync(0xffffffffu, band);
+                unsigned long long key = gt ? ~0ull : 0ull;
+                while (bb) {                                // one warp-wide dot per band cube
+                    const int src = __ffs(bb) - 1;
+                    bb &= bb - 1;
+                    const int jj = j0 + src;
+                    const double s = warp_sum_f64(qrow.partial(Kh + (long long)jj * d, Kl + (long long)jj * d, lane)) * inv_sqrt_d;
+                    if (lane == src) key = f64_key(s);
+                }
+                if (j < nt) keys[j] = key;
+            }
+            __syncwarp();
+            warp_topk(keys, nt, topk, hist, out, lane);
+            __syncwarp();
+            __threadfence_block();
+            if (lane == 0) atomicExch(&sh->lock, 0);
+        }
+    }
+}
+
+// Work items in claim order, for G head groups of hg heads (the last group
+// may be smaller): P_0, P_1, S_0, P_2, S_1, ..., P_{G-1}, S_{G-2}, S_{G-1},
+// where P_g are the 2 * B * ceil(nt / cpi) pool items of group g (cpi cubes,
+// batch, q|k) and
+// S_g its score items (b, head, block of 16 query cubes).  The pooling of
+// group g + 1 (HBM bound) is under way while group g is scored (compute
+// bound); a score item of group g needs exactly the pool items of P_g, all
+// of which come earlier in the order.
+struct SelItem {
+    int kind;                   // 0 pool, 1 score, -1 none
+    int group, local;
+};
+
+__device__ __forceinline__ SelItem decode_item(int item, const Grid& g, const int hg, const int ngroups,
+                                               const int n_pool) {
+    const int rb = ceil_div_i(g.nt, kSelRows);
+    if (item < n_pool) return {0, 0, item};
+    item -= n_pool;
+    for (int grp = 0; grp < ngroups; ++grp) {
+        if (grp + 1 < ngroups) {
+            if (item < n_pool) return {0, grp + 1, item};
+            item -= n_pool;
+        }
+        const int nh = min(hg, g.heads - grp * hg);
+        const int n_score = g.B * nh * rb;
+        if (item < n_score) return {1, grp, item};
+        item -= n_score;
+    }
+    return {-1, 0, 0};
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2)
+select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g, const int topk,
+              const int hg, const int ngroups, const int cpi, float* __restrict__ pooled,
+              unsigned long long* __restrict__ fallback, unsigned int* __restrict__ ctr,
+              int32_t* __restrict__ idx, int* status) {
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    SelShared* sh = reinterpret_cast<SelShared*>(sel_smem);
+    const int cubes_per_b = ceil_div_i(g.nt, cpi);
+    const unsigned n_pool = 2u * g.B * cubes_per_b;     // pool items per group
+    const int rb = ceil_div_i(g.nt, kSelRows);
+    if (threadIdx.x == 0) sh->lock = 0;
+    for (;;) {
+        __syncthreads();                                   // the previous item is done with smem
+        if (threadIdx.x == 0) sh->item = (int)atomicAdd(&ctr[0], 1u);
+        __syncthreads();
+        const SelItem it = decode_item(sh->item, g, hg, ngroups, (int)n_pool);
+        if (it.kind < 0) break;
+        const int h0 = it.group * hg, nh = min(hg, g.heads - h0);
+        if (it.kind == 0) {
+            const int jb = it.local % cubes_per_b, b = (it.local / cubes_per_b) % g.B;
+            const int which = it.local / (cubes_per_b * g.B);
+            pool_item(q, k, g, jb * cpi, cpi, b, which, h0, nh, pooled);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                __threadfence();                           // the item's means, then the count
+                atomicAdd(&ctr[1 + it.group], 1u);
+            }
+            continue;
+        }
+        if (threadIdx.x == 0) {                            // the group's pooling, bounded wait
+            const unsigned long long t0 = clock64();
+            unsigned int done = 0;
+            while (true) {
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(done) : "l"(ctr + 1 + it.group) : "memory");
+                if (done >= n_pool || clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) break;
+                __nanosleep(200);
+            }
+            __threadfence();
+            sh->ready = done >= n_pool ? 1 : -1;
+            if (sh->ready < 0) report(status, kStatusTimeout);
+        }
+        __syncthreads();
+        if (sh->ready < 0) break;
+        // local = (b * nh + head in group) * rb + row block
+        const int bl = it.local / rb, rbi = it.local % rb;
+        const int b = bl / nh, head = h0 + bl % nh;
+        score_item(g, topk, (b * g.heads + head) * rb + rbi, pooled, fallback, idx, sel_smem, status);
+    }
 }
 
 // ------------------------------------------------------------------ launchers
 
+// Scratch: 256 bytes of counters, the pooled means as fp32 hi + lo
+// (2 * 2 * B * heads * nt * d * 4 bytes) and one fallback row of nt 64-bit
+// keys per CTA.
 size_t select_scratch_bytes(const Grid& g) {
-    const size_t pooled = 2ull * g.B * g.heads * g.nt * g.d * sizeof(double);
-    const size_t scores = (size_t)g.B * g.heads * g.nt * g.nt * sizeof(double);
-    return pooled + scores;
-}
-
-static int topk_warps_per_cta(int nt) {
-    // shared memory per warp: nt keys (8 B) + 256 histogram bins (4 B)
-    const size_t per_warp = (size_t)nt * 8 + 1024;
-    int w = 8;
-    while (w > 1 && per_warp * w > 96 * 1024) w >>= 1;
-    return w;
+    const size_t pooled = 4ull * g.B * g.heads * g.nt * g.d * sizeof(float);
+    const size_t fallback = (size_t)kSelMaxCtas * g.nt * sizeof(unsigned long long);
+    return 256 + pooled + fallback;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     const Grid& g = a.g;
-    double* pooled = reinterpret_cast<double*>(a.scratch);
-    double* scores = pooled + 2ull * g.B * g.heads * g.nt * g.d;
-    pool_kernel<<<dim3(g.nt, g.B, 2), 320, 0, stream>>>(a.q, a.k, g, pooled);
-    cudaError_t e = cudaGetLastError();
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(a.scratch);
+    float* pooled = reinterpret_cast<float*>(static_cast<uint8_t*>(a.scratch) + 256);
+    unsigned long long* fallback = reinterpret_cast<unsigned long long*>(pooled + 4ull * g.B * g.heads * g.nt * g.d);
+    const size_t smem = sel_smem_bytes(g.nt, g.d);
+    if (smem > 232448) return cudaErrorInvalidValue;    // nt beyond ~3400 cubes
+    static int configured_device = -1, sms = 0;         // per process: once per device
+    int dev = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const double* qp = pooled;
-    const double* kp = pooled + (size_t)g.B * g.heads * g.nt * g.d;
-    const int tiles = ceil_div_i(g.nt, 64);
-    coarse_kernel<<<dim3(tiles, tiles, g.B * g.heads), 128, 0, stream>>>(qp, kp, g, 1.0 / sqrt((double)g.d), scores);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const int wpc = topk_warps_per_cta(g.nt);
-    const size_t smem = (size_t)wpc * ((size_t)g.nt * 8 + 1024);
-    if (smem > 48 * 1024) {
-        e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (configured_device != dev) {
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
     }
-    const long long rows = (long long)g.B * g.heads * g.nt;
-    const unsigned blocks = (unsigned)((rows + wpc - 1) / wpc);
-    topk_kernel<<<blocks, 32 * wpc, smem, stream>>>(scores, g.nt, a.topk, rows, a.block_idx);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // head groups of hg heads: at most 63, so that their counters and the
+    // claim counter fit the 256-byte counter block
+    const int hg = std::max(8, ceil_div_i(g.heads, 63));
+    const int ngroups = ceil_div_i(g.heads, hg);
+    const int cpi = std::max(1, kSelThreads / (hg * g.d / 8));   // cubes per pool item: ~one vector per thread
+    const long long items = 2ll * g.B * ceil_div_i(g.nt, cpi) * ngroups +
+                            (long long)g.B * g.heads * ceil_div_i(g.nt, kSelRows);
+    const int grid = (int)std::min<long long>(items, std::min(kSelMaxCtas, sms * per_sm));
+    e = cudaMemsetAsync(ctr, 0, (1 + ngroups) * sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
+    select_kernel<<<grid, kSelThreads, smem, stream>>>(a.q, a.k, g, a.topk, hg, ngroups, cpi, pooled, fallback, ctr,
+                                                       a.block_idx, a.status);
     return cudaGetLastError();
 }
 

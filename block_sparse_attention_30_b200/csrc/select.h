@@ -15,6 +15,7 @@ struct SelectArgs {
     int topk;
     int32_t* block_idx;     // [B][heads][nt][topk]
     void* scratch;          // select_scratch_bytes(g) bytes, 16-byte aligned
+    int* status;            // device status word (timeouts), or null
 };
 
 size_t select_scratch_bytes(const Grid& g);

@@ -85,9 +85,11 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
 
 /* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
  * for these shapes: a 256-byte status block followed by a scratch area that
- * holds either the selection's fp64 cube means of q and k
- * ([2][B][heads][nt][d]) and coarse scores ([B][heads][nt][nt]), or the linear branch's operand image (B*heads*(4*d*d + 4*d)
- * bytes), whichever is larger (the backward passes' scratch fits it too: the
+ * holds either the selection's intermediates (256 bytes of counters, the cube
+ * means of q and k as fp32 hi + lo pairs [2][2][B][heads][nt][d] and one
+ * fallback row of nt 64-bit keys for each of at most 1024 CTAs:
+ * 256 + 16*B*heads*nt*d + 8192*nt bytes; no nt x nt term), or the linear
+ * branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is larger (the backward passes' scratch fits it too: the
  * sparse branch's row terms and block-index transpose, the linear branch's
  * two operand images and fp32 gradient sums).  Returns 0 for invalid shapes.  The
  * same workspace may be passed to every call of one forward pass; calls that
@@ -114,11 +116,15 @@ vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int he
                              vsa_stream_t stream);
 
 /* Block selection ("2. 视频稀疏注意力VSA": pick the key blocks each query block
- * attends to).  Mean-pools q and k per cube over valid tokens (fp64), scores
- * C[i][j] = Qp[i].Kp[j]/sqrt(d) in fp64 and writes, per (b, head, i), the
+ * attends to).  Mean-pools q and k per cube over valid tokens (fp64 sums),
+ * scores C[i][j] = Qp[i].Kp[j]/sqrt(d) and writes, per (b, head, i), the
  * topk key cubes with the largest C (ties -> lower j) in ascending order to
- * block_idx.  1 <= topk <= nt.  Needs vsa_workspace_bytes() of workspace.
- * Three launches: the cube means, the coarse scores, the top-k. */
+ * block_idx.  The kept set is the one fp64 scores give: the scores are formed
+ * in fp32 with a bound on their error, and every score the bound leaves
+ * undecided is recomputed in fp64.  1 <= topk <= nt; nt up to about 3400
+ * cubes (VSA_ERR_CUDA beyond).  Needs vsa_workspace_bytes() of workspace.
+ * One kernel (after a 8-byte memset of its work counters): the cube means
+ * go through the workspace, the nt x nt scores only through shared memory. */
 vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
                              int head_dim, int T, int H, int W, int tt, int th, int tw,
                              int topk, int32_t* block_idx, void* workspace,
@@ -278,21 +284,25 @@ vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
  * allocate device memory (no cudaMalloc: a callback or runtime that forbids
  * allocation, a fixed memory budget, an embedding without an allocator) and
  * so cannot provide vsa_select_blocks' workspace.  It computes exactly what
- * vsa_select_blocks computes, with the same kernels, but keeps the
- * intermediate fp64 cube means and coarse scores in one file-scope device
- * array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved on every GPU that loads
- * the library until the process exits.  It allocates and frees nothing.
+ * vsa_select_blocks computes, with the same kernel, but keeps the
+ * selection's intermediates (work counters, cube means, fallback rows) in one
+ * file-scope device array of VSA_NOALLOC_SELECT_SCRATCH_BYTES, reserved on
+ * every GPU that loads the library until the process exits.  It allocates and
+ * frees nothing.
  *
  *  - The caller still passes q, k (device, bf16 [B][N][heads][d]) and
  *    block_idx (device, int32 [B][heads][nt][topk]), 16-byte aligned.
  *  - Shapes whose intermediates exceed the array
- *    (2*B*heads*nt*d*8 + B*heads*nt*nt*8 bytes > the maximum) are rejected
+ *    (256 + 16*B*heads*nt*d + 8192*nt bytes > the maximum) are rejected
  *    with VSA_ERR_WORKSPACE before anything is enqueued; argument errors as
  *    for vsa_select_blocks.
  *  - All calls share the array, which keeps the last call's contents; every
- *    call rewrites what it reads, so nothing needs clearing.  Calls that
- *    overlap on the GPU (other streams, unordered host threads) race on it:
- *    order them on one stream.
+ *    call clears its work counters (a memset it enqueues) and rewrites what
+ *    it reads.  Calls that overlap on the GPU (other streams, unordered host
+ *    threads) race on it: order them on one stream.
+ *  - There is no status word: a wait that gives up (the kernel's bounded
+ *    wait for its own pooling, about 2 s) leaves rows of block_idx unwritten
+ *    without a report.  vsa_select_blocks reports it as VSA_ERR_TIMEOUT.
  *  - The first call on each device (and the first after the device's
  *    primary context was reset) looks up the array's device address with that
  *    device current; make that first call before any stream capture.

@@ -26,7 +26,7 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(vsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_expected_entry_points():
@@ -34,7 +34,8 @@ def test_header_declares_expected_entry_points():
     for n in ["vsa_select_blocks", "vsa_sparse_attn_fwd", "vsa_linear_branch_fwd",
               "vsa_sparse_attn_fwd_train", "vsa_sparse_attn_bwd", "vsa_linear_branch_bwd",
               "vsa_gather_tiles", "vsa_scatter_tiles", "vsa_workspace_bytes",
-              "vsa_device_status", "vsa_status_string"]:
+              "vsa_device_status", "vsa_status_string", "vsa_quantize_qk_e4m3",
+              "vsa_sparse_attn_fwd_e4m3", "vsa_sparse_linear_attn_fwd_e4m3"]:
         assert n in names
 
 
@@ -56,7 +57,10 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_num_tiles(4, 32, 32, 4, 4, 4) == 64
     assert L.vsa_num_tiles(0, 4, 4, 4, 4, 4) == 0
     nt, B, h, d = 455, 1, 40, 128
-    want = 256 + 2 * B * h * nt * d * 8 + B * h * nt * nt * 8
+    # status block + the selection's scratch: 256 bytes of counters, the
+    # pooled means as fp32 hi + lo for q and k, one fallback row of nt 64-bit
+    # keys for each of at most 1024 CTAs (no nt^2 term)
+    want = 256 + 256 + 4 * B * h * nt * d * 4 + 1024 * nt * 8
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 46) == want
     assert L.vsa_workspace_bytes(B, h, 96, 20, 28, 52, 4, 4, 4, 46) == 0       # d unsupported
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32
@@ -129,6 +133,13 @@ def test_other_entry_points_validate(L):
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 5, FAKE, 1024, None) == INVALID     # topk > nt
     assert fe(*[FAKE] * 6, FAKE + 2, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == INVALID
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 8, None) == WORKSPACE
+    fl = L.vsa_sparse_linear_attn_fwd_e4m3                 # q8 k8 sq sk q v idx S z out
+    image = 2 * (4 * 128 * 128 + 4 * 128)
+    assert fl(*[FAKE] * 10, 1, 2, 64, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == UNSUPPORTED   # d = 64
+    assert fl(*[FAKE] * 10, 1, 2, 128, 4, 8, 8, 4, 4, 4, 0, FAKE, 1 << 20, None) == INVALID     # topk < 1
+    assert fl(*[FAKE] * 7, None, FAKE, FAKE, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == INVALID
+    assert fl(*[FAKE] * 4, FAKE + 2, *[FAKE] * 5, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == INVALID
+    assert fl(*[FAKE] * 10, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 256 + image - 16, None) == WORKSPACE
     ft = L.vsa_sparse_attn_fwd_train
     assert ft(*[FAKE] * 7, *SHAPE, 2, None, 1 << 30, None) == WORKSPACE
     assert ft(*[FAKE] * 5, FAKE + 4, FAKE, *SHAPE, 2, FAKE, 1 << 30, None) == INVALID        # out_f32
@@ -193,6 +204,7 @@ def test_cuda_failures_surface_as_status_codes(L):
     assert L.vsa_linear_branch_bwd(*[FAKE] * 9, 0, *SH[:6], FAKE, ws, None) == CUDA
     assert L.vsa_quantize_qk_e4m3(*[FAKE] * 6, *SH, None) == CUDA
     assert L.vsa_sparse_attn_fwd_e4m3(*[FAKE] * 7, *SH, 2, FAKE, ws, None) == CUDA
+    assert L.vsa_sparse_linear_attn_fwd_e4m3(*[FAKE] * 10, *SH, 2, FAKE, ws, None) == CUDA
     assert L.vsa_selftest_wait_timeout(FAKE, ws, 1000, None) == CUDA
     assert L.vsa_device_status(FAKE, None) == CUDA
 

@@ -151,6 +151,34 @@ def test_exact_ties_take_lowest_cube_ids(ops, d, topk):
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
 
 
+@pytest.mark.parametrize("levels,topk", [(1, 40), (2, 40), (2, 100), (5, 7)])
+def test_ties_beyond_the_refined_candidates(ops, levels, topk):
+    """128 key cubes in `levels` classes of identical tokens: a row then has
+    64 or more cubes whose scores tie at the k-th, more than the selection
+    refines one by one, so it takes its fallback (fp64 keys for the whole row
+    and a 64-bit radix select); the result must still follow the tie rule
+    exactly."""
+    T, H, W, heads, d = 8, 32, 32, 2, 128                # 2 x 8 x 8 = 128 cubes
+    c = Small(T, H, W, heads, d, topk, seed=9)
+    g = torch.Generator().manual_seed(321)
+    lv = torch.randn(levels, heads, d, generator=g).to(torch.bfloat16)
+    slots = O.tile_slots(T, H, W, (4, 4, 4))
+    k = c.k.clone()
+    for j in range(slots.shape[0]):
+        toks = torch.as_tensor(slots[j][slots[j] >= 0])
+        k[0, toks] = lv[j % levels]
+    idx, _ = run_select(ops, c, c.q.cuda(), k.cuda())
+    ref_idx, _ = O.select(c.q, k, 1, heads, d, T, H, W, topk, (4, 4, 4), with_scores=True)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+
+
+def test_selection_keeps_every_cube_at_k_equal_nt(ops):
+    T, H, W, heads, d = 8, 12, 12, 3, 64                 # 2 x 3 x 3 = 18 cubes
+    c = Small(T, H, W, heads, d, 18, seed=4)
+    idx, _ = run_select(ops, c, c.q.cuda(), c.k.cuda())
+    np.testing.assert_array_equal(idx.cpu().numpy(), np.broadcast_to(np.arange(18), (1, heads, 18, 18)))
+
+
 @pytest.mark.parametrize("case", [(5, 6, 7, 3, 128, 3), (4, 8, 12, 2, 64, 4)])
 def test_batch_of_two(ops, case):
     """B = 2: batch indexing of the pooled means, TMA boxes and outputs."""
