@@ -17,8 +17,9 @@
 //   score items  one per (b, head, block of 16 query cubes): the coarse
 //                scores of the 16 rows against all nt key cubes,
 //                C = Qp Kp^T / sqrt(d), in fp32 (packed fp32x2 FMA, the 16
-//                rows' Qp in shared memory, four key cubes per lane, the
-//                features split over two warps) into shared memory -- the nt x nt
+//                rows' Qp in shared memory, four key cubes per lane read
+//                from a feature-major copy of Kp, the features split over
+//                two warps) into shared memory -- the nt x nt
 //                score matrix never reaches HBM -- then per row (one warp)
 //                the exact top-k:
 //                  1. a bracket [lo, hi] around the k-th largest fp32 score
@@ -74,11 +75,12 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 raw) {
 
 // Means of cubes j0 .. j0 + cpi - 1 (those < nt) of batch b of q (which = 0)
 // or k (which = 1), heads h0 .. h0 + nh - 1, written as fp32 hi + lo into
-// pooled[which][0|1][b][head][j][d].  Thread t takes (cube, 16-byte vector)
+// pooled[which][0|1][b][head][j][d], and for k the hi part once more
+// feature-major into kt[b][head][d][ntp] (the coarse scores' loads).  Thread t takes (cube, 16-byte vector)
 // pairs t, t + 256, ...
 __device__ void pool_item(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid& g,
                           const int j0, const int cpi, const int b, const int which, const int h0, const int nh,
-                          float* __restrict__ pooled) {
+                          float* __restrict__ pooled, float* __restrict__ kt, const int ntp) {
     const uint16_t* x = which ? k : q;
     const int row_elems = g.heads * g.d;              // one token: all heads
     const int nvec = nh * g.d / 8;                    // per cube: heads h0 .. h0 + nh - 1
@@ -130,6 +132,11 @@ __device__ void pool_item(const uint16_t* __restrict__ q, const uint16_t* __rest
         reinterpret_cast<float4*>(hi + off)[1] = make_float4(h8[4], h8[5], h8[6], h8[7]);
         reinterpret_cast<float4*>(lo + off)[0] = make_float4(l8[0], l8[1], l8[2], l8[3]);
         reinterpret_cast<float4*>(lo + off)[1] = make_float4(l8[4], l8[5], l8[6], l8[7]);
+        if (which) {                                  // k hi once more, feature-major
+            float* t = kt + (((long long)b * g.heads + head) * g.d + c0) * ntp + j;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[(long long)e * ntp] = h8[e];
+        }
     }
 }
 
@@ -144,7 +151,7 @@ __device__ __forceinline__ unsigned long long ordered_key(double x) {
 // 256 shared-memory bins of this warp's own): MSD radix select of the k-th
 // largest key, then the kept indices in ascending order (equal keys lowest j
 // first) written to out[0..k).
-__device__ void warp_topk(const unsigned long long* __restrict__ keys, const int nt, const int k,
+__device__ __noinline__ void warp_topk(const unsigned long long* __restrict__ keys, const int nt, const int k,
                           unsigned int* __restrict__ hist, int32_t* __restrict__ out, const int lane) {
     // Skip the leading bytes every key shares (for scores of one magnitude
     // the sign and exponent byte): start at the highest byte where the
@@ -274,7 +281,7 @@ __device__ __forceinline__ int bin256(float x) {
 // holds x in [t1 + t2 / 256, t1 + (t2 + 1) / 256] up to the rounding of x
 // (3.1 ulp relative, at most 3.2 * 2^-24 * (max - min) in s); the bracket is
 // widened by 8 * 2^-24 * (|min| + |max| + max - min).
-__device__ void warp_bracket(const float* __restrict__ row, const int nt, const int k,
+__device__ __noinline__ void warp_bracket(const float* __restrict__ row, const int nt, const int k,
                              unsigned int* __restrict__ hist, const int lane, double& lo, double& hi) {
     float mn = INFINITY, mx = -INFINITY;
     for (int j0 = 0; j0 < nt; j0 += 128) {
@@ -389,6 +396,7 @@ __host__ __device__ inline size_t sel_smem_bytes(int nt, int d) {
 }
 
 __device__ void score_item(const Grid& g, const int topk, const int item, const float* __restrict__ pooled,
+                           const float* __restrict__ kt,
                            unsigned long long* __restrict__ fallback, int32_t* __restrict__ idx,
                            uint8_t* smem, int* status) {
     SelShared* sh = reinterpret_cast<SelShared*>(smem);
@@ -421,39 +429,47 @@ __device__ void score_item(const Grid& g, const int topk, const int item, const 
     if (tid == 0) sh->kmax2[0] = sh->kmax2[1] = 0.f;
     __syncthreads();
 
-    // ---- coarse scores, fp32: each lane four key cubes and all 16 rows
-    // (acc[b][p] holds rows 2p, 2p+1 of key b; one packed fp32x2 FMA per row
-    // pair); warps w and w + 4 take the two halves of the features of the
-    // same 128 keys, each half summed in feature order, and the two partial
-    // sums meet in shared memory (C = (half 0 + half 1) / sqrt(d)).
+    // ---- coarse scores, fp32: each lane four consecutive key cubes and all
+    // 16 rows (acc[b][p] holds rows 2p, 2p+1 of key b; one packed fp32x2 FMA
+    // per row pair); warps w and w + 4 take the two halves of the features of
+    // the same 128 keys, each half summed in feature order, and the two
+    // partial sums meet in shared memory (C = (half 0 + half 1) / sqrt(d)).
+    // The keys come from the feature-major copy kt: one 16-byte load per lane
+    // and feature, 512 contiguous bytes per warp, PF features in flight.
     const int half = warp >> 2, kw = warp & 3, dh = d / 2, c0 = half * dh;
     const int passes = ceil_div_i(nt, 512);
+    const float* Kt = kt + (long long)bh * d * ntp;
     float kmax2 = 0.f;                                    // max_j of this half's |Kp_j|^2
     for (int ps = 0; ps < passes; ++ps) {
         const int j0 = ps * 512 + kw * 128 + 4 * lane;
-        const float* kbase = Kh + (long long)j0 * d + c0;
+        const bool live = j0 < ntp;                       // ntp and j0 multiples of 4
+        const float* kp = Kt + (long long)c0 * ntp + (live ? j0 : 0);
         uint64_t acc[4][kSelRows / 2];
 #pragma unroll
         for (int b = 0; b < 4; ++b)
 #pragma unroll
             for (int p = 0; p < kSelRows / 2; ++p) acc[b][p] = 0ull;
         float nrm[4] = {0.f, 0.f, 0.f, 0.f};
-        float4 cur[4];
-        for (int dc = 0; dc < dh; dc += 4) {
+        constexpr int PF = 2;
+        float4 ring[PF];
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
-                cur[b] = j0 + b < nt ? __ldcg(reinterpret_cast<const float4*>(kbase + (long long)b * d + dc))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < PF; ++e)
+            ring[e] = live ? __ldcg(reinterpret_cast<const float4*>(kp + (long long)e * ntp)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < dh; c += PF) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4* qq = reinterpret_cast<const float4*>(sQ + (c0 + dc + c) * kSelRows);
+            for (int e = 0; e < PF; ++e) {
+                const float4 kv4 = ring[e];
+                const int cn = c + e + PF;
+                ring[e] = live && cn < dh ? __ldcg(reinterpret_cast<const float4*>(kp + (long long)cn * ntp))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float kv[4] = {kv4.x, kv4.y, kv4.z, kv4.w};
                 uint64_t kd[4];
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
-                    const float kv = c == 0 ? cur[b].x : c == 1 ? cur[b].y : c == 2 ? cur[b].z : cur[b].w;
-                    nrm[b] = fmaf(kv, kv, nrm[b]);
-                    kd[b] = f32x2(kv, kv);
+                    nrm[b] = fmaf(kv[b], kv[b], nrm[b]);
+                    kd[b] = f32x2(kv[b], kv[b]);
                 }
+                const float4* qq = reinterpret_cast<const float4*>(sQ + (c0 + c + e) * kSelRows);
 #pragma unroll
                 for (int p4 = 0; p4 < kSelRows / 4; ++p4) {
                     const float4 q4 = qq[p4];
@@ -643,7 +659,7 @@ __device__ __forceinline__ SelItem decode_item(int item, const Grid& g, const in
 
 __global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const Grid g, const int topk,
-              const int hg, const int ngroups, const int cpi, float* __restrict__ pooled,
+              const int hg, const int ngroups, const int cpi, float* __restrict__ pooled, float* __restrict__ kt,
               unsigned long long* __restrict__ fallback, unsigned int* __restrict__ ctr,
               int32_t* __restrict__ idx, int* status) {
     extern __shared__ __align__(16) uint8_t sel_smem[];
@@ -662,7 +678,7 @@ select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, co
         if (it.kind == 0) {
             const int jb = it.local % cubes_per_b, b = (it.local / cubes_per_b) % g.B;
             const int which = it.local / (cubes_per_b * g.B);
-            pool_item(q, k, g, jb * cpi, cpi, b, which, h0, nh, pooled);
+            pool_item(q, k, g, jb * cpi, cpi, b, which, h0, nh, pooled, kt, sel_ntp(g.nt));
             __syncthreads();
             if (threadIdx.x == 0) {
                 __threadfence();                           // the item's means, then the count
@@ -687,26 +703,29 @@ select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, co
         // local = (b * nh + head in group) * rb + row block
         const int bl = it.local / rb, rbi = it.local % rb;
         const int b = bl / nh, head = h0 + bl % nh;
-        score_item(g, topk, (b * g.heads + head) * rb + rbi, pooled, fallback, idx, sel_smem, status);
+        score_item(g, topk, (b * g.heads + head) * rb + rbi, pooled, kt, fallback, idx, sel_smem, status);
     }
 }
 
 // ------------------------------------------------------------------ launchers
 
 // Scratch: 256 bytes of counters, the pooled means as fp32 hi + lo
-// (2 * 2 * B * heads * nt * d * 4 bytes) and one fallback row of nt 64-bit
-// keys per CTA.
+// (2 * 2 * B * heads * nt * d * 4 bytes), the feature-major copy of the k hi
+// means (B * heads * d * ntp * 4 bytes, ntp = nt rounded up to 4) and one
+// fallback row of nt 64-bit keys per CTA.
 size_t select_scratch_bytes(const Grid& g) {
     const size_t pooled = 4ull * g.B * g.heads * g.nt * g.d * sizeof(float);
+    const size_t kt = (size_t)g.B * g.heads * g.d * sel_ntp(g.nt) * sizeof(float);
     const size_t fallback = (size_t)kSelMaxCtas * g.nt * sizeof(unsigned long long);
-    return 256 + pooled + fallback;
+    return 256 + pooled + kt + fallback;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     const Grid& g = a.g;
     unsigned int* ctr = reinterpret_cast<unsigned int*>(a.scratch);
     float* pooled = reinterpret_cast<float*>(static_cast<uint8_t*>(a.scratch) + 256);
-    unsigned long long* fallback = reinterpret_cast<unsigned long long*>(pooled + 4ull * g.B * g.heads * g.nt * g.d);
+    float* kt = pooled + 4ull * g.B * g.heads * g.nt * g.d;
+    unsigned long long* fallback = reinterpret_cast<unsigned long long*>(kt + (size_t)g.B * g.heads * g.d * sel_ntp(g.nt));
     const size_t smem = sel_smem_bytes(g.nt, g.d);
     if (smem > 232448) return cudaErrorInvalidValue;    // nt beyond ~3400 cubes
     static int configured_device = -1, sms = 0;         // per process: once per device
@@ -733,7 +752,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     const int grid = (int)std::min<long long>(items, std::min(kSelMaxCtas, sms * per_sm));
     e = cudaMemsetAsync(ctr, 0, (1 + ngroups) * sizeof(unsigned int), stream);
     if (e != cudaSuccess) return e;
-    select_kernel<<<grid, kSelThreads, smem, stream>>>(a.q, a.k, g, a.topk, hg, ngroups, cpi, pooled, fallback, ctr,
+    select_kernel<<<grid, kSelThreads, smem, stream>>>(a.q, a.k, g, a.topk, hg, ngroups, cpi, pooled, kt, fallback, ctr,
                                                        a.block_idx, a.status);
     return cudaGetLastError();
 }

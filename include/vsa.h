@@ -86,9 +86,11 @@ int vsa_num_tiles(int T, int H, int W, int tt, int th, int tw);
 /* Bytes of device workspace vsa_select_blocks and vsa_sparse_attn_fwd need
  * for these shapes: a 256-byte status block followed by a scratch area that
  * holds either the selection's intermediates (256 bytes of counters, the cube
- * means of q and k as fp32 hi + lo pairs [2][2][B][heads][nt][d] and one
- * fallback row of nt 64-bit keys for each of at most 1024 CTAs:
- * 256 + 16*B*heads*nt*d + 8192*nt bytes; no nt x nt term), or the linear
+ * means of q and k as fp32 hi + lo pairs [2][2][B][heads][nt][d], a
+ * feature-major copy of the k means [B][heads][d][ntp] (ntp = nt rounded up
+ * to a multiple of 4) and one fallback row of nt 64-bit keys for each of at
+ * most 1024 CTAs: 256 + 16*B*heads*nt*d + 4*B*heads*d*ntp + 8192*nt bytes;
+ * no nt x nt term), or the linear
  * branch's operand image (B*heads*(4*d*d + 4*d) bytes), whichever is larger (the backward passes' scratch fits it too: the
  * sparse branch's row terms and block-index transpose, the linear branch's
  * two operand images and fp32 gradient sums).  Returns 0 for invalid shapes.  The
@@ -293,7 +295,8 @@ vsa_status vsa_device_status(void* workspace, vsa_stream_t stream);
  *  - The caller still passes q, k (device, bf16 [B][N][heads][d]) and
  *    block_idx (device, int32 [B][heads][nt][topk]), 16-byte aligned.
  *  - Shapes whose intermediates exceed the array
- *    (256 + 16*B*heads*nt*d + 8192*nt bytes > the maximum) are rejected
+ *    (256 + 16*B*heads*nt*d + 4*B*heads*d*ntp + 8192*nt bytes, ntp = nt
+ *    rounded up to 4, > the maximum) are rejected
  *    with VSA_ERR_WORKSPACE before anything is enqueued; argument errors as
  *    for vsa_select_blocks.
  *  - All calls share the array, which keeps the last call's contents; every

@@ -58,9 +58,11 @@ def test_num_tiles_and_workspace(L):
     assert L.vsa_num_tiles(0, 4, 4, 4, 4, 4) == 0
     nt, B, h, d = 455, 1, 40, 128
     # status block + the selection's scratch: 256 bytes of counters, the
-    # pooled means as fp32 hi + lo for q and k, one fallback row of nt 64-bit
-    # keys for each of at most 1024 CTAs (no nt^2 term)
-    want = 256 + 256 + 4 * B * h * nt * d * 4 + 1024 * nt * 8
+    # pooled means as fp32 hi + lo for q and k, the feature-major copy of the
+    # k means (nt rounded up to 4), one fallback row of nt 64-bit keys for
+    # each of at most 1024 CTAs (no nt^2 term)
+    ntp = (nt + 3) // 4 * 4
+    want = 256 + 256 + 4 * B * h * nt * d * 4 + B * h * d * ntp * 4 + 1024 * nt * 8
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 4, 46) == want
     assert L.vsa_workspace_bytes(B, h, 96, 20, 28, 52, 4, 4, 4, 46) == 0       # d unsupported
     assert L.vsa_workspace_bytes(B, h, d, 20, 28, 52, 4, 4, 2, 46) == 0        # volume 32

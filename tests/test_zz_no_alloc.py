@@ -59,7 +59,7 @@ def test_noalloc_select_matches_workspace_select_twice(L):
 
 
 def test_noalloc_select_rejects_shapes_beyond_the_array(L):
-    w = WORKLOADS["wan14b_480p"]             # 41 MB of intermediates: too large
+    w = WORKLOADS["wan14b_480p"]             # 50 MB of intermediates: too large
     tt, th, tw = w.tile
     fake = 0x10000                           # never dereferenced: refused before launch
     code = L.vsa_select_blocks_noalloc(fake, fake, w.B, w.heads, w.head_dim, w.T, w.H, w.W,
