@@ -497,6 +497,11 @@ def run_kernels(args):
             ("sparse_attn_fwd_e4m3 (E4M3 Q K^T, bf16 P V)", lambda: ops.vsa_sparse_attn_fwd_e4m3(
                 q8, k8, sq, sk, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, w.tile),
              "tensor", w.fine_flops()),
+            ("sparse_linear_attn_fwd_e4m3 (SageSLA: E4M3 sparse + linear apply)",
+             lambda: ops.vsa_sparse_linear_attn_fwd_e4m3(
+                 q8, k8, sq, sk, q, v, attn.block_idx, attn.lin_S, attn.lin_z, out, w.T, w.H, w.W, w.topk,
+                 attn.workspace, w.tile),
+             "tensor", w.fine_flops()),
         ]
     for name, fn, bound, units in rows:
         ms = timed(fn)

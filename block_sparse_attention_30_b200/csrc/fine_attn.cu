@@ -183,6 +183,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             int issued = 0;
             if (is_k) {
                 const TileCoord qc = tile_coord(g, i);
+                VSA_DEBUG_CHECK(qc.t0 < g.T && qc.h0 < g.H && qc.w0 < g.W, status, kStatusBadCoord);
                 mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
                 for (int c = 0; c < C::NCH_QK; ++c)
                     tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + (128 / C::QB) * c, qc.w0, qc.h0, qc.t0, b);
@@ -217,6 +218,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 mbar_arrive_expect_tx(&full[st], ntl * (is_k ? C::K_CUBE_BYTES : C::V_CUBE_BYTES));
                 for (int t = 0; t < ntl; ++t) {
                     const TileCoord kc = tile_coord(g, jt[t]);
+                    VSA_DEBUG_CHECK(kc.t0 < g.T && kc.h0 < g.H && kc.w0 < g.W, status, kStatusBadCoord);
                     for (int c = 0; c < nch; ++c)
                         tma_load_5d(ring + st * pair_bytes + c * C::CHUNK_STRIDE + t * 8192, map,
                                     &full[st], head * D + cw * c, kc.w0, kc.h0, kc.t0, b);
@@ -476,6 +478,14 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o[e] *= inv;
                 }
+#ifdef VSA_DEBUG_CHECKS
+                if (valid) {
+                    bool finite = true;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) finite = finite && isfinite(o[e]);
+                    VSA_DEBUG_CHECK(finite, status, kStatusNonFinite);
+                }
+#endif
                 uint4 w0, w1;
                 w0.x = pack_bf16x2(o[0], o[1]);
                 w0.y = pack_bf16x2(o[2], o[3]);

@@ -955,3 +955,10 @@ def test_debug_check_build_reports_non_finite_output(ops):
     assert st == 6, _lib.STATUS_NAMES.get(st, st)     # VSA_ERR_DEVICE_CHECK
     _, st = fine_debug(vd)
     assert st == 0                                     # the word was cleared by the report
+    # the one-cube kernel (rows of more than 24 kept cubes): k = 26 of 32
+    idx26, ws26 = run_select(ops, Small(8, 16, 16, 2, 128, 26, seed=3), qd, kd)
+    out = torch.zeros_like(qd)
+    call = lambda v: L.vsa_sparse_attn_fwd(qd.data_ptr(), kd.data_ptr(), v.data_ptr(), idx26.data_ptr(), None,
+                                           None, out.data_ptr(), *shape, 26, ws26.data_ptr(), ws26.numel(), stream)
+    assert call(vd) == 0 and L.vsa_device_status(ws26.data_ptr(), stream) == 0
+    assert call(bad) == 0 and L.vsa_device_status(ws26.data_ptr(), stream) == 6
