@@ -484,25 +484,24 @@ def run_kernels(args):
             q, k, v, g_out, attn.lin_S, attn.lin_z, dq, dk, dv, w.T, w.H, w.W, attn.workspace),
          "hbm", 7 * elem),
     ]
-    if w.head_dim == 128:
-        # low-precision fine pass: E4M3 codes of q and k (one byte each) with
-        # per-cube scales, then the fine kernel with Q K^T in E4M3; its FLOPs
-        # are the same effective count, its fraction is of the bf16 peak (half
-        # of the products run at the E4M3 rate, so a mixed ceiling is 4/3 of it)
-        q8, k8 = (torch.empty(q.shape, dtype=torch.uint8, device=dev) for _ in range(2))
-        sq, sk = (torch.empty((w.B, w.heads, nt), dtype=torch.float32, device=dev) for _ in range(2))
-        rows += [
-            ("quantize_qk_e4m3 (low-precision pre-pass)", lambda: ops.vsa_quantize_qk_e4m3(
-                q, k, q8, k8, sq, sk, w.T, w.H, w.W, w.tile), "hbm", 3 * elem),
-            ("sparse_attn_fwd_e4m3 (E4M3 Q K^T, bf16 P V)", lambda: ops.vsa_sparse_attn_fwd_e4m3(
-                q8, k8, sq, sk, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, w.tile),
-             "tensor", w.fine_flops()),
-            ("sparse_linear_attn_fwd_e4m3 (SageSLA: E4M3 sparse + linear apply)",
-             lambda: ops.vsa_sparse_linear_attn_fwd_e4m3(
-                 q8, k8, sq, sk, q, v, attn.block_idx, attn.lin_S, attn.lin_z, out, w.T, w.H, w.W, w.topk,
-                 attn.workspace, w.tile),
-             "tensor", w.fine_flops()),
-        ]
+    # low-precision fine pass: E4M3 codes of q and k (one byte each) with
+    # per-cube scales, then the fine kernel with Q K^T in E4M3; its FLOPs
+    # are the same effective count, its fraction is of the bf16 peak (half
+    # of the products run at the E4M3 rate, so a mixed ceiling is 4/3 of it)
+    q8, k8 = (torch.empty(q.shape, dtype=torch.uint8, device=dev) for _ in range(2))
+    sq, sk = (torch.empty((w.B, w.heads, nt), dtype=torch.float32, device=dev) for _ in range(2))
+    rows += [
+        ("quantize_qk_e4m3 (low-precision pre-pass)", lambda: ops.vsa_quantize_qk_e4m3(
+            q, k, q8, k8, sq, sk, w.T, w.H, w.W, w.tile), "hbm", 3 * elem),
+        ("sparse_attn_fwd_e4m3 (E4M3 Q K^T, bf16 P V)", lambda: ops.vsa_sparse_attn_fwd_e4m3(
+            q8, k8, sq, sk, v, attn.block_idx, out, w.T, w.H, w.W, w.topk, attn.workspace, w.tile),
+         "tensor", w.fine_flops()),
+        ("sparse_linear_attn_fwd_e4m3 (SageSLA: E4M3 sparse + linear apply)",
+         lambda: ops.vsa_sparse_linear_attn_fwd_e4m3(
+             q8, k8, sq, sk, q, v, attn.block_idx, attn.lin_S, attn.lin_z, out, w.T, w.H, w.W, w.topk,
+             attn.workspace, w.tile),
+         "tensor", w.fine_flops()),
+    ]
     for name, fn, bound, units in rows:
         ms = timed(fn)
         if bound == "hbm":

@@ -70,18 +70,19 @@ bool encode_grid_map(CUtensorMap* m, const void* base, const vsa::Grid& g) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The same 5-D view over E4M3 codes (one byte per element): box {128 codes
-// (= 128 bytes, the whole d of a head at d = 128), tw, th, tt, 1}.
+// The same 5-D view over E4M3 codes (one byte per element): box {d codes
+// (the whole d of a head: 128 bytes with the 128-byte swizzle at d = 128,
+// 64 bytes with the 64-byte swizzle at d = 64), tw, th, tt, 1}.
 bool encode_grid_map_u8(CUtensorMap* m, const void* base, const vsa::Grid& g) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t row = (cuuint64_t)g.heads * g.d;
     cuuint64_t dims[5] = {row, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T, (cuuint64_t)g.B};
     cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
-    cuuint32_t box[5] = {128, (cuuint32_t)g.tw, (cuuint32_t)g.th, (cuuint32_t)g.tt, 1};
+    cuuint32_t box[5] = {(cuuint32_t)g.d, (cuuint32_t)g.tw, (cuuint32_t)g.th, (cuuint32_t)g.tt, 1};
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, g.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -344,7 +345,6 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
                                     vsa_stream_t stream) {
     vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
     if (s != VSA_OK) return s;
-    if (head_dim != 128) return VSA_ERR_UNSUPPORTED;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
     for (const void* p : {(const void*)q8, (const void*)k8, (const void*)q_scale, (const void*)k_scale,
@@ -382,7 +382,6 @@ vsa_status vsa_sparse_linear_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8,
                                            vsa_stream_t stream) {
     vsa_status s = check_shape(B, heads, head_dim, T, H, W, tt, th, tw);
     if (s != VSA_OK) return s;
-    if (head_dim != 128) return VSA_ERR_UNSUPPORTED;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
     for (const void* p : {(const void*)q8, (const void*)k8, (const void*)q_scale, (const void*)k_scale,

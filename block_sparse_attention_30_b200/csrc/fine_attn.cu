@@ -30,11 +30,12 @@
 // Two CTAs share an SM (256 TMEM columns and ~112 KB of shared memory each),
 // so one CTA's softmax overlaps the other's MMAs.
 //
-// Low-precision variant (Q8, d = 128): q and k arrive as FP8 E4M3 codes with
-// one scale per (b, head, cube) (quant.cu); Q K^T runs as tcgen05
-// kind::f8f6f4 (K = 32 per MMA, one 128-byte row per token), the softmax
-// multiplies each half row by its query and key cube scales, P V stays bf16.
-// The halved Q and K tiles make room for a second V stage.  With the linear
+// Low-precision variant (Q8): q and k arrive as FP8 E4M3 codes with one scale
+// per (b, head, cube) (quant.cu); Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
+// per MMA; one row of d bytes per token: 128-byte swizzle at d = 128, 64-byte
+// swizzle at d = 64), the softmax multiplies each half row by its query and
+// key cube scales, P V stays bf16.  At d = 128 the halved Q and K tiles make
+// room for a second V stage.  With the linear
 // branch (SageSLA: the sparse + linear attention on quantised products), the
 // branch itself stays bf16 hi + lo: phi(q) comes from the bf16 q in global
 // memory and goes into the K ring, the (S, z) image into the V ring.
@@ -58,7 +59,9 @@ template <int D, bool Q8 = false>
 struct FineCfg {
     static constexpr int QB = Q8 ? 1 : 2;              // bytes per q / k element
     static constexpr int NCH = D / 64;                 // 128-byte d chunks of V
-    static constexpr int NCH_QK = D * QB / 128;        // 128-byte d chunks of Q and K
+    static constexpr int QK_ROW = D * QB < 128 ? D * QB : 128;   // bytes of a Q / K box row
+    static constexpr int NCH_QK = D * QB / QK_ROW;     // d chunks of Q and K (boxes per cube)
+    static constexpr int QK_BOX = 64 * QK_ROW;         // bytes of one cube's box
     static constexpr int Q_BYTES = 64 * D * QB;        // one query cube
     static constexpr int K_CUBE_BYTES = 64 * D * QB;   // one key cube of K
     static constexpr int V_CUBE_BYTES = 64 * D * 2;    // one key cube of V
@@ -66,9 +69,10 @@ struct FineCfg {
     static constexpr int V_PAIR_BYTES = 2 * V_CUBE_BYTES;
     static constexpr int CHUNK_STRIDE = 128 * 128;     // bytes between d chunks of a pair
     static constexpr int NK = (D == 128) ? 2 : 3;      // K pair stages
+    static_assert(QK_ROW == 128 || (Q8 && D == 64), "64-byte rows only for E4M3 at d = 64");
     // the smaller K and Q of the low-precision variant leave room for a
     // second V stage within two CTAs per SM
-    static constexpr int NV = Q8 ? 2 : ((D == 128) ? 1 : 3);   // V pair stages
+    static constexpr int NV = (D == 128) ? (Q8 ? 2 : 1) : 3;   // V pair stages
     static constexpr int TMEM_COLS = 256;
     // A ring slot is free once the MMAs reading it are done.  With two K stages
     // the stage of pair p is the S buffer p & 1, so the K producer can wait on
@@ -103,6 +107,8 @@ static_assert(sizeof(FineBars<128>) <= FineCfg<128>::BAR_BYTES, "barrier block")
 static_assert(sizeof(FineBars<64>) <= FineCfg<64>::BAR_BYTES, "barrier block");
 static_assert(sizeof(FineBars<128, true>) <= FineCfg<128, true>::BAR_BYTES, "barrier block");
 static_assert(FineCfg<128, true>::SMEM_BYTES <= 232448 / 2 - 1024, "two CTAs per SM");
+static_assert(sizeof(FineBars<64, true>) <= FineCfg<64, true>::BAR_BYTES, "barrier block");
+static_assert(FineCfg<64, true>::SMEM_BYTES <= 232448 / 2 - 1024, "two CTAs per SM");
 
 template <int D, bool LIN, bool Q8>
 __global__ void __launch_bounds__(224, 2)
@@ -114,7 +120,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                  const float* __restrict__ q_scale, const float* __restrict__ k_scale,
                  const __nv_bfloat16* __restrict__ q_bf16, int* status) {
     using C = FineCfg<D, Q8>;
-    static_assert(!Q8 || D == 128, "the low-precision variant is d = 128");
+
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023) {               // uniform early exit, before any sync
         if (threadIdx.x == 0) report(status, kStatusMisaligned);
@@ -186,7 +192,8 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 VSA_DEBUG_CHECK(qc.t0 < g.T && qc.h0 < g.H && qc.w0 < g.W, status, kStatusBadCoord);
                 mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
                 for (int c = 0; c < C::NCH_QK; ++c)
-                    tma_load_5d(sQ + c * 8192, &mq, &bars->q_full, head * D + (128 / C::QB) * c, qc.w0, qc.h0, qc.t0, b);
+                    tma_load_5d(sQ + c * C::QK_BOX, &mq, &bars->q_full, head * D + (C::QK_ROW / C::QB) * c, qc.w0,
+                                qc.h0, qc.t0, b);
             }
             const int nst = is_k ? C::NK : C::NV;
             uint64_t* full = is_k ? bars->k_full : bars->v_full;
@@ -211,16 +218,17 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     if (!is_k && C::V_ON_O) { bar = &bars->o_ready[(p - 1) & 1]; par = ((p - 1) >> 1) & 1; }
                     if (!mbar_wait(bar, par, abort_flag)) { fail(); break; }
                 }
-                // K: NCH_QK chunks of 128 / QB elements; V: NCH chunks of 64
+                // K: NCH_QK chunks of QK_ROW / QB elements; V: NCH chunks of 64
                 const int nch = is_k ? C::NCH_QK : C::NCH;
-                const int cw = is_k ? 128 / C::QB : 64;
+                const int cw = is_k ? C::QK_ROW / C::QB : 64;
+                const int cube_box = is_k ? C::QK_BOX : 8192;
                 const int pair_bytes = is_k ? C::K_PAIR_BYTES : C::V_PAIR_BYTES;
                 mbar_arrive_expect_tx(&full[st], ntl * (is_k ? C::K_CUBE_BYTES : C::V_CUBE_BYTES));
                 for (int t = 0; t < ntl; ++t) {
                     const TileCoord kc = tile_coord(g, jt[t]);
                     VSA_DEBUG_CHECK(kc.t0 < g.T && kc.h0 < g.H && kc.w0 < g.W, status, kStatusBadCoord);
                     for (int c = 0; c < nch; ++c)
-                        tma_load_5d(ring + st * pair_bytes + c * C::CHUNK_STRIDE + t * 8192, map,
+                        tma_load_5d(ring + st * pair_bytes + c * C::CHUNK_STRIDE + t * cube_box, map,
                                     &full[st], head * D + cw * c, kc.w0, kc.h0, kc.t0, b);
                 }
                 ++issued;
@@ -270,12 +278,14 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 if (!mbar_wait(&bars->k_full[sk], (p / C::NK) & 1, abort_flag)) return false;
                 tc_fence_after();
                 if constexpr (Q8) {
-                    // E4M3 codes: K = 32 per MMA, one 128-byte row per token
+                    // E4M3 codes: K = 32 per MMA, one row of D bytes per token
+                    // (8-row groups of 1024 bytes at d = 128, 512 at d = 64)
                     const uint32_t id_s = idesc_e4m3_f32(64, nkeys, false, false);
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk) {
-                        const uint64_t a = smem_desc_sw128(q_addr + kk * 32, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(k_addr + sk * C::K_PAIR_BYTES + kk * 32, 16, 1024);
+                        const uint32_t qa = q_addr + kk * 32, ka = k_addr + sk * C::K_PAIR_BYTES + kk * 32;
+                        const uint64_t a = D == 128 ? smem_desc_sw128(qa, 16, 1024) : smem_desc_sw64(qa, 16, 512);
+                        const uint64_t bd = D == 128 ? smem_desc_sw128(ka, 16, 1024) : smem_desc_sw64(ka, 16, 512);
                         mma_e4m3_ss(tS(p & 1), a, bd, id_s, kk > 0);
                     }
                 } else {
@@ -542,8 +552,9 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fine_single(const FineArgs& a, cudaStream_t stream) {
     const bool lin = a.lin_image != nullptr;
-    if (a.q_scale)                                                      // E4M3 q, k (d = 128)
+    if (a.q_scale && a.g.d == 128)                                      // E4M3 q, k
         return lin ? launch_fine_impl<128, true, true>(a, stream) : launch_fine_impl<128, false, true>(a, stream);
+    if (a.q_scale) return lin ? launch_fine_impl<64, true, true>(a, stream) : launch_fine_impl<64, false, true>(a, stream);
     if (a.g.d == 128) return lin ? launch_fine_impl<128, true>(a, stream) : launch_fine_impl<128, false>(a, stream);
     return lin ? launch_fine_impl<64, true>(a, stream) : launch_fine_impl<64, false>(a, stream);
 }

@@ -234,8 +234,8 @@ vsa_status vsa_quantize_qk_e4m3(const vsa_bf16* q, const vsa_bf16* k, uint8_t* q
 /* Step 2, vsa_sparse_attn_fwd_e4m3: the fine pass of vsa_sparse_attn_fwd with
  * Q K^T on the tensor cores in E4M3 (fp32 accumulation), scores rescaled by
  * q_scale[query cube] * k_scale[key cube], softmax and P V as in the bf16
- * pass (bf16 P and v), output bf16 in grid order.  head_dim 128 only
- * (VSA_ERR_UNSUPPORTED otherwise); the linear branch is added by
+ * pass (bf16 P and v), output bf16 in grid order.  head_dim 64 or 128; the
+ * linear branch is added by
  * vsa_sparse_linear_attn_fwd_e4m3 below.  Needs
  * vsa_workspace_bytes() of workspace (status word only). */
 vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,
@@ -253,8 +253,8 @@ vsa_status vsa_sparse_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const 
  * from the bf16 q (the quantisation covers the sparse branch's Q K^T only;
  * the branch's products run as bf16 hi + lo pairs, fp32-level, as in
  * vsa_sparse_attn_fwd).  q8, k8, q_scale, k_scale from vsa_quantize_qk_e4m3;
- * q, v bf16 [B][N][heads][d].  head_dim 128 only (VSA_ERR_UNSUPPORTED
- * otherwise).  All pointers 16-byte aligned (VSA_ERR_INVALID_ARGUMENT).
+ * q, v bf16 [B][N][heads][d].  head_dim 64 or 128.  All pointers 16-byte
+ * aligned (VSA_ERR_INVALID_ARGUMENT).
  * Needs vsa_workspace_bytes() of workspace: the status word plus the
  * operand image of (S, z) (VSA_ERR_WORKSPACE when smaller). */
 vsa_status vsa_sparse_linear_attn_fwd_e4m3(const uint8_t* q8, const uint8_t* k8, const float* q_scale,

@@ -131,13 +131,13 @@ def test_other_entry_points_validate(L):
     assert qz(*[FAKE] * 6, 1, 2, 96, 4, 8, 8, 4, 4, 4, None) == UNSUPPORTED
     assert qz(FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, 1, 2, 128, 4, 8, 8, 4, 4, 4, None) == INVALID
     fe = L.vsa_sparse_attn_fwd_e4m3
-    assert fe(*[FAKE] * 7, 1, 2, 64, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == UNSUPPORTED   # d = 64
+    assert fe(*[FAKE] * 7, 1, 2, 96, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == UNSUPPORTED   # d = 96
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 5, FAKE, 1024, None) == INVALID     # topk > nt
     assert fe(*[FAKE] * 6, FAKE + 2, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1024, None) == INVALID
     assert fe(*[FAKE] * 7, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 8, None) == WORKSPACE
     fl = L.vsa_sparse_linear_attn_fwd_e4m3                 # q8 k8 sq sk q v idx S z out
     image = 2 * (4 * 128 * 128 + 4 * 128)
-    assert fl(*[FAKE] * 10, 1, 2, 64, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == UNSUPPORTED   # d = 64
+    assert fl(*[FAKE] * 10, 1, 2, 96, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == UNSUPPORTED   # d = 96
     assert fl(*[FAKE] * 10, 1, 2, 128, 4, 8, 8, 4, 4, 4, 0, FAKE, 1 << 20, None) == INVALID     # topk < 1
     assert fl(*[FAKE] * 7, None, FAKE, FAKE, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == INVALID
     assert fl(*[FAKE] * 4, FAKE + 2, *[FAKE] * 5, 1, 2, 128, 4, 8, 8, 4, 4, 4, 2, FAKE, 1 << 20, None) == INVALID

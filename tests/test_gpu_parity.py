@@ -697,11 +697,14 @@ def test_training_gradients_both_branches_batch_of_two(ops):
 E4M3_REL_FRO, E4M3_MAX_REL = 5e-2, 0.1
 
 E4M3_CASES = [
-    # B, T, H, W, heads, topk
-    (1, 4, 8, 8, 2, 2),          # 4 cubes, even k
-    (1, 5, 6, 7, 3, 3),          # ragged on every axis, odd k, heads not a multiple of 4
-    (2, 8, 16, 16, 5, 8),        # B = 2, 5 heads
-    (1, 6, 10, 9, 2, 9),         # ragged, several pairs + odd tail
+    # B, T, H, W, heads, topk, d
+    (1, 4, 8, 8, 2, 2, 128),     # 4 cubes, even k
+    (1, 5, 6, 7, 3, 3, 128),     # ragged on every axis, odd k, heads not a multiple of 4
+    (2, 8, 16, 16, 5, 8, 128),   # B = 2, 5 heads
+    (1, 6, 10, 9, 2, 9, 128),    # ragged, several pairs + odd tail
+    (1, 4, 8, 8, 2, 2, 64),      # d = 64: 64-byte rows
+    (1, 9, 13, 10, 3, 5, 64),    # d = 64, ragged, odd k
+    (2, 8, 16, 16, 2, 7, 64),    # d = 64, B = 2, several pairs + odd tail
 ]
 
 
@@ -722,12 +725,12 @@ def run_e4m3(ops, q, k, v, T, H, W, topk):
 
 @pytest.mark.parametrize("case", E4M3_CASES)
 def test_e4m3_quantise_and_fine(ops, case):
-    B, T, H, W, heads, topk = case
-    q, k, v = synth.make_qkv(B, heads, 128, T, H, W, amplitude=0.7, seed=sum(case))
+    B, T, H, W, heads, topk, d = case
+    q, k, v = synth.make_qkv(B, heads, d, T, H, W, amplitude=0.7, seed=sum(case))
     idx, q8, k8, sq, sk, out = run_e4m3(ops, q, k, v, T, H, W, topk)
     # quantisation: codes and scales bit for bit
-    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, 128, T, H, W)
-    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, 128, T, H, W)
+    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, d, T, H, W)
+    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, d, T, H, W)
     np.testing.assert_array_equal(q8.cpu().numpy(), cq)
     np.testing.assert_array_equal(k8.cpu().numpy(), ck)
     np.testing.assert_array_equal(sq.cpu().numpy(), sq_ref)
@@ -736,12 +739,12 @@ def test_e4m3_quantise_and_fine(ops, case):
     idx_np = idx.cpu().numpy()
     qh = O.dequant_e4m3_cubes(cq, sq_ref, T, H, W)
     kh = O.dequant_e4m3_cubes(ck, sk_ref, T, H, W)
-    ref_q = O.fine_real(qh, kh, v, idx_np, B, heads, 128, T, H, W)
+    ref_q = O.fine_real(qh, kh, v, idx_np, B, heads, d, T, H, W)
     got = to_f64(out)
     assert not np.isnan(got).any()
     check_close(got, ref_q)
     # and against the exact bf16 oracle, with the stated looser bound
-    ref = O.fine(q, k, v, idx_np, B, heads, 128, T, H, W)
+    ref = O.fine(q, k, v, idx_np, B, heads, d, T, H, W)
     err = np.abs(got - ref).max()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     print(f"vs exact: max-abs {err:.3e} (scale {np.abs(ref).max():.3e}), rel-Frobenius {rel:.3%}")
@@ -749,7 +752,8 @@ def test_e4m3_quantise_and_fine(ops, case):
 
 
 def test_e4m3_quantise_d64_bit_exact(ops):
-    """The quantisation kernel also serves d = 64 (the E4M3 fine pass is d = 128)."""
+    """The quantisation kernel at d = 64 on a ragged grid, codes and scales bit
+    for bit."""
     B, T, H, W, heads = 1, 9, 13, 10, 3
     q, k, _ = synth.make_qkv(B, heads, 64, T, H, W, amplitude=0.7, seed=4)
     nt = ops.vsa_num_tiles(T, H, W)
@@ -818,21 +822,21 @@ def test_e4m3_linear_small_full(ops, case):
     the oracle's fine pass on the dequantised q, k plus its linear branch on
     the bf16 q, k, v (the bf16 bar), and against the exact oracle (fine pass on
     bf16 q, k) within the stated E4M3 bound."""
-    B, T, H, W, heads, topk = case
-    q, k, v = synth.make_qkv(B, heads, 128, T, H, W, amplitude=0.7, seed=sum(case) + 3)
+    B, T, H, W, heads, topk, d = case
+    q, k, v = synth.make_qkv(B, heads, d, T, H, W, amplitude=0.7, seed=sum(case) + 3)
     idx, out = run_e4m3_linear(ops, q, k, v, T, H, W, topk)
     idx_np = idx.cpu().numpy()
     N = T * H * W
-    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, 128, T, H, W)
-    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, 128, T, H, W)
+    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, d, T, H, W)
+    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, d, T, H, W)
     qh = O.dequant_e4m3_cubes(cq, sq_ref, T, H, W)
     kh = O.dequant_e4m3_cubes(ck, sk_ref, T, H, W)
-    Sr, zr = O.linear_state(k, v, B, heads, 128, N)
-    lin = O.linear_apply(q, Sr, zr, B, heads, 128, N)
+    Sr, zr = O.linear_state(k, v, B, heads, d, N)
+    lin = O.linear_apply(q, Sr, zr, B, heads, d, N)
     got = to_f64(out)
     assert not np.isnan(got).any()
-    check_close(got, O.fine_real(qh, kh, v, idx_np, B, heads, 128, T, H, W) + lin)
-    ref = O.fine(q, k, v, idx_np, B, heads, 128, T, H, W) + lin
+    check_close(got, O.fine_real(qh, kh, v, idx_np, B, heads, d, T, H, W) + lin)
+    ref = O.fine(q, k, v, idx_np, B, heads, d, T, H, W) + lin
     err = np.abs(got - ref).max()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert err <= E4M3_MAX_REL * np.abs(ref).max() and rel <= E4M3_REL_FRO, (err, rel)
