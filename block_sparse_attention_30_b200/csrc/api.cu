@@ -160,6 +160,7 @@ vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int he
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(block_idx)) return VSA_ERR_INVALID_ARGUMENT;
     if (!aligned16(workspace)) return VSA_ERR_WORKSPACE;
+    if (!vsa::select_supported(g)) return VSA_ERR_UNSUPPORTED;
     if (workspace_bytes < kStatusBytes + vsa::select_scratch_bytes(g)) return VSA_ERR_WORKSPACE;
     vsa::SelectArgs a;
     a.g = g;

@@ -105,6 +105,7 @@ vsa_status vsa_select_blocks_noalloc(const vsa_bf16* q, const vsa_bf16* k, int B
     const vsa::Grid g = vsa::make_grid(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(block_idx)) return VSA_ERR_INVALID_ARGUMENT;
+    if (!vsa::select_supported(g)) return VSA_ERR_UNSUPPORTED;
     if (vsa::select_scratch_bytes(g) > (size_t)VSA_NOALLOC_SELECT_SCRATCH_BYTES)
         return VSA_ERR_WORKSPACE;
     void* scratch = nullptr;

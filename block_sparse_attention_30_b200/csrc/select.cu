@@ -713,6 +713,9 @@ select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, co
 // (2 * 2 * B * heads * nt * d * 4 bytes), the feature-major copy of the k hi
 // means (B * heads * d * ntp * 4 bytes, ntp = nt rounded up to 4) and one
 // fallback row of nt 64-bit keys per CTA.
+// The 16 score rows of a work item must fit one CTA's shared memory.
+bool select_supported(const Grid& g) { return sel_smem_bytes(g.nt, g.d) <= 232448; }
+
 size_t select_scratch_bytes(const Grid& g) {
     const size_t pooled = 4ull * g.B * g.heads * g.nt * g.d * sizeof(float);
     const size_t kt = (size_t)g.B * g.heads * g.d * sel_ntp(g.nt) * sizeof(float);
@@ -727,7 +730,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
     float* kt = pooled + 4ull * g.B * g.heads * g.nt * g.d;
     unsigned long long* fallback = reinterpret_cast<unsigned long long*>(kt + (size_t)g.B * g.heads * g.d * sel_ntp(g.nt));
     const size_t smem = sel_smem_bytes(g.nt, g.d);
-    if (smem > 232448) return cudaErrorInvalidValue;    // nt beyond ~3400 cubes
+    if (!select_supported(g)) return cudaErrorInvalidValue;   // refused earlier by the entry points
     static int configured_device = -1, sms = 0;         // per process: once per device
     int dev = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);

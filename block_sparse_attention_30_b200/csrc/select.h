@@ -18,6 +18,7 @@ struct SelectArgs {
     int* status;            // device status word (timeouts), or null
 };
 
+bool select_supported(const Grid& g);   // nt small enough for the score rows in shared memory
 size_t select_scratch_bytes(const Grid& g);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 

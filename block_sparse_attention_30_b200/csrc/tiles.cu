@@ -15,13 +15,16 @@
 
 namespace vsa {
 
-// One CTA per (cube j, batch b).  For each of the cube's slots the token row
-// -- all heads, heads*d bf16, contiguous in grid order -- is copied with
-// 16-byte vectors; in cube-major order the same vector lands in row
-// ((b*heads + head)*nt + j)*vol + slot.  Consecutive threads take consecutive
-// vectors of one row, so reads cover whole 128-byte lines of grid order and
-// writes whole d-wide rows of cube-major order.  Four slots are in flight per
-// thread.
+// One CTA per (cube j, batch b, group of kSlotsPerCta slots).  For each of its
+// slots the token row -- all heads, heads*d bf16, contiguous in grid order --
+// is copied with 16-byte vectors; in cube-major order the same vector lands
+// in row ((b*heads + head)*nt + j)*vol + slot.  Consecutive threads take
+// consecutive vectors of one row, so reads cover whole 128-byte lines of grid
+// order and writes whole d-wide rows of cube-major order.  Four slots are in
+// flight per thread; splitting a cube's slots over several CTAs gives the
+// small grids (a few hundred cubes) enough CTAs to fill every SM.
+constexpr int kSlotsPerCta = 16;
+
 template <bool GATHER, int VPR>     // VPR: 16-byte vectors per (slot, head) row = d/8
 __global__ void __launch_bounds__(256)
 tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const Grid g) {
@@ -29,7 +32,8 @@ tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const G
     const int vol = g.tt * g.th * g.tw;
     const int it = j / (g.nh * g.nw), ih = (j / g.nw) % g.nh, iw = j % g.nw;
     const int row_vec = g.heads * VPR;                       // vectors per token row
-    for (int s0 = 0; s0 < vol; s0 += 4) {
+    const int s_end = min(vol, ((int)blockIdx.z + 1) * kSlotsPerCta);
+    for (int s0 = blockIdx.z * kSlotsPerCta; s0 < s_end; s0 += 4) {
         long long n[4];
         bool valid[4];
 #pragma unroll
@@ -37,7 +41,7 @@ tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const G
             const int s = s0 + u;
             const int dt = s / (g.th * g.tw), dh = (s / g.tw) % g.th, dw = s % g.tw;
             const int t = it * g.tt + dt, h = ih * g.th + dh, w = iw * g.tw + dw;
-            valid[u] = s < vol && t < g.T && h < g.H && w < g.W;
+            valid[u] = s < s_end && t < g.T && h < g.H && w < g.W;
             n[u] = ((long long)t * g.H + h) * g.W + w;
         }
         for (int v = threadIdx.x; v < row_vec; v += blockDim.x) {
@@ -53,7 +57,7 @@ tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const G
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if (s0 + u >= vol) continue;
+                if (s0 + u >= s_end) continue;
                 const long long gi = ((long long)b * g.N + n[u]) * row_vec + v;
                 const long long ti = (tile_row + s0 + u) * VPR + c;
                 if (GATHER) dst[ti] = val[u];
@@ -66,7 +70,7 @@ tile_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const G
 template <bool GATHER>
 static cudaError_t launch_copy(const Grid& g, const void* src, void* dst, cudaStream_t stream) {
     if ((long long)g.B * g.nt == 0) return cudaSuccess;
-    const dim3 grid(g.nt, g.B);
+    const dim3 grid(g.nt, g.B, ceil_div_i(g.tt * g.th * g.tw, kSlotsPerCta));
     const uint4* s = reinterpret_cast<const uint4*>(src);
     uint4* d = reinterpret_cast<uint4*>(dst);
     if (g.d == 128) tile_copy_kernel<GATHER, 16><<<grid, 256, 0, stream>>>(s, d, g);

@@ -123,8 +123,9 @@ vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int he
  * topk key cubes with the largest C (ties -> lower j) in ascending order to
  * block_idx.  The kept set is the one fp64 scores give: the scores are formed
  * in fp32 with a bound on their error, and every score the bound leaves
- * undecided is recomputed in fp64.  1 <= topk <= nt; nt up to about 3400
- * cubes (VSA_ERR_CUDA beyond).  Needs vsa_workspace_bytes() of workspace.
+ * undecided is recomputed in fp64.  1 <= topk <= nt; nt up to about 3200
+ * cubes (the 16 score rows of a work item live in shared memory: 64*nt +
+ * 64*d + 14464 bytes must fit 227 KB, VSA_ERR_UNSUPPORTED beyond).  Needs vsa_workspace_bytes() of workspace.
  * One kernel (after a 8-byte memset of its work counters): the cube means
  * go through the workspace, the nt x nt scores only through shared memory. */
 vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,

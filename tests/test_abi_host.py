@@ -92,6 +92,11 @@ def test_select_argument_validation(L):
     assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == UNSUPPORTED
     bad = list(SHAPE); bad[6] = 2
     assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == UNSUPPORTED
+    # 3300 cubes: 16 score rows of 3300 fp32 values no longer fit a CTA's
+    # shared memory beside the rest of a work item's state
+    wide = [1, 1, 128, 4, 4, 4 * 3300, 4, 4, 4]
+    assert f(FAKE, FAKE, *wide, 2, FAKE, FAKE, big, None) == UNSUPPORTED
+    assert L.vsa_select_blocks_noalloc(FAKE, FAKE, *wide, 2, FAKE, None) == UNSUPPORTED
     bad = list(SHAPE); bad[3] = 0
     assert f(FAKE, FAKE, *bad, 2, FAKE, FAKE, big, None) == INVALID
 
