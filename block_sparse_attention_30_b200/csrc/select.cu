@@ -602,18 +602,31 @@ __device__ void score_item(const Grid& g, const int topk, const int item, const 
             }
             if (!got) { if (lane == 0) report(status, kStatusTimeout); continue; }
             unsigned long long* keys = fallback + (long long)blockIdx.x * nt;
+            // the query row in fp64 in this warp's histogram bins (d <= 128
+            // doubles = 1 KB; the radix select below reuses them afterwards),
+            // then each lane the fp64 score of its own band cube, 32 at a time
+            double* qs = reinterpret_cast<double*>(hist);
+            const float* qh = Qh + (long long)i * d;
+            const float* ql = Ql + (long long)i * d;
+            for (int c = lane; c < d; c += 32) qs[c] = (double)__ldcg(qh + c) + (double)__ldcg(ql + c);
+            __syncwarp();
             for (int j0 = 0; j0 < nt; j0 += 32) {
                 const int j = j0 + lane;
                 const float v = j < nt ? row[j] : -INFINITY;
                 const bool gt = v > hi, band = j < nt && !gt && v >= lo;
-                unsigned bb = __ballot_sync(0xffffffffu, band);
                 unsigned long long key = gt ? ~0ull : 0ull;
-                while (bb) {                                // one warp-wide dot per band cube
-                    const int src = __ffs(bb) - 1;
-                    bb &= bb - 1;
-                    const int jj = j0 + src;
-                    const double s = warp_sum_f64(qrow.partial(Kh + (long long)jj * d, Kl + (long long)jj * d, lane)) * inv_sqrt_d;
-                    if (lane == src) key = f64_key(s);
+                if (band) {
+                    const float4* kh4 = reinterpret_cast<const float4*>(Kh + (long long)j * d);
+                    const float4* kl4 = reinterpret_cast<const float4*>(Kl + (long long)j * d);
+                    double sacc = 0.0;
+                    for (int c4 = 0; c4 < d / 4; ++c4) {
+                        const float4 h = __ldcg(kh4 + c4), l = __ldcg(kl4 + c4);
+                        sacc = fma(qs[4 * c4], (double)h.x + l.x, sacc);
+                        sacc = fma(qs[4 * c4 + 1], (double)h.y + l.y, sacc);
+                        sacc = fma(qs[4 * c4 + 2], (double)h.z + l.z, sacc);
+                        sacc = fma(qs[4 * c4 + 3], (double)h.w + l.w, sacc);
+                    }
+                    key = f64_key(sacc * inv_sqrt_d);
                 }
                 if (j < nt) keys[j] = key;
             }

@@ -172,6 +172,29 @@ def test_ties_beyond_the_refined_candidates(ops, levels, topk):
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
 
 
+def test_selection_all_scores_tied(ops):
+    """q = 0: every coarse score of a row is exactly 0, so every cube is in the
+    error band and every row takes the fallback (fp64 keys for the whole row
+    and the radix select); the tie rule keeps cubes 0 .. k-1.  At a 14B-480P
+    sized grid (455 cubes), timed, so that this degenerate input stays within
+    a small factor of the regular selection."""
+    T, H, W, heads, d, topk = 20, 28, 52, 4, 128, 46
+    c = Small(T, H, W, heads, d, topk, seed=6)
+    q0 = torch.zeros_like(c.q).cuda()
+    kd = c.k.cuda()
+    idx, ws = run_select(ops, c, q0, kd)
+    nt = ops.vsa_num_tiles(T, H, W)
+    want = np.broadcast_to(np.arange(topk, dtype=np.int32), (1, heads, nt, topk))
+    np.testing.assert_array_equal(idx.cpu().numpy(), want)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    ops.vsa_select_blocks(q0, kd, T, H, W, topk, idx, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"all-tied selection: {e0.elapsed_time(e1):.3f} ms for {heads * nt} rows")
+    assert e0.elapsed_time(e1) < 50.0
+
+
 def test_selection_keeps_every_cube_at_k_equal_nt(ops):
     T, H, W, heads, d = 8, 12, 12, 3, 64                 # 2 x 3 x 3 = 18 cubes
     c = Small(T, H, W, heads, d, 18, seed=4)
