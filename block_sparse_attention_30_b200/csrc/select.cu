@@ -7,7 +7,8 @@
 // indices emitted ascending) is this library's reading of that outline.
 //
 // One persistent kernel, select_kernel, does the whole selection.  Its CTAs
-// claim work items from an atomic counter, per group of up to 8 heads:
+// claim work items from an atomic counter, per group of 8 heads (more per
+// group beyond 504 heads, so that at most 63 groups need counters):
 //   pool items   one per (cubes j0 .. j0 + cpi - 1, batch, q|k) of the group:
 //                16-byte vector loads of the cubes' valid token rows (the
 //                group's heads, contiguous within a token row), fp64 sums,
