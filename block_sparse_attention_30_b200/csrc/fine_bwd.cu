@@ -178,12 +178,19 @@ struct BwdCfg {
     static constexpr int ACC_COL = 0;                    // dQ | dV (lanes 0-15), dK (lanes 16-31)
     static constexpr int S_COL = 128;                    // S buffer b at S_COL + 64 b: S / P (lanes 0-15),
                                                          // dP / dS (lanes 16-31)
-    static constexpr int SMEM = 6 * CUBE_BYTES + 1024 + 256;  // own 2 cubes + 2 x 2 slots, lse/D, barriers
+    // dQ body: own Q, dO + 3 K slots + 2 V slots; dK/dV body: own K, V + 2 Q
+    // slots + 2 dO slots + their lse / D; barriers after either
+    static constexpr int SMEM_DQ = 7 * CUBE_BYTES;
+    static constexpr int SMEM_DKDV = 6 * CUBE_BYTES + 1024;
+    static constexpr int SMEM = (SMEM_DQ > SMEM_DKDV ? SMEM_DQ : SMEM_DKDV) + 256;
+    static constexpr int NK = 3;                         // dQ body's K slots
 };
+
+static_assert(BwdCfg<128>::SMEM <= 232448 / 2 - 1024, "two CTAs per SM");
 
 struct BwdBars {
     uint64_t a_full;                 // the CTA's own cubes: Q + dO, or K + V
-    uint64_t x_full[2], x_empty[2];  // ring 1 (K cubes / Q cubes + lse)
+    uint64_t x_full[3], x_empty[3];  // ring 1 (K cubes: 3 slots / Q cubes + lse: 2 slots)
     uint64_t y_full[2], y_empty[2];  // ring 2 (V cubes / dO cubes + D)
     uint64_t s_full[2], ds_full[2], mma_done;
     uint32_t tmem_base;
@@ -267,9 +274,10 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
     using C = BwdCfg<D>;
     uint8_t* sQ = smem;
     uint8_t* sG = sQ + C::CUBE_BYTES;
-    uint8_t* sK = sG + C::CUBE_BYTES;                 // 2 slots
-    uint8_t* sV = sK + 2 * C::CUBE_BYTES;             // 2 slots
-    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + 6 * C::CUBE_BYTES + 1024);
+    uint8_t* sK = sG + C::CUBE_BYTES;                 // NK = 3 slots: a K cube is read by S and,
+                                                      // after the softmax, by dQ
+    uint8_t* sV = sK + C::NK * C::CUBE_BYTES;         // 2 slots (read by dP only)
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::SMEM_DQ);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i = (int)(row_id % g.nt);
@@ -281,10 +289,10 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
         bars->abort = 0;
         mbar_init(&bars->a_full, 1);
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&bars->x_full[x], 1); mbar_init(&bars->x_empty[x], 1);
             mbar_init(&bars->y_full[x], 1); mbar_init(&bars->y_empty[x], 1);
             mbar_init(&bars->s_full[x], 1); mbar_init(&bars->ds_full[x], 128);
         }
+        for (int x = 0; x < C::NK; ++x) { mbar_init(&bars->x_full[x], 1); mbar_init(&bars->x_empty[x], 1); }
         mbar_init(&bars->mma_done, 1);
         fence_barrier_init();
     }
@@ -297,7 +305,10 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
 
     if (warp == 4 || warp == 6) {
         if (lane == 0) {
+            // step t uses K slot t % 3 (released by dQ of step t - 3) and V
+            // slot t % 2 (released by dP of step t - 2)
             const bool is_k = warp == 4;
+            const int nslot = is_k ? C::NK : 2;
             uint64_t* full = is_k ? bars->x_full : bars->y_full;
             uint64_t* empty = is_k ? bars->x_empty : bars->y_empty;
             uint8_t* ring = is_k ? sK : sV;
@@ -311,15 +322,16 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
             for (int t = 0; t < topk; ++t) {
                 int j = __ldg(my_idx + t);
                 if (j < 0 || j >= g.nt) { if (is_k) report(status, kStatusBadIndex); j = 0; }
-                const int x = t & 1;
-                if (t >= 2 && !mbar_wait(&empty[x], ((t >> 1) - 1) & 1, abort_flag)) { fail(); break; }
+                const int x = t % nslot;
+                if (t >= nslot && !mbar_wait(&empty[x], ((t / nslot) - 1) & 1, abort_flag)) { fail(); break; }
                 mbar_arrive_expect_tx(&full[x], C::CUBE_BYTES);
                 load_cube<D>(ring + x * C::CUBE_BYTES, map, &full[x], g, j, head, b);
                 ++issued;
             }
             if (*abort_flag) {
                 if (is_k) wait_noabort(&bars->a_full, 0);
-                for (int n = issued > 2 ? issued - 2 : 0; n < issued; ++n) wait_noabort(&full[n & 1], (n >> 1) & 1);
+                for (int n = issued > nslot ? issued - nslot : 0; n < issued; ++n)
+                    wait_noabort(&full[n % nslot], (n / nslot) & 1);
             }
         }
     } else if (warp == 5) {
@@ -328,11 +340,11 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
             const uint32_t tAcc = tbase + C::ACC_COL;
             auto sbuf = [&](int x) { return tbase + C::S_COL + 64 * x; };
             auto issue_s = [&](int t) -> bool {
-                const int x = t & 1;
-                if (!mbar_wait(&bars->x_full[x], (t >> 1) & 1, abort_flag) ||
+                const int x = t & 1, xk = t % C::NK;
+                if (!mbar_wait(&bars->x_full[xk], (t / C::NK) & 1, abort_flag) ||
                     !mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_s_dp<D>(sbuf(x), q_addr, smem_u32(sK + x * C::CUBE_BYTES), g_addr,
+                issue_s_dp<D>(sbuf(x), q_addr, smem_u32(sK + xk * C::CUBE_BYTES), g_addr,
                               smem_u32(sV + x * C::CUBE_BYTES));
                 mma_commit(&bars->s_full[x]);
                 mma_commit(&bars->y_empty[x]);             // V cube read by dP only
@@ -344,8 +356,8 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
                 const int x = t & 1;
                 if (!mbar_wait(&bars->ds_full[x], (t >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                issue_acc<D>(tAcc, sbuf(x), smem_u32(sK + x * C::CUBE_BYTES), t > 0);   // dQ += dS K
-                mma_commit(&bars->x_empty[x]);
+                issue_acc<D>(tAcc, sbuf(x), smem_u32(sK + (t % C::NK) * C::CUBE_BYTES), t > 0);   // dQ += dS K
+                mma_commit(&bars->x_empty[t % C::NK]);
                 if (t + 2 < topk && !issue_s(t + 2)) { ok = false; break; }
             }
             if (!ok) fail();
@@ -427,7 +439,7 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
     uint8_t* sG = sQ + 2 * C::CUBE_BYTES;             // 2 slots
     float* sL = reinterpret_cast<float*>(smem + 6 * C::CUBE_BYTES);   // lse of the slots' query cubes [2][64]
     float* sD = sL + 128;                                              // D of the slots' query cubes [2][64]
-    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + 6 * C::CUBE_BYTES + 1024);
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::SMEM_DKDV);
     volatile int* abort_flag = &bars->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = (int)(row_id % g.nt);           // row_id = (b*heads + head)*nt + j
