@@ -865,6 +865,56 @@ def test_e4m3_linear_small_full(ops, case):
     assert err <= E4M3_MAX_REL * np.abs(ref).max() and rel <= E4M3_REL_FRO, (err, rel)
 
 
+def test_e4m3_tiny_workload_full(ops):
+    """The tiny configuration (d = 64, 4 x 32 x 32 grid, k = 13 of 64) through
+    the E4M3 pass with and without the linear branch, every output element."""
+    w, q, k, v, qd, kd, vd = inputs("tiny_4x32x32")
+    B, heads, d = w.B, w.heads, w.head_dim
+    idx, q8, k8, sq, sk, out = run_e4m3(ops, q, k, v, w.T, w.H, w.W, w.topk)
+    idx_np = idx.cpu().numpy()
+    cq, sq_ref = O.quant_e4m3_cubes(q, B, heads, d, w.T, w.H, w.W)
+    ck, sk_ref = O.quant_e4m3_cubes(k, B, heads, d, w.T, w.H, w.W)
+    np.testing.assert_array_equal(q8.cpu().numpy(), cq)
+    np.testing.assert_array_equal(k8.cpu().numpy(), ck)
+    qh = O.dequant_e4m3_cubes(cq, sq_ref, w.T, w.H, w.W)
+    kh = O.dequant_e4m3_cubes(ck, sk_ref, w.T, w.H, w.W)
+    ref_q = O.fine_real(qh, kh, v, idx_np, B, heads, d, w.T, w.H, w.W)
+    check_close(to_f64(out), ref_q)
+    _, out_lin = run_e4m3_linear(ops, q, k, v, w.T, w.H, w.W, w.topk)
+    Sr, zr = O.linear_state(k, v, B, heads, d, w.N)
+    check_close(to_f64(out_lin), ref_q + O.linear_apply(q, Sr, zr, B, heads, d, w.N))
+
+
+def test_e4m3_linear_headline_sampled(ops):
+    """SageSLA at the 14B-480P shape (the E4M3 one-cube kernel at k = 46 with
+    the linear branch): sampled query cubes of two heads against the oracle
+    on the dequantised q, k plus the linear branch on bf16 q, k, v."""
+    w, q, k, v, qd, kd, vd = inputs("wan14b_480p")
+    idx, out = run_e4m3_linear(ops, q, k, v, w.T, w.H, w.W, w.topk)
+    nt = w.num_tiles
+    hs = [0, 1]
+    sub = lambda x: x[:, :, hs].contiguous()
+    cq, sq_ref = O.quant_e4m3_cubes(sub(q), 1, 2, 128, w.T, w.H, w.W)
+    ck, sk_ref = O.quant_e4m3_cubes(sub(k), 1, 2, 128, w.T, w.H, w.W)
+    qh = O.dequant_e4m3_cubes(cq, sq_ref, w.T, w.H, w.W)
+    kh = O.dequant_e4m3_cubes(ck, sk_ref, w.T, w.H, w.W)
+    Sr, zr = O.linear_state(sub(k), sub(v), 1, 2, 128, w.N)
+    rows = np.arange(0, 2 * nt, 37)
+    idx2 = idx[:, hs].cpu().numpy()
+    part = O.fine_tiles_real(qh, kh, sub(v), idx2, rows, 1, 2, 128, w.T, w.H, w.W)
+    slots = O.tile_slots(w.T, w.H, w.W)
+    got, ref = [], []
+    for r, row in enumerate(rows):
+        head, i = divmod(int(row), nt)
+        ok = slots[i] >= 0
+        toks = slots[i][ok]
+        qrow = q[:, torch.as_tensor(toks), head:head + 1].contiguous()
+        lin = O.linear_apply(qrow, Sr[:, head:head + 1], zr[:, head:head + 1], 1, 1, 128, len(toks))[0, :, 0]
+        ref.append(part[r][ok] + lin)
+        got.append(to_f64(out[0, torch.as_tensor(toks), head]))
+    check_close(np.concatenate(got), np.concatenate(ref))
+
+
 def test_e4m3_linear_sparse97_sampled(ops):
     """The 97 %-sparsity + linear-branch workload with E4M3 Q K^T: sampled query
     cubes against the oracle on the dequantised q, k plus the linear branch on
