@@ -644,6 +644,7 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     int32_t* off = reinterpret_cast<int32_t*>(scratch + up(rows * 64 * sizeof(float)));
     int32_t* ents = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(off) +
                                                up((size_t)g.B * g.heads * (g.nt + 1) * sizeof(int32_t)));
+    if (2 * rows > 0x7fffffffll) return cudaErrorInvalidConfiguration;   // a dQ and a dK/dV CTA per cube
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (g.T % g.tt) || (g.H % g.th) || (g.W % g.tw);
 

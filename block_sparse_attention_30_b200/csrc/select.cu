@@ -727,8 +727,12 @@ select_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, co
 // (2 * 2 * B * heads * nt * d * 4 bytes), the feature-major copy of the k hi
 // means (B * heads * d * ntp * 4 bytes, ntp = nt rounded up to 4) and one
 // fallback row of nt 64-bit keys per CTA.
-// The 16 score rows of a work item must fit one CTA's shared memory.
-bool select_supported(const Grid& g) { return sel_smem_bytes(g.nt, g.d) <= 232448; }
+// The 16 score rows of a work item must fit one CTA's shared memory, and the
+// work items (claimed through a 32-bit counter) must number fewer than 2^30.
+bool select_supported(const Grid& g) {
+    const long long items = 2ll * g.B * g.nt * ceil_div_i(g.heads, 8) + (long long)g.B * g.heads * ceil_div_i(g.nt, kSelRows);
+    return sel_smem_bytes(g.nt, g.d) <= 232448 && items < (1ll << 30);
+}
 
 size_t select_scratch_bytes(const Grid& g) {
     const size_t pooled = 4ull * g.B * g.heads * g.nt * g.d * sizeof(float);
