@@ -25,10 +25,15 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 vsa_status check_shape(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {
     switch (vsa::shape_error(B, heads, d, T, H, W, tt, th, tw)) {
-        case 0: return VSA_OK;
+        case 0: break;
         case 2: return VSA_ERR_UNSUPPORTED;
         default: return VSA_ERR_INVALID_ARGUMENT;
     }
+    // the fine pass and its backward launch one or two CTAs per (b, head,
+    // query cube): at most 2^30 cubes in all
+    const long long nt = (long long)vsa::ceil_div_i(T, tt) * vsa::ceil_div_i(H, th) * vsa::ceil_div_i(W, tw);
+    if ((long long)B * heads * nt >= (1ll << 30)) return VSA_ERR_UNSUPPORTED;
+    return VSA_OK;
 }
 
 vsa::Grid grid_of(int B, int heads, int d, int T, int H, int W, int tt, int th, int tw) {

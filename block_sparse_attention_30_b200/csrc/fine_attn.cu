@@ -541,7 +541,6 @@ static cudaError_t launch_fine_impl(const FineArgs& a, cudaStream_t stream) {
         configured_device = dev;
     }
     const long long rows = (long long)a.g.B * a.g.heads * a.g.nt;
-    if (rows > 0x7fffffffll) return cudaErrorInvalidConfiguration;   // one CTA per query cube
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (a.g.T % a.g.tt) || (a.g.H % a.g.th) || (a.g.W % a.g.tw);
     fine_attn_kernel<D, LIN, Q8><<<(unsigned)rows, 224, C::SMEM_BYTES, stream>>>(

@@ -69,7 +69,8 @@ typedef struct CUstream_st* vsa_stream_t;  /* == cudaStream_t              */
 typedef enum {
     VSA_OK = 0,
     VSA_ERR_INVALID_ARGUMENT = 1,  /* bad shape, null/misaligned pointer, bad topk */
-    VSA_ERR_UNSUPPORTED = 2,       /* head_dim not in {64,128}, tile volume != 64  */
+    VSA_ERR_UNSUPPORTED = 2,       /* head_dim not in {64,128}, tile volume != 64,
+                                      2^30 or more cubes in all (B*heads*nt)   */
     VSA_ERR_WORKSPACE = 3,         /* workspace missing or smaller than required   */
     VSA_ERR_CUDA = 4,              /* a CUDA runtime/driver call or launch failed  */
     VSA_ERR_TIMEOUT = 5,           /* a device-side bounded wait gave up           */
@@ -125,9 +126,10 @@ vsa_status vsa_scatter_tiles(const vsa_bf16* x_tiles, vsa_bf16* x, int B, int he
  * in fp32 with a bound on their error, and every score the bound leaves
  * undecided is recomputed in fp64.  1 <= topk <= nt; nt up to about 3200
  * cubes (the 16 score rows of a work item live in shared memory: 64*nt +
- * 64*d + 14464 bytes must fit 227 KB, VSA_ERR_UNSUPPORTED beyond).  Needs vsa_workspace_bytes() of workspace.
- * One kernel (after a 8-byte memset of its work counters): the cube means
- * go through the workspace, the nt x nt scores only through shared memory. */
+ * 64*d + 14464 bytes must fit 227 KB, VSA_ERR_UNSUPPORTED beyond).  Needs
+ * vsa_workspace_bytes() of workspace.  One kernel (after a memset of its
+ * work counters, at most 256 bytes): the cube means go through the
+ * workspace, the nt x nt scores only through shared memory. */
 vsa_status vsa_select_blocks(const vsa_bf16* q, const vsa_bf16* k, int B, int heads,
                              int head_dim, int T, int H, int W, int tt, int th, int tw,
                              int topk, int32_t* block_idx, void* workspace,
