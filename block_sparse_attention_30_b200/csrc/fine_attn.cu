@@ -99,6 +99,7 @@ struct FineBars {
     uint64_t k_full[FineCfg<D, Q8>::NK], k_empty[FineCfg<D, Q8>::NK];
     uint64_t v_full[FineCfg<D, Q8>::NV], v_empty[FineCfg<D, Q8>::NV];
     uint64_t s_full[2], p_full[2], o_ready[2];   // per S / O buffer (pair parity)
+    uint64_t vc_full[2], v_half;                 // one V stage: per-cube halves (see the V producer)
     uint64_t mma_done, lin_full, lin_ready, lin_done;
     uint32_t tmem_base;
     int abort;
@@ -158,6 +159,7 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         mbar_init(&bars->q_full, 1);
         for (int s = 0; s < C::NK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
         for (int s = 0; s < C::NV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
+        mbar_init(&bars->vc_full[0], 1); mbar_init(&bars->vc_full[1], 1); mbar_init(&bars->v_half, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(&bars->s_full[x], 1);
             mbar_init(&bars->p_full[x], 128);
@@ -200,6 +202,12 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
             uint8_t* ring = is_k ? sK : sV;
             const CUtensorMap* map = is_k ? &mk : &mv;
+            // With one V stage the two cubes of a pair have a barrier each
+            // (vc_full): cube 0 of pair p is loaded as soon as P V of pair
+            // p - 1 has read its cube 0 (v_half), cube 1 once all of that
+            // P V is done (o_ready), so the stage refills in two halves.
+            const bool vsplit = C::V_ON_O && !is_k;
+            int last_half[2] = {-1, -1};                // pair of the last load into each half
             int jn[2] = {__ldg(my_idx), topk > 1 ? __ldg(my_idx + 1) : 0};
             for (int p = 0; p < n_pairs; ++p) {
                 const int ntl = min(2, topk - 2 * p);
@@ -210,6 +218,26 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 }
                 for (int t = 0; t < ntl; ++t)
                     if (jt[t] < 0 || jt[t] >= g.nt) { if (is_k) report(status, kStatusBadIndex); jt[t] = 0; }
+                if (vsplit) {
+                    bool ok_v = true;
+                    for (int t = 0; t < ntl && ok_v; ++t) {
+                        if (p >= 1) {
+                            ok_v = t == 0 ? mbar_wait(&bars->v_half, (p - 1) & 1, abort_flag)
+                                          : mbar_wait(&bars->o_ready[(p - 1) & 1], ((p - 1) >> 1) & 1, abort_flag);
+                            if (!ok_v) break;
+                        }
+                        const TileCoord kc = tile_coord(g, jt[t]);
+                        VSA_DEBUG_CHECK(kc.t0 < g.T && kc.h0 < g.H && kc.w0 < g.W, status, kStatusBadCoord);
+                        mbar_arrive_expect_tx(&bars->vc_full[t], C::V_CUBE_BYTES);
+                        for (int c = 0; c < C::NCH; ++c)
+                            tma_load_5d(ring + c * C::CHUNK_STRIDE + t * 8192, map, &bars->vc_full[t],
+                                        head * D + 64 * c, kc.w0, kc.h0, kc.t0, b);
+                        last_half[t] = p;
+                    }
+                    if (!ok_v) { fail(); break; }
+                    ++issued;
+                    continue;
+                }
                 const int st = p % nst;
                 if (p >= nst) {
                     uint64_t* bar = &empty[st];
@@ -257,8 +285,13 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             if (*abort_flag) {
                 // drain: the last load issued into each stage must land before exit
                 if (is_k) wait_noabort(&bars->q_full, 0);
-                for (int n = max(0, issued - nst); n < issued; ++n)
-                    wait_noabort(&full[n % nst], (n / nst) & 1);
+                if (vsplit) {
+                    for (int t = 0; t < 2; ++t)
+                        if (last_half[t] >= 0) wait_noabort(&bars->vc_full[t], last_half[t] & 1);
+                } else {
+                    for (int n = max(0, issued - nst); n < issued; ++n)
+                        wait_noabort(&full[n % nst], (n / nst) & 1);
+                }
                 if (lin_issued) wait_noabort(&bars->lin_full, 0);
             }
         }
@@ -307,11 +340,26 @@ fine_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 const int nkeys = min(2, topk - 2 * p) * 64;
                 const int sv = p % C::NV, x = p & 1;
                 if (!mbar_wait(&bars->p_full[x], (p >> 1) & 1, abort_flag)) { ok = false; break; }
-                if (!mbar_wait(&bars->v_full[sv], (p / C::NV) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                for (int kk = 0; kk < nkeys / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(v_addr + sv * C::V_PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
-                    mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
+                if constexpr (C::V_ON_O) {
+                    // one V stage in two cube halves: the first 64 keys as soon
+                    // as cube 0 landed, then release that half (v_half)
+                    for (int t = 0; t < nkeys / 64; ++t) {
+                        if (!mbar_wait(&bars->vc_full[t], p & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int kk = 4 * t; kk < 4 * t + 4; ++kk) {
+                            const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, C::CHUNK_STRIDE, 1024);
+                            mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
+                        }
+                        if (t == 0) mma_commit(&bars->v_half);
+                    }
+                    if (!ok) break;
+                } else {
+                    if (!mbar_wait(&bars->v_full[sv], (p / C::NV) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 0; kk < nkeys / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(v_addr + sv * C::V_PAIR_BYTES + kk * 2048, C::CHUNK_STRIDE, 1024);
+                        mma_bf16_ts(tO(x), tS(x) + kk * 8, bd, id_pv, (p >= 2 || kk > 0));
+                    }
                 }
                 mma_commit(&bars->o_ready[x]);
                 if (!C::V_ON_O) mma_commit(&bars->v_empty[sv]);
