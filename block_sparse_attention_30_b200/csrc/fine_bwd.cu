@@ -339,26 +339,33 @@ __device__ __forceinline__ void dq_body(const CUtensorMap& mq, const CUtensorMap
             const uint32_t q_addr = smem_u32(sQ), g_addr = smem_u32(sG);
             const uint32_t tAcc = tbase + C::ACC_COL;
             auto sbuf = [&](int x) { return tbase + C::S_COL + 64 * x; };
-            auto issue_s = [&](int t) -> bool {
-                const int x = t & 1, xk = t % C::NK;
-                if (!mbar_wait(&bars->x_full[xk], (t / C::NK) & 1, abort_flag) ||
-                    !mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                issue_s_dp<D>(sbuf(x), q_addr, smem_u32(sK + xk * C::CUBE_BYTES), g_addr,
-                              smem_u32(sV + x * C::CUBE_BYTES));
-                mma_commit(&bars->s_full[x]);
-                mma_commit(&bars->y_empty[x]);             // V cube read by dP only
-                return true;
-            };
-            // S of step t+2 is issued right after dQ of step t (the last reader of its buffer)
-            bool ok = mbar_wait(&bars->a_full, 0, abort_flag) && issue_s(0) && (topk < 2 || issue_s(1));
-            for (int t = 0; ok && t < topk; ++t) {
-                const int x = t & 1;
-                if (!mbar_wait(&bars->ds_full[x], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                issue_acc<D>(tAcc, sbuf(x), smem_u32(sK + (t % C::NK) * C::CUBE_BYTES), t > 0);   // dQ += dS K
-                mma_commit(&bars->x_empty[t % C::NK]);
-                if (t + 2 < topk && !issue_s(t + 2)) { ok = false; break; }
+            // Two streams of MMAs, issued as their inputs arrive: S/dP of step
+            // s (its K and V cubes loaded; S buffer s % 2 free once dQ of step
+            // s - 2 is issued, as MMAs run in issue order) and dQ of step a
+            // (its dS written).
+            int s = 0, a = 0;
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
+            unsigned long long t0 = clock64();
+            while (ok && a < topk) {
+                if (s < topk && s <= a + 1 && mbar_test_wait(&bars->x_full[s % C::NK], (s / C::NK) & 1) &&
+                    mbar_test_wait(&bars->y_full[s & 1], (s >> 1) & 1)) {
+                    const int x = s & 1, xk = s % C::NK;
+                    tc_fence_after();
+                    issue_s_dp<D>(sbuf(x), q_addr, smem_u32(sK + xk * C::CUBE_BYTES), g_addr,
+                                  smem_u32(sV + x * C::CUBE_BYTES));
+                    mma_commit(&bars->s_full[x]);
+                    mma_commit(&bars->y_empty[x]);         // V cube read by dP only
+                    ++s;
+                    t0 = clock64();
+                } else if (a < s && mbar_test_wait(&bars->ds_full[a & 1], (a >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_acc<D>(tAcc, sbuf(a & 1), smem_u32(sK + (a % C::NK) * C::CUBE_BYTES), a > 0);   // dQ += dS K
+                    mma_commit(&bars->x_empty[a % C::NK]);
+                    ++a;
+                    t0 = clock64();
+                } else if (*abort_flag || clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) {
+                    ok = false;
+                }
             }
             if (!ok) fail();
             mma_commit(&bars->mma_done);
@@ -503,27 +510,39 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap& mq, const CUtensorM
             const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
             const uint32_t tdV = tbase + C::ACC_COL, tdK = tbase + C::ACC_COL + (16u << 16);
             auto sbuf = [&](int x) { return tbase + C::S_COL + 64 * x; };
-            auto issue_s = [&](int t) -> bool {
-                const int x = t & 1;
-                if (!mbar_wait(&bars->x_full[x], (t >> 1) & 1, abort_flag) ||
-                    !mbar_wait(&bars->y_full[x], (t >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                // S^T = K Q^T (lanes 0-15), dP^T = V dO^T (lanes 16-31)
-                issue_s_dp<D>(sbuf(x), k_addr, smem_u32(sQ + x * C::CUBE_BYTES), v_addr,
-                              smem_u32(sG + x * C::CUBE_BYTES));
-                mma_commit(&bars->s_full[x]);
-                return true;
-            };
-            bool ok = mbar_wait(&bars->a_full, 0, abort_flag) && (nq < 1 || issue_s(0)) && (nq < 2 || issue_s(1));
-            for (int t = 0; ok && t < nq; ++t) {
-                const int x = t & 1;
-                if (!mbar_wait(&bars->ds_full[x], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                issue_acc<D>(tdV, sbuf(x), smem_u32(sG + x * C::CUBE_BYTES), t > 0);                   // dV += P^T dO
-                issue_acc<D>(tdK, sbuf(x) + (16u << 16), smem_u32(sQ + x * C::CUBE_BYTES), t > 0);     // dK += dS^T Q
-                mma_commit(&bars->x_empty[x]);
-                mma_commit(&bars->y_empty[x]);
-                if (t + 2 < nq && !issue_s(t + 2)) { ok = false; break; }
+            // Two streams of MMAs, issued as their inputs arrive: S/dP of step
+            // s (its Q and dO cubes loaded; S buffer s % 2 free once the dV/dK
+            // MMAs of step s - 2 are issued, as MMAs run in issue order) and
+            // dV/dK of step a (its P / dS written).  The Q and dO slots of
+            // step s + 2 are refilled only when dV/dK of step s complete, so a
+            // fixed order (dV/dK of t, then S of t + 2) would hold dV/dK of
+            // t + 1 behind that refill; here they go first when ready.
+            int s = 0, a = 0;
+            bool ok = mbar_wait(&bars->a_full, 0, abort_flag);
+            unsigned long long t0 = clock64();
+            while (ok && a < nq) {
+                if (s < nq && s <= a + 1 && mbar_test_wait(&bars->x_full[s & 1], (s >> 1) & 1) &&
+                    mbar_test_wait(&bars->y_full[s & 1], (s >> 1) & 1)) {
+                    const int x = s & 1;
+                    tc_fence_after();
+                    // S^T = K Q^T (lanes 0-15), dP^T = V dO^T (lanes 16-31)
+                    issue_s_dp<D>(sbuf(x), k_addr, smem_u32(sQ + x * C::CUBE_BYTES), v_addr,
+                                  smem_u32(sG + x * C::CUBE_BYTES));
+                    mma_commit(&bars->s_full[x]);
+                    ++s;
+                    t0 = clock64();
+                } else if (a < s && mbar_test_wait(&bars->ds_full[a & 1], (a >> 1) & 1)) {
+                    const int x = a & 1;
+                    tc_fence_after();
+                    issue_acc<D>(tdV, sbuf(x), smem_u32(sG + x * C::CUBE_BYTES), a > 0);                   // dV += P^T dO
+                    issue_acc<D>(tdK, sbuf(x) + (16u << 16), smem_u32(sQ + x * C::CUBE_BYTES), a > 0);     // dK += dS^T Q
+                    mma_commit(&bars->x_empty[x]);
+                    mma_commit(&bars->y_empty[x]);
+                    ++a;
+                    t0 = clock64();
+                } else if (*abort_flag || clock64() - t0 > VSA_WAIT_LIMIT_CYCLES) {
+                    ok = false;
+                }
             }
             if (!ok) fail();
             mma_commit(&bars->mma_done);
