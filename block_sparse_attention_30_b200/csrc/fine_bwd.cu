@@ -10,9 +10,9 @@
 //
 // Kernels:
 //   delta_kernel   D per cube slot, fp32 (0 for padded slots).
-//   csr_*          the transpose of the block index: for every key cube the
-//                  ascending list of query cubes that kept it (deterministic;
-//                  one warp per key cube).
+//   csr_bitmap_kernel  the transpose of the block index: for every key cube
+//                  the ascending list of query cubes that kept it
+//                  (deterministic; a shared-memory bitmap per (b, head)).
 //   dq_body        one CTA per query cube: per kept key cube, S = Q K^T
 //                  (TMEM lanes 0-15) and dP = dO V^T (lanes 16-31 of the same
 //                  columns) on the tensor cores, dS written as bf16 over S by
@@ -27,6 +27,8 @@
 // Both run in one launch (bwd_kernel: even CTAs dQ, odd CTAs dK/dV).  One
 // K/Q tile serves as the K-major operand of one product and the MN-major
 // operand of the other, as V does in the forward.  Every wait is bounded.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -89,79 +91,79 @@ delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout
 }
 
 // ---------------------------------------------------------------- transpose
-// One warp per (b*heads, key cube j): count (pass 0) or list (pass 1) the
-// query cubes i whose ascending block-index row contains j.  The lanes test
-// 32 consecutive i at a time; a ballot keeps the list in increasing i, so the
-// result is deterministic.
-__device__ __forceinline__ bool row_has(const int32_t* row, int k, int j) {
-    int lo = 0, hi = k - 1;
-    while (lo <= hi) {
-        const int mid = (lo + hi) >> 1;
-        const int x = __ldg(row + mid);
-        if (x == j) return true;
-        if (x < j) lo = mid + 1; else hi = mid - 1;
-    }
-    return false;
-}
+// The transpose of the block index, one CTA per (b, head): bit (j, i) of a
+// shared-memory bitmap is set when query cube i kept key cube j, for key
+// cubes j0 .. j0 + chunk - 1 at a time (the head's index rows are read once
+// per chunk); the set bits of row j in ascending i are key cube j's list
+// (deterministic, and a cube listed twice in one row counts once), off[j + 1]
+// the running count.  Entries outside 0 .. nt-1 are skipped (the dQ body
+// reports them).  chunk <= kCsrThreads: one thread per bitmap row for the
+// counts and the writes.
+constexpr int kCsrThreads = 512;
 
-__global__ void __launch_bounds__(256)
-csr_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, const int pass,
-           int32_t* __restrict__ off, int32_t* __restrict__ entries) {
-    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const long long bhs = (long long)g.B * g.heads;
-    if (wid >= bhs * g.nt) return;                    // whole warp
-    const long long bh = wid / g.nt;
-    const int j = (int)(wid % g.nt);
+__global__ void __launch_bounds__(kCsrThreads)
+csr_bitmap_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, const int chunk,
+                  int32_t* __restrict__ off, int32_t* __restrict__ entries) {
+    extern __shared__ uint32_t bm[];                 // [chunk][words]
+    __shared__ int32_t wsum[kCsrThreads / 32];
+    __shared__ int32_t carry;
+    const int words = (g.nt + 31) / 32;
+    const long long bh = blockIdx.x;
     const int32_t* rows = idx + bh * g.nt * k;
     int32_t* o = off + bh * (g.nt + 1);
     int32_t* e = entries + bh * g.nt * k;
-    int base = pass == 0 ? 0 : o[j];
-    const unsigned lt = (1u << lane) - 1u;
-    for (int i0 = 0; i0 < g.nt; i0 += 32) {
-        const int i = i0 + lane;
-        const bool has = i < g.nt && row_has(rows + (long long)i * k, k, j);
-        const unsigned ball = __ballot_sync(0xffffffffu, has);
-        if (pass == 1 && has) e[base + __popc(ball & lt)] = i;
-        base += __popc(ball);
-    }
-    if (pass == 0 && lane == 0) o[j + 1] = base;      // counts; scanned by csr_scan_kernel
-}
-
-// One CTA per b*heads: off[0] = 0, off[j+1] = sum of the counts up to j.
-__global__ void __launch_bounds__(1024)
-csr_scan_kernel(const Grid g, int32_t* __restrict__ off) {
-    __shared__ int32_t carry;
-    int32_t* o = off + (long long)blockIdx.x * (g.nt + 1);
-    if (threadIdx.x == 0) { carry = 0; o[0] = 0; }
-    __syncthreads();
-    for (int base = 0; base < g.nt; base += blockDim.x) {
-        const int j = base + threadIdx.x;
-        int v = j < g.nt ? o[j + 1] : 0;
-        // inclusive scan of this block of counts
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-        __shared__ int32_t wsum[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long total = (long long)g.nt * k;
+    if (tid == 0) { carry = 0; o[0] = 0; }
+    for (int j0 = 0; j0 < g.nt; j0 += chunk) {
+        const int nj = min(chunk, g.nt - j0);
+        for (int w = tid; w < nj * words; w += kCsrThreads) bm[w] = 0u;
+        __syncthreads();
+#pragma unroll 4
+        for (long long t = tid; t < total; t += kCsrThreads) {
+            const int j = __ldg(rows + t);
+            if (j >= j0 && j < j0 + nj) {
+                const int i = (int)(t / k);
+                atomicOr(&bm[(j - j0) * words + (i >> 5)], 1u << (i & 31));
+            }
+        }
+        __syncthreads();
+        // row tid: its count, then an exclusive scan over the chunk's rows
+        int cnt = 0;
+        if (tid < nj)
+            for (int w = 0; w < words; ++w) cnt += __popc(bm[tid * words + w]);
+        int incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, v, d);
-            if (lane >= d) v += y;
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
         }
-        if (lane == 31) wsum[warp] = v;
+        if (lane == 31) wsum[warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            int w = wsum[lane];
+            int w = lane < kCsrThreads / 32 ? wsum[lane] : 0;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, w, d);
                 if (lane >= d) w += y;
             }
-            wsum[lane] = w;
+            if (lane < kCsrThreads / 32) wsum[lane] = w;
         }
         __syncthreads();
-        const int incl = v + (warp > 0 ? wsum[warp - 1] : 0) + carry;
-        if (j < g.nt) o[j + 1] = incl;
+        const int base = carry + (warp > 0 ? wsum[warp - 1] : 0) + incl - cnt;
+        if (tid < nj) {
+            o[j0 + tid + 1] = base + cnt;
+            int n = base;
+            for (int w = 0; w < words; ++w) {
+                uint32_t bits = bm[tid * words + w];
+                while (bits) {
+                    e[n++] = 32 * w + __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                }
+            }
+        }
         __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = incl;
+        if (tid == 0) carry += wsum[kCsrThreads / 32 - 1];
         __syncthreads();
     }
 }
@@ -670,12 +672,12 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     delta_kernel<<<(unsigned)rows, 256, 0, stream>>>(                 // 8 warps x 8 slots per cube
         a.out32, static_cast<const __nv_bfloat16*>(a.dout), g, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const long long keys = (long long)g.B * g.heads * g.nt;     // one warp each
-    csr_kernel<<<(unsigned)((keys + 7) / 8), 256, 0, stream>>>(a.block_idx, g, a.topk, 0, off, ents);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    csr_scan_kernel<<<(unsigned)(g.B * g.heads), 1024, 0, stream>>>(g, off);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    csr_kernel<<<(unsigned)((keys + 7) / 8), 256, 0, stream>>>(a.block_idx, g, a.topk, 1, off, ents);
+    // bitmap rows of (nt + 31) / 32 words, in at most 40 KB of dynamic shared
+    // memory (below the default limit without an opt-in)
+    const int words = (g.nt + 31) / 32;
+    const int chunk = std::max(1, std::min(std::min(kCsrThreads, g.nt), (40 * 1024) / (4 * words)));
+    csr_bitmap_kernel<<<(unsigned)(g.B * g.heads), kCsrThreads, (size_t)chunk * words * 4, stream>>>(
+        a.block_idx, g, a.topk, chunk, off, ents);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_kernel<D><<<(unsigned)(2 * rows), 224, SMEM, stream>>>(
         *a.mq, *a.mk, *a.mv, *a.mg, g, a.block_idx, a.topk, scale_log2, ragged, off, ents, a.lse, delta,
