@@ -170,8 +170,9 @@ csr_bitmap_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, co
 
 // ---------------------------------------------------------- shared layout
 // Both bodies walk single cubes (64 keys or 64 queries per step) so that the
-// streamed cubes get two ring slots and S two TMEM buffers within the
-// budget of two CTAs per SM; step t uses ring slot t % 2 and S buffer t % 2.
+// streamed cubes get two ring slots (three for the dQ body's K cubes) and S
+// two TMEM buffers within the budget of two CTAs per SM; step t uses S
+// buffer t % 2 and ring slot t mod the ring's depth.
 template <int D>
 struct BwdCfg {
     static constexpr int NCH = D / 64;
