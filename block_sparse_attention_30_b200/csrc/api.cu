@@ -281,6 +281,7 @@ vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_b
     if (s != VSA_OK) return s;
     const vsa::Grid g = grid_of(B, heads, head_dim, T, H, W, tt, th, tw);
     if (topk < 1 || topk > g.nt) return VSA_ERR_INVALID_ARGUMENT;
+    if (!vsa::bwd_supported(g)) return VSA_ERR_UNSUPPORTED;
     for (const void* p : {(const void*)q, (const void*)k, (const void*)v, (const void*)out_f32,
                           (const void*)dout, (const void*)block_idx, (const void*)lse, (const void*)dq,
                           (const void*)dk, (const void*)dv})

@@ -100,6 +100,7 @@ delta_kernel(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout
 // reports them).  chunk <= kCsrThreads: one thread per bitmap row for the
 // counts and the writes.
 constexpr int kCsrThreads = 512;
+constexpr int kCsrSmemBytes = 40 * 1024;             // dynamic shared memory, below the default limit
 
 __global__ void __launch_bounds__(kCsrThreads)
 csr_bitmap_kernel(const int32_t* __restrict__ idx, const Grid g, const int k, const int chunk,
@@ -644,6 +645,8 @@ size_t bwd_scratch_bytes(const Grid& g, int topk) {
     return up(delta) + up(offs) + up(ents);
 }
 
+bool bwd_supported(const Grid& g) { return 4ll * ((g.nt + 31) / 32) <= kCsrSmemBytes; }   // nt <= 327680
+
 template <int D>
 static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     using C = BwdCfg<D>;
@@ -667,16 +670,17 @@ static cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t stream) {
     int32_t* ents = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(off) +
                                                up((size_t)g.B * g.heads * (g.nt + 1) * sizeof(int32_t)));
     if (2 * rows > 0x7fffffffll) return cudaErrorInvalidConfiguration;   // a dQ and a dK/dV CTA per cube
+    if (!bwd_supported(g)) return cudaErrorInvalidConfiguration;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const int ragged = (g.T % g.tt) || (g.H % g.th) || (g.W % g.tw);
 
     delta_kernel<<<(unsigned)rows, 256, 0, stream>>>(                 // 8 warps x 8 slots per cube
         a.out32, static_cast<const __nv_bfloat16*>(a.dout), g, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // bitmap rows of (nt + 31) / 32 words, in at most 40 KB of dynamic shared
-    // memory (below the default limit without an opt-in)
+    // bitmap rows of (nt + 31) / 32 words, in at most kCsrSmemBytes of dynamic
+    // shared memory (one row at least: bwd_supported)
     const int words = (g.nt + 31) / 32;
-    const int chunk = std::max(1, std::min(std::min(kCsrThreads, g.nt), (40 * 1024) / (4 * words)));
+    const int chunk = std::max(1, std::min(std::min(kCsrThreads, g.nt), kCsrSmemBytes / (4 * words)));
     csr_bitmap_kernel<<<(unsigned)(g.B * g.heads), kCsrThreads, (size_t)chunk * words * 4, stream>>>(
         a.block_idx, g, a.topk, chunk, off, ents);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -28,6 +28,7 @@ struct BwdArgs {
 };
 
 size_t bwd_scratch_bytes(const Grid& g, int topk);
+bool bwd_supported(const Grid& g);   // one row of the transpose's bitmap fits its shared memory
 cudaError_t launch_fine_bwd(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace vsa

@@ -190,7 +190,9 @@ vsa_status vsa_sparse_attn_fwd_train(const vsa_bf16* q, const vsa_bf16* k, const
  * P recomputed from lse, products on the tensor cores with fp32
  * accumulation.  Uses the workspace scratch (vsa_workspace_bytes()) for the
  * row terms and the transpose of block_idx, so it overwrites an earlier
- * selection's scratch on the same workspace (not block_idx). */
+ * selection's scratch on the same workspace (not block_idx).  The transpose
+ * keeps one bitmap row of nt bits in shared memory: nt <= 327680, else
+ * VSA_ERR_UNSUPPORTED before any launch. */
 vsa_status vsa_sparse_attn_bwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                                const float* out_f32, const vsa_bf16* dout, const int32_t* block_idx,
                                const float* lse, vsa_bf16* dq, vsa_bf16* dk, vsa_bf16* dv, int B,

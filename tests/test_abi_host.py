@@ -161,6 +161,12 @@ def test_other_entry_points_validate(L):
     assert bw(*[FAKE] * 10, *SHAPE, 2, FAKE, need - 16, None) == WORKSPACE
     assert bw(*[FAKE] * 7, FAKE + 8, FAKE, FAKE, *SHAPE, 2, FAKE, need, None) == INVALID      # dq
     assert bw(*[FAKE] * 10, *SHAPE, 0, FAKE, need, None) == INVALID                           # topk < 1
+    # the transpose of the block index keeps one bitmap row of nt bits in
+    # shared memory: 327680 cubes fit, 327681 do not (refused before any launch)
+    edge = [1, 1, 128, 4, 4, 4 * 327680, 4, 4, 4]
+    over = [1, 1, 128, 4, 4, 4 * 327681, 4, 4, 4]
+    assert bw(*[FAKE] * 10, *edge, 2, FAKE, 16, None) == WORKSPACE                            # passes the limit
+    assert bw(*[FAKE] * 10, *over, 2, FAKE, 1 << 40, None) == UNSUPPORTED
     assert L.vsa_workspace_init(None, 1024, None) == INVALID
     assert L.vsa_workspace_init(FAKE, 8, None) == WORKSPACE
     assert L.vsa_device_status(None, None) == INVALID
